@@ -1,0 +1,194 @@
+"""Seeded synthetic inputs for the MoE dispatch/combine workloads.
+
+This module only draws inputs: hidden rows, routing (top-k expert ids) and
+top-k weights.  It holds none of the dispatch/combine arithmetic, and it is
+the one module that both the CUDA side (tests, benchmark) and the CPU oracle
+side take their inputs from.
+
+Generator: numpy PCG64 streams, one per (workload seed, rank, stream kind),
+built from ``numpy.random.SeedSequence([seed, rank, kind])``.
+
+Workloads (shapes of DeepSeek-V3-style expert routing; all synthetic):
+
+=========  ==  ===  =====  =====  ==  ==========================================
+name        R    E      T      H   K  routing
+=========  ==  ===  =====  =====  ==  ==========================================
+tiny        2    8     64    256   2  K distinct experts, uniform
+dsv3        8  256   4096   7168   8  K distinct uniform, each slot -1 w.p. 0.02
+ll         16  256    128   7168   8  K distinct uniform; Tmax = 128
+zipf       32  256   8192   7168   8  K without replacement, Zipf(s=1.2)
+                                       popularity over a seeded permutation
+reuse       8  256   4096   4096   8  4 distinct ranks per token, then K
+                                       distinct experts among their 4*32
+=========  ==  ===  =====  =====  ==  ==========================================
+
+Hidden rows are N(0, 1) drawn in fp32 and rounded to bf16 (round to nearest
+even).  Weights are a softmax (computed in fp64, stored fp32) of N(0, 1)
+logits over the K slots; masked slots keep their weight.
+"""
+from __future__ import annotations
+
+import concurrent.futures as _cf
+import dataclasses
+
+import numpy as np
+
+SEED_BASE = 0xE9000
+
+_KIND_ROUTING = 1
+_KIND_MASK = 2
+_KIND_WEIGHTS = 3
+_KIND_X = 4
+_KIND_Y = 5
+_KIND_BIAS = 6
+_KIND_PERM = 7
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    num_ranks: int          # R
+    num_experts: int        # E
+    num_tokens: int         # T (per rank)
+    hidden: int             # H
+    topk: int               # K
+    routing: str            # uniform | uniform_masked | zipf | group_limited
+    seed: int
+    num_channels: int = 10  # C
+    max_tokens_per_rank: int = 0   # Tmax for the low-latency path (0 -> T)
+    mask_prob: float = 0.0
+    zipf_s: float = 1.2
+    group_ranks: int = 4
+
+    @property
+    def local_experts(self) -> int:
+        return self.num_experts // self.num_ranks
+
+    @property
+    def tmax(self) -> int:
+        return self.max_tokens_per_rank or self.num_tokens
+
+    def scaled(self, num_tokens: int | None = None, hidden: int | None = None,
+               name: str | None = None) -> "Workload":
+        return dataclasses.replace(
+            self,
+            num_tokens=self.num_tokens if num_tokens is None else num_tokens,
+            hidden=self.hidden if hidden is None else hidden,
+            max_tokens_per_rank=0 if num_tokens is not None else self.max_tokens_per_rank,
+            name=name or f"{self.name}-T{num_tokens or self.num_tokens}-H{hidden or self.hidden}")
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", 2, 8, 64, 256, 2, "uniform", SEED_BASE + 0),
+    "dsv3": Workload("dsv3", 8, 256, 4096, 7168, 8, "uniform_masked", SEED_BASE + 1,
+                     mask_prob=0.02),
+    "ll": Workload("ll", 16, 256, 128, 7168, 8, "uniform", SEED_BASE + 2,
+                   max_tokens_per_rank=128),
+    "zipf": Workload("zipf", 32, 256, 8192, 7168, 8, "zipf", SEED_BASE + 3),
+    "reuse": Workload("reuse", 8, 256, 4096, 4096, 8, "group_limited", SEED_BASE + 4),
+}
+
+
+def _rng(seed: int, rank: int, kind: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, rank, kind])))
+
+
+def _distinct_uniform(rng, T, n, K):
+    """K distinct values of range(n) per row, uniformly at random, in draw order."""
+    keys = rng.random((T, n))
+    return np.argsort(keys, axis=1, kind="stable")[:, :K]
+
+
+def _zipf_weights(E, s):
+    ranks = np.arange(1, E + 1, dtype=np.float64)
+    p = ranks ** (-s)
+    return p / p.sum()
+
+
+def topk_idx(w: Workload) -> np.ndarray:
+    """[R, T, K] int64 expert ids (-1 = unused slot)."""
+    R, E, T, K = w.num_ranks, w.num_experts, w.num_tokens, w.topk
+    out = np.empty((R, T, K), np.int64)
+    if w.routing == "zipf":
+        perm = _rng(w.seed, 0, _KIND_PERM).permutation(E)
+        p = _zipf_weights(E, w.zipf_s)
+        logp = np.empty(E)
+        logp[perm] = np.log(p)          # expert perm[i] has popularity rank i+1
+    for s in range(R):
+        rng = _rng(w.seed, s, _KIND_ROUTING)
+        if w.routing in ("uniform", "uniform_masked"):
+            out[s] = _distinct_uniform(rng, T, E, K)
+        elif w.routing == "zipf":
+            # Sequential draws without replacement, each proportional to the
+            # remaining popularity mass, are the top-K of log p + Gumbel noise.
+            g = -np.log(-np.log(rng.random((T, E))))
+            out[s] = np.argsort(-(logp[None, :] + g), axis=1, kind="stable")[:, :K]
+        elif w.routing == "group_limited":
+            L = w.local_experts
+            ranks = _distinct_uniform(rng, T, w.num_ranks, w.group_ranks)          # [T, G]
+            cand = (ranks[:, :, None] * L + np.arange(L)[None, None, :]).reshape(T, -1)
+            pick = _distinct_uniform(rng, T, cand.shape[1], K)
+            out[s] = np.take_along_axis(cand, pick, axis=1)
+        else:
+            raise ValueError(w.routing)
+        if w.mask_prob > 0:
+            m = _rng(w.seed, s, _KIND_MASK).random((T, K)) < w.mask_prob
+            out[s][m] = -1
+    return out
+
+
+def topk_weights(w: Workload) -> np.ndarray:
+    """[R, T, K] float32 softmax weights."""
+    R, T, K = w.num_ranks, w.num_tokens, w.topk
+    out = np.empty((R, T, K), np.float32)
+    for s in range(R):
+        logits = _rng(w.seed, s, _KIND_WEIGHTS).standard_normal((T, K))
+        z = np.exp(logits - logits.max(axis=1, keepdims=True))
+        out[s] = (z / z.sum(axis=1, keepdims=True)).astype(np.float32)
+    return out
+
+
+def _normal_bf16_rows(seed, kind, shape_per_rank, num_parts, torch_out):
+    """Fill torch_out[part] (bf16) with N(0,1) fp32 draws rounded to bf16."""
+    import torch
+
+    def one(part):
+        a = _rng(seed, part, kind).standard_normal(shape_per_rank, dtype=np.float32)
+        torch_out[part].copy_(torch.from_numpy(a).to(torch.bfloat16))
+
+    workers = min(8, max(1, num_parts))
+    with _cf.ThreadPoolExecutor(workers) as ex:
+        list(ex.map(one, range(num_parts)))
+    return torch_out
+
+
+def hidden_rows(w: Workload, pin_memory: bool = False):
+    """x [R, T, H] torch.bfloat16 on the CPU."""
+    import torch
+    x = torch.empty((w.num_ranks, w.num_tokens, w.hidden), dtype=torch.bfloat16,
+                    pin_memory=pin_memory)
+    return _normal_bf16_rows(w.seed, _KIND_X, (w.num_tokens, w.hidden), w.num_ranks, x)
+
+
+def expert_rows(seed: int, num_rows: int, hidden: int, chunk: int = 65536):
+    """An independent N(0,1) bf16 tensor [num_rows, H] (stand-in expert outputs)."""
+    import torch
+    y = torch.empty((num_rows, hidden), dtype=torch.bfloat16)
+    parts = (num_rows + chunk - 1) // chunk
+
+    def one(part):
+        lo, hi = part * chunk, min(num_rows, (part + 1) * chunk)
+        a = _rng(seed, part, _KIND_Y).standard_normal((hi - lo, hidden), dtype=np.float32)
+        y[lo:hi].copy_(torch.from_numpy(a).to(torch.bfloat16))
+
+    with _cf.ThreadPoolExecutor(min(8, max(1, parts))) as ex:
+        list(ex.map(one, range(parts)))
+    return y
+
+
+def bias_rows(w: Workload, which: int):
+    """bias tensor [R, T, H] bf16, N(0,1)."""
+    import torch
+    b = torch.empty((w.num_ranks, w.num_tokens, w.hidden), dtype=torch.bfloat16)
+    return _normal_bf16_rows(w.seed + 7919 * (which + 1), _KIND_BIAS,
+                             (w.num_tokens, w.hidden), w.num_ranks, b)

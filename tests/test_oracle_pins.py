@@ -1,0 +1,502 @@
+"""Pins for the CPU oracle, checked against things other than the oracle itself.
+
+* a hand-worked fixture (tests/golden/tiny_handle.txt);
+* a second, independent formulation by brute force: one global stable sort of
+  (destination, source, token) triples, pure Python, tiny inputs;
+* closed forms: identity experts make the combine return fan-out * x, the
+  low-latency combine with weights 1/8 returns (valid slots / 8) * x;
+* exact integer-valued rows, so any dropped, doubled or misplaced term shows;
+* invariants (counts, monotone prefixes, permutation inverses);
+* special cases: one rank, top-1, all slots masked, no tokens, more channels
+  than tokens;
+* the bf16 rounding step against exact rational arithmetic and against torch.
+
+All CPU, no GPU.
+"""
+import bisect
+import fractions
+import itertools
+import os
+import struct
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "tiny_handle.txt")
+
+
+# ----------------------------------------------------------------------------
+# helpers written for the tests (independent of the oracle)
+
+def bf16_to_f64(u16: np.ndarray) -> np.ndarray:
+    return (u16.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def f32_to_bf16_torch(a: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bits via torch's conversion (round to nearest even)."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def brute_handle(topk, E, C):
+    """Independent formulation: sort all (d, s, t) triples once."""
+    R, T, K = topk.shape
+    L = E // R
+    triples = []
+    for s in range(R):
+        for t in range(T):
+            dests = sorted({int(e) // L for e in topk[s, t] if e != -1})
+            for d in dests:
+                triples.append((d, s, t))
+    triples.sort()
+    N = [0] * R
+    for d, _, _ in triples:
+        N[d] += 1
+    off = [0]
+    for d in range(R):
+        off.append(off[-1] + N[d])
+    send_head = -np.ones((R, T, R), np.int64)
+    recv_src = np.zeros(len(triples), np.int64)
+    for row, (d, s, t) in enumerate(triples):
+        send_head[s, t, d] = row - off[d]
+        recv_src[row] = t
+    q = -(-T // C) if T else 0
+    start = [min(c * q, T) for c in range(C + 1)]
+    # recv_channel_prefix[d][s][c] = number of triples that sort before (d, s, start(c))
+    rcp = np.zeros((R, R, C), np.int64)
+    cp = np.zeros((R, R, C), np.int64)
+    for d in range(R):
+        for s in range(R):
+            for c in range(C):
+                rcp[d, s, c] = bisect.bisect_left(triples, (d, s, start[c])) - off[d]
+                cp[s, d, c] = sum(1 for (dd, ss, tt) in triples
+                                  if dd == d and ss == s and tt < start[c + 1])
+    rp = np.zeros((R, R), np.int64)
+    for i in range(R):
+        for d in range(R):
+            rp[i, d] = sum(1 for (dd, ss, _) in triples if dd == d and ss <= i)
+    return dict(send_head=send_head, recv_src_idx=recv_src, recv_rank_offset=np.array(off),
+                rank_prefix_matrix=rp, channel_prefix_matrix=cp,
+                recv_channel_prefix_matrix=rcp, triples=triples)
+
+
+def brute_ll(topk, E):
+    R, T, K = topk.shape
+    L = E // R
+    lists = {e: [] for e in range(E)}
+    for s in range(R):
+        for t in range(T):
+            for e in set(int(v) for v in topk[s, t] if v != -1):
+                lists[e].append((s, t))
+    for e in lists:
+        lists[e].sort()
+    return lists
+
+
+def random_topk(rng, R, E, T, K, mask_p=0.0, distinct=True):
+    out = np.empty((R, T, K), np.int64)
+    for s in range(R):
+        for t in range(T):
+            if distinct:
+                out[s, t] = rng.choice(E, size=K, replace=False)
+            else:
+                out[s, t] = rng.integers(0, E, size=K)
+    if mask_p:
+        out[rng.random(out.shape) < mask_p] = -1
+    return out
+
+
+def run_oracle_dispatch(topk, E, C, x=None, w=None):
+    ntr, nte, tin = oracle.layout(topk, E)
+    h = oracle.dispatch_handle(tin, nte, C)
+    rows = None
+    if x is not None:
+        rows = oracle.dispatch_rows(x, topk, w, h, E)
+    return ntr, nte, tin, h, rows
+
+
+# ----------------------------------------------------------------------------
+# hand-worked fixture
+
+def load_golden():
+    vals = {}
+    with open(GOLDEN) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *rest = line.split()
+            vals[key] = [int(v) for v in rest]
+    return vals
+
+
+def test_golden_layout_and_handle():
+    g = load_golden()
+    R, E, T, K, C = g["R"][0], g["E"][0], g["T"][0], g["K"][0], g["C"][0]
+    topk = np.array(g["topk_idx"], np.int64).reshape(R, T, K)
+    ntr, nte, tin = oracle.layout(topk, E)
+    assert tin.ravel().tolist() == g["is_token_in_rank"]
+    assert ntr.ravel().tolist() == g["num_tokens_per_rank"]
+    assert nte.ravel().tolist() == g["num_tokens_per_expert"]
+    h = oracle.dispatch_handle(tin, nte, C)
+    for key in ("send_head", "recv_rank_offset", "recv_src_idx", "rank_prefix_matrix",
+                "channel_prefix_matrix", "recv_channel_prefix_matrix",
+                "num_recv_tokens_per_expert"):
+        assert h[key].ravel().tolist() == g[key], key
+
+
+def test_golden_rows_and_combine():
+    g = load_golden()
+    R, E, T, K, C, H = (g[k][0] for k in ("R", "E", "T", "K", "C", "H"))
+    topk = np.array(g["topk_idx"], np.int64).reshape(R, T, K)
+    xv = np.array(g["x"], np.float32).reshape(R, T, H)
+    x = f32_to_bf16_torch(xv)
+    w = np.full((R, T, K), 0.5, np.float32)
+    _, _, _, h, (recv_x, recv_idx, recv_w) = run_oracle_dispatch(topk, E, C, x, w)
+    assert recv_idx.ravel().tolist() == g["recv_topk_idx"]
+    out, _ = oracle.combine(recv_x, h)
+    assert bf16_to_f64(out).ravel().tolist() == g["combine_identity"]
+
+
+def test_golden_ll():
+    g = load_golden()
+    R, E, T, K, H, Tmax = (g[k][0] for k in ("R", "E", "T", "K", "H", "TMAX"))
+    topk = np.array(g["topk_idx"], np.int64).reshape(R, T, K)
+    x = f32_to_bf16_torch(np.array(g["x"], np.float32).reshape(R, T, H))
+    ll = oracle.ll_dispatch(x, topk, E, Tmax)
+    assert ll["packed_recv_count"].ravel().tolist() == g["ll_count"]
+    L = E // R
+    for e in range(E):
+        n = g["ll_count"][e]
+        assert ll["src_info"][e // L, e % L, :n].tolist() == g[f"ll_src_info_e{e}"]
+    assert ll["layout_range"].ravel().tolist() == g["ll_layout_range"]
+
+
+# ----------------------------------------------------------------------------
+# brute force (independent sort-based formulation)
+
+@pytest.mark.parametrize("R,E,T,K,C,mask_p", [
+    (2, 8, 13, 2, 3, 0.0), (4, 16, 9, 3, 2, 0.1), (3, 9, 7, 4, 5, 0.3),
+    (1, 4, 6, 2, 2, 0.2), (5, 10, 4, 2, 7, 0.0), (8, 32, 11, 8, 3, 0.05),
+])
+def test_handle_matches_sort_formulation(R, E, T, K, C, mask_p):
+    rng = np.random.default_rng(R * 1000 + E * 10 + T)
+    topk = random_topk(rng, R, E, T, K, mask_p)
+    ntr, nte, tin, h, _ = run_oracle_dispatch(topk, E, C)
+    b = brute_handle(topk, E, C)
+    for key in ("send_head", "recv_src_idx", "recv_rank_offset", "rank_prefix_matrix",
+                "channel_prefix_matrix", "recv_channel_prefix_matrix"):
+        np.testing.assert_array_equal(h[key], b[key], err_msg=key)
+    # layout by brute counting
+    L = E // R
+    for s in range(R):
+        for t in range(T):
+            dests = {int(e) // L for e in topk[s, t] if e != -1}
+            assert [int(v) for v in tin[s, t]] == [int(d in dests) for d in range(R)]
+    exp_nte = np.zeros((R, E), np.int64)
+    for s, t, k in itertools.product(range(R), range(T), range(K)):
+        if topk[s, t, k] != -1:
+            exp_nte[s, topk[s, t, k]] += 1
+    np.testing.assert_array_equal(nte, exp_nte)
+    np.testing.assert_array_equal(h["num_recv_tokens_per_expert"],
+                                  exp_nte.sum(0).reshape(R, L))
+
+
+def test_dispatch_rows_and_combine_integer_rows():
+    """Rows carry exact small integers; the combine sum and every row copy are exact."""
+    rng = np.random.default_rng(7)
+    R, E, T, K, C, H = 4, 16, 10, 3, 3, 16
+    topk = random_topk(rng, R, E, T, K, mask_p=0.15)
+    w = rng.random((R, T, K)).astype(np.float32)
+    xv = rng.integers(-20, 21, size=(R, T, H)).astype(np.float32)
+    x = f32_to_bf16_torch(xv)
+    _, _, tin, h, (recv_x, recv_idx, recv_w) = run_oracle_dispatch(topk, E, C, x, w)
+    b = brute_handle(topk, E, C)
+    L = E // R
+    for row, (d, s, t) in enumerate(b["triples"]):
+        np.testing.assert_array_equal(recv_x[row], x[s, t])
+        for k in range(K):
+            e = topk[s, t, k]
+            here = e != -1 and e // L == d
+            assert recv_idx[row, k] == (e % L if here else -1)
+            assert recv_w[row, k] == (w[s, t, k] if here else 0.0)
+    # Each received row gets its own integer signature; the combine must add
+    # exactly the rows that belong to the token.
+    yv = rng.integers(-8, 9, size=recv_x.shape).astype(np.float32)
+    y = f32_to_bf16_torch(yv)
+    out, out_w = oracle.combine(y, h, recv_w)
+    exp = np.zeros((R, T, H))
+    for row, (d, s, t) in enumerate(b["triples"]):
+        exp[s, t] += yv[row]
+    np.testing.assert_array_equal(bf16_to_f64(out), exp)
+    # weights: exactly one destination owns each valid slot
+    exp_w = np.where(topk != -1, w, 0.0).astype(np.float32)
+    np.testing.assert_array_equal(out_w, exp_w)
+
+
+def test_combine_identity_experts_closed_form():
+    """y = recv_x  =>  out = bf16(fan-out * x) (exact: fan-out * x fits in fp32)."""
+    w_ = synth.WORKLOADS["dsv3"].scaled(num_tokens=40, hidden=64)
+    topk = synth.topk_idx(w_)
+    x = synth.hidden_rows(w_).view(torch.int16).numpy().view(np.uint16)
+    _, _, tin, h, (recv_x, _, _) = run_oracle_dispatch(topk, w_.num_experts, w_.num_channels, x)
+    out, _ = oracle.combine(recv_x, h)
+    fan = tin.sum(-1).astype(np.float32)
+    exp = f32_to_bf16_torch(fan[..., None] * bf16_to_f64(x).astype(np.float32))
+    np.testing.assert_array_equal(out, exp)
+
+
+def test_combine_bias_closed_form():
+    rng = np.random.default_rng(3)
+    R, E, T, K, C, H = 2, 4, 5, 2, 2, 8
+    topk = random_topk(rng, R, E, T, K)
+    b0v = rng.integers(-5, 6, (R, T, H)).astype(np.float32)
+    b1v = rng.integers(-5, 6, (R, T, H)).astype(np.float32)
+    x = f32_to_bf16_torch(np.zeros((R, T, H), np.float32))
+    _, _, _, h, (recv_x, _, _) = run_oracle_dispatch(topk, E, C, x)
+    out, _ = oracle.combine(recv_x, h, bias0=f32_to_bf16_torch(b0v), bias1=f32_to_bf16_torch(b1v))
+    np.testing.assert_array_equal(bf16_to_f64(out), b0v + b1v)
+
+
+def test_combine_token_subset_matches_full():
+    w_ = synth.WORKLOADS["tiny"]
+    topk = synth.topk_idx(w_)
+    x = synth.hidden_rows(w_).view(torch.int16).numpy().view(np.uint16)
+    _, _, _, h, (recv_x, _, recv_w) = run_oracle_dispatch(
+        topk, w_.num_experts, w_.num_channels, x, synth.topk_weights(w_))
+    full, full_w = oracle.combine(recv_x, h, recv_w)
+    toks = np.array([5, 0, 127, 64, 3])
+    part, part_w = oracle.combine(recv_x, h, recv_w, tokens=toks)
+    np.testing.assert_array_equal(part, full.reshape(-1, w_.hidden)[toks])
+    np.testing.assert_array_equal(part_w, full_w.reshape(-1, w_.topk)[toks])
+
+
+# ----------------------------------------------------------------------------
+# invariants on the synthetic workloads (small token counts)
+
+@pytest.mark.parametrize("name", ["tiny", "dsv3", "ll", "zipf", "reuse"])
+def test_layout_and_handle_invariants(name):
+    w_ = synth.WORKLOADS[name]
+    w_ = w_.scaled(num_tokens=min(w_.num_tokens, 300), hidden=8)
+    topk = synth.topk_idx(w_)
+    R, T, K = topk.shape
+    ntr, nte, tin, h, _ = run_oracle_dispatch(topk, w_.num_experts, w_.num_channels)
+    L = w_.local_experts
+    valid = topk != -1
+    np.testing.assert_array_equal(ntr.sum(1), tin.reshape(R, -1).sum(1))
+    np.testing.assert_array_equal(nte.sum(1), valid.reshape(R, -1).sum(1))
+    assert (ntr <= nte.reshape(R, R, L).sum(-1)).all()
+    rp, cp, rcp = h["rank_prefix_matrix"], h["channel_prefix_matrix"], h["recv_channel_prefix_matrix"]
+    N = h["recv_rank_offset"][1:] - h["recv_rank_offset"][:-1]
+    assert (np.diff(rp, axis=0) >= 0).all()
+    np.testing.assert_array_equal(rp[-1], N)
+    np.testing.assert_array_equal(rp[-1], ntr.sum(0))
+    assert (np.diff(cp, axis=2) >= 0).all()
+    np.testing.assert_array_equal(cp[:, :, -1], ntr)
+    assert (np.diff(rcp.reshape(R, -1), axis=1) >= 0).all()
+    # permutation inverse: recv_src_idx o send_head = token id, rows form a bijection
+    sh = h["send_head"]
+    seen = np.zeros(int(h["recv_rank_offset"][-1]), bool)
+    for d in range(R):
+        s_idx, t_idx = np.nonzero(sh[:, :, d] >= 0)
+        rows = h["recv_rank_offset"][d] + sh[s_idx, t_idx, d]
+        np.testing.assert_array_equal(h["recv_src_idx"][rows], t_idx)
+        assert not seen[rows].any()
+        seen[rows] = True
+        np.testing.assert_array_equal(sh[:, :, d] >= 0, tin[:, :, d].astype(bool))
+    assert seen.all()
+    # the first token of each non-empty (source, channel) block sits at recv_channel_prefix
+    C = w_.num_channels
+    q = -(-T // C)
+    for d in range(R):
+        for s in range(R):
+            for c in range(C):
+                lo, hi = min(c * q, T), min((c + 1) * q, T)
+                members = np.nonzero(tin[s, lo:hi, d])[0]
+                if members.size:
+                    assert sh[s, lo + members[0], d] == rcp[d, s, c]
+
+
+# ----------------------------------------------------------------------------
+# special cases
+
+def test_single_rank_is_identity_on_routed_tokens():
+    rng = np.random.default_rng(11)
+    topk = random_topk(rng, 1, 6, 20, 2, mask_p=0.4)
+    x = f32_to_bf16_torch(rng.standard_normal((1, 20, 8)).astype(np.float32))
+    _, _, tin, h, (recv_x, _, _) = run_oracle_dispatch(topk, 6, 4, x)
+    routed = np.nonzero(tin[0, :, 0])[0]
+    np.testing.assert_array_equal(h["recv_src_idx"], routed)
+    np.testing.assert_array_equal(recv_x, x[0, routed])
+
+
+def test_top1_combine_of_identity_returns_x():
+    rng = np.random.default_rng(12)
+    R, E, T, H = 4, 8, 16, 32
+    topk = random_topk(rng, R, E, T, 1, mask_p=0.2)
+    x = f32_to_bf16_torch(rng.standard_normal((R, T, H)).astype(np.float32))
+    _, _, tin, h, (recv_x, _, _) = run_oracle_dispatch(topk, E, 3, x)
+    out, _ = oracle.combine(recv_x, h)
+    routed = tin.any(-1)
+    np.testing.assert_array_equal(out[routed], x[routed])
+    assert (out[~routed] == 0).all()
+
+
+def test_all_masked_and_empty():
+    R, E, T, K, C, H = 3, 6, 5, 2, 4, 8
+    topk = -np.ones((R, T, K), np.int64)
+    x = np.ones((R, T, H), np.uint16) * 0x3f80
+    ntr, nte, tin, h, (recv_x, _, _) = run_oracle_dispatch(topk, E, C, x)
+    assert ntr.sum() == 0 and nte.sum() == 0 and tin.sum() == 0
+    assert h["recv_rank_offset"].tolist() == [0] * (R + 1)
+    assert (h["send_head"] == -1).all()
+    assert not h["rank_prefix_matrix"].any() and not h["channel_prefix_matrix"].any()
+    out, _ = oracle.combine(np.zeros((0, H), np.uint16), h)
+    assert (out == 0).all()
+    # no tokens at all
+    topk0 = np.zeros((R, 0, K), np.int64)
+    ntr, nte, tin, h, _ = run_oracle_dispatch(topk0, E, C)
+    assert h["recv_rank_offset"].tolist() == [0] * (R + 1)
+    assert not h["recv_channel_prefix_matrix"].any()
+
+
+def test_more_channels_than_tokens():
+    rng = np.random.default_rng(5)
+    topk = random_topk(rng, 2, 4, 3, 2)
+    _, _, _, h, _ = run_oracle_dispatch(topk, 4, 8)
+    b = brute_handle(topk, 4, 8)
+    np.testing.assert_array_equal(h["channel_prefix_matrix"], b["channel_prefix_matrix"])
+    np.testing.assert_array_equal(h["recv_channel_prefix_matrix"], b["recv_channel_prefix_matrix"])
+
+
+def test_bad_expert_id_is_rejected():
+    topk = np.array([[[0, 9]]], np.int64)
+    with pytest.raises(oracle.OracleError):
+        oracle.layout(topk, 4)
+    with pytest.raises(oracle.OracleError):
+        oracle.layout(np.array([[[-2, 0]]], np.int64), 4)
+
+
+# ----------------------------------------------------------------------------
+# low-latency path
+
+@pytest.mark.parametrize("R,E,T,K,Tmax,distinct", [
+    (2, 8, 12, 2, 12, True), (4, 16, 9, 4, 11, True), (3, 6, 10, 3, 10, False),
+])
+def test_ll_dispatch_matches_lists(R, E, T, K, Tmax, distinct):
+    rng = np.random.default_rng(R + E + T)
+    topk = random_topk(rng, R, E, T, K, mask_p=0.1, distinct=distinct)
+    H = 8
+    x = f32_to_bf16_torch(rng.standard_normal((R, T, H)).astype(np.float32))
+    ll = oracle.ll_dispatch(x, topk, E, Tmax)
+    lists = brute_ll(topk, E)
+    L = E // R
+    total = 0
+    for e, lst in lists.items():
+        d, j = divmod(e, L)
+        assert ll["packed_recv_count"][d, j] == len(lst)
+        total += len(lst)
+        for slot, (s, t) in enumerate(lst):
+            assert ll["src_info"][d, j, slot] == t
+            np.testing.assert_array_equal(ll["packed_recv_x"][d, j, slot], x[s, t])
+        for s in range(R):
+            begin = sum(1 for (ss, _) in lst if ss < s)
+            cnt = sum(1 for (ss, _) in lst if ss == s)
+            assert ll["layout_range"][d, j, s].tolist() == [begin, cnt]
+    assert total == sum(len({int(v) for v in topk[s, t] if v != -1})
+                        for s in range(R) for t in range(T))
+
+
+def test_ll_combine_closed_form_uniform_weights():
+    """Weights 1/8 on identity experts: out = bf16((valid slots / 8) * x), exactly."""
+    w_ = synth.WORKLOADS["ll"].scaled(num_tokens=12, hidden=32)
+    topk = synth.topk_idx(w_)
+    rng = np.random.default_rng(1)
+    topk[rng.random(topk.shape) < 0.2] = -1
+    x = synth.hidden_rows(w_).view(torch.int16).numpy().view(np.uint16)
+    ll = oracle.ll_dispatch(x, topk, w_.num_experts, w_.tmax)
+    wts = np.full(topk.shape, 0.125, np.float32)
+    out = oracle.ll_combine(ll["packed_recv_x"], topk, wts, ll["src_info"], ll["layout_range"],
+                            w_.num_experts, w_.tmax)
+    n_valid = (topk != -1).sum(-1).astype(np.float32)
+    exp = f32_to_bf16_torch(n_valid[..., None] / 8 * bf16_to_f64(x).astype(np.float32))
+    np.testing.assert_array_equal(out, exp)
+
+
+def test_ll_combine_integer_rows_weighted():
+    """Per-slot integer rows and power-of-two weights: every term is exact."""
+    rng = np.random.default_rng(21)
+    R, E, T, K, H = 3, 12, 7, 3, 4
+    topk = random_topk(rng, R, E, T, K, mask_p=0.2)
+    ll = oracle.ll_dispatch(None, topk, E, T, with_rows=False)
+    L = E // R
+    cap = R * T
+    yv = rng.integers(-6, 7, size=(R, L, cap, H)).astype(np.float32)
+    y = f32_to_bf16_torch(yv)
+    wts = (2.0 ** rng.integers(-3, 2, size=topk.shape)).astype(np.float32)
+    out = oracle.ll_combine(y, topk, wts, ll["src_info"], ll["layout_range"], E, T)
+    lists = brute_ll(topk, E)
+    exp = np.zeros((R, T, H))
+    for s in range(R):
+        for t in range(T):
+            for k in range(K):
+                e = int(topk[s, t, k])
+                if e == -1:
+                    continue
+                slot = lists[e].index((s, t))
+                exp[s, t] += float(wts[s, t, k]) * yv[e // L, e % L, slot]
+    np.testing.assert_array_equal(bf16_to_f64(out), exp)
+
+
+# ----------------------------------------------------------------------------
+# bf16 rounding
+
+def _exact_nearest_bf16(v: float) -> float:
+    """Nearest bf16 by exact rational comparison of the two bracketing values."""
+    if v == 0:
+        return v
+    f = fractions.Fraction(v)
+    a = abs(f)
+    e = 0
+    while a >= 2:
+        a /= 2
+        e += 1
+    while a < 1:
+        a *= 2
+        e -= 1
+    q = fractions.Fraction(2) ** max(e - 7, -133)        # spacing of bf16 values here
+    lo = (abs(f) // q) * q
+    hi = lo + q
+    dlo, dhi = abs(f) - lo, hi - abs(f)
+    if dlo < dhi:
+        r = lo
+    elif dhi < dlo:
+        r = hi
+    else:
+        r = lo if (lo / q) % 2 == 0 else hi
+    r = float(r)
+    return -r if v < 0 else r
+
+
+def test_round_bf16_against_exact_and_torch():
+    rng = np.random.default_rng(0)
+    f32 = rng.standard_normal(20000).astype(np.float32)
+    ties = (np.frombuffer(f32.tobytes(), np.uint32) & 0xFFFF0000 | 0x8000).view(np.float32)
+    vals32 = np.concatenate([f32, ties, np.float32([1e-40, -3e-39, 3.0e38, 1.0, -0.0])])
+    np.testing.assert_array_equal(oracle.round_bf16(vals32.astype(np.float64)),
+                                  f32_to_bf16_torch(vals32))
+    # doubles that are not float32 values: one-step rounding must beat double rounding
+    dbl = np.concatenate([
+        rng.standard_normal(2000) * 10.0 ** rng.integers(-30, 30, 2000),
+        np.array([1.0 + 2.0 ** -8 + 2.0 ** -40, 1.0 + 2.0 ** -8 - 2.0 ** -40,
+                  1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8)]),
+    ])
+    got = bf16_to_f64(oracle.round_bf16(dbl))
+    exp = np.array([_exact_nearest_bf16(float(v)) for v in dbl])
+    np.testing.assert_array_equal(got, exp)
+    assert struct.pack(">H", int(oracle.round_bf16(np.array([1.0 + 2.0 ** -8 + 2.0 ** -40]))[0])) \
+        == b"\x3f\x81"
