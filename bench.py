@@ -1,0 +1,420 @@
+"""Benchmark: MoE dispatch + combine on virtual EP ranks of one B200.
+
+One step = the whole hot path over one batch of synthetic DeepSeek-V3-shaped
+routing (8 virtual ranks, 256 experts, 4096 tokens per rank, hidden 7168 bf16,
+top-8 with ~2% masked slots):
+    ep_get_dispatch_layout -> ep_dispatch (prefix scan + row scatter, with
+    top-k ids and weights) -> ep_combine (y = received rows, i.e. identity
+    experts; fp32 rank-ordered reduction + combined weights).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line.  `value` is algorithmic HBM traffic per second (GB/s,
+bytes the method must move / device time, inputs resident in HBM); tokens/s,
+per-kernel times, the dominant kernel's roofline fraction, an end-to-end
+number through host buffers, clocks and a CPU-oracle baseline ride along.
+With N > 1 (torchrun), every rank runs its own independent batch (weak
+scaling, no data-path collective) and the time is the max over ranks.
+`--impl reference` times the CPU oracle on a bounded sample of the same
+workload (there is no runnable upstream implementation).
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+WORKLOAD = "dsv3"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+CPU_SAMPLE_TOKENS = 2048       # oracle baseline: first 2048 tokens of every rank
+
+
+# ------------------------------------------------------------------ bytes
+
+def step_bytes(R, T, H, K, N):
+    """Algorithmic bytes of each kernel of one step (what the method must move)."""
+    X = R * T * H * 2
+    Y = N * H * 2
+    G = R * T
+    b = {
+        "layout": G * K * 8 + G * R + R * R * 4 + R * 256 * 4,
+        "scan": G * R + G * R * 4,
+        "dispatch": X + G * R * 4 + G * K * 12 + Y + N * (K * 12 + 4),
+        "combine": Y + G * R * 4 + N * K * 4 + X + G * K * 4,
+    }
+    b["step"] = sum(b.values())
+    return b
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "combine_ep_get_11_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source
+    is unchanged since it was taken."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel]
+    except Exception:
+        return None
+    if rec.get("source_hash") != source_hash(*rec.get("sources", [])):
+        return None
+    return rec.get("dram_bytes_per_launch_full")
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(device_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        self.t_start = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), sm_max=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hw_thermal=parts[6], sw_thermal=parts[7],
+                                 sw_power=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                              ("sw_thermal", "sw_thermal_slowdown"), ("sw_power", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
+                "sm_max_mhz": max(r["sm_max"] for r in rows),
+                "power_w_max": max(r["power"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist.get_rank(), world, local
+    return 0, 1, 0
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (timing only; not on the data path)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- CPU arm
+
+def oracle_sample(w: synth.Workload, tokens: int):
+    """Run the CPU oracle over a bounded sample of the workload; returns (seconds, bytes, tokens)."""
+    import torch
+
+    import oracle
+    ws = w.scaled(num_tokens=tokens)
+    topk = synth.topk_idx(ws)
+    wts = synth.topk_weights(ws)
+    x = synth.hidden_rows(ws).view(torch.int16).numpy().view(np.uint16)
+    t0 = time.perf_counter()
+    ntr, nte, tin = oracle.layout(topk, ws.num_experts)
+    h = oracle.dispatch_handle(tin, nte, ws.num_channels)
+    recv_x, _, recv_w = oracle.dispatch_rows(x, topk, wts, h, ws.num_experts)
+    oracle.combine(recv_x, h, recv_w)
+    dt = time.perf_counter() - t0
+    N = int(h["recv_rank_offset"][-1])
+    b = step_bytes(ws.num_ranks, tokens, ws.hidden, ws.topk, N)["step"]
+    return dt, b, ws.num_ranks * tokens
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    w = synth.WORKLOADS[WORKLOAD]
+    tokens = args.cpu_sample_tokens
+    for _ in range(args.warmup):
+        oracle_sample(w, min(tokens, 64))
+    total_s, total_b, total_tok = 0.0, 0, 0
+    for _ in range(args.steps):
+        dt, b, tok = oracle_sample(w, tokens)
+        total_s += dt
+        total_b += b
+        total_tok += tok
+    gbs = total_b / total_s / 1e9
+    sample = (f"first {tokens} of {w.num_tokens} tokens of each of the {w.num_ranks} ranks, full "
+              f"hidden/top-k; layout+handle+dispatch rows+combine in the single-threaded C++ oracle")
+    line = {
+        "impl": "reference", "metric": "dispatch+combine algorithmic HBM GB/s (tokens/s alongside)",
+        "value": round(gbs, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_s / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "tokens_per_s": round(total_tok / total_s, 1),
+        "config": config_dict(w, l2_note="CPU"),
+        "cpu_baseline": {"value": round(gbs, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(gbs, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w, l2_note):
+    return {"workload": f"{w.name}: {w.num_ranks} virtual ranks, {w.num_experts} experts, "
+                        f"{w.num_tokens} tokens/rank, hidden {w.hidden} bf16, top-{w.topk} "
+                        f"({w.routing}, mask p={w.mask_prob})",
+            "num_ranks": w.num_ranks, "num_experts": w.num_experts, "tokens_per_rank": w.num_tokens,
+            "hidden": w.hidden, "topk": w.topk, "num_channels": w.num_channels,
+            "l2": l2_note}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_ours(args):
+    import torch
+
+    import combine_ep_get_11_b200 as ep
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    ep.load()
+    w = synth.WORKLOADS[WORKLOAD]
+    R, E, T, H, K, C = w.num_ranks, w.num_experts, w.num_tokens, w.hidden, w.topk, w.num_channels
+
+    # seeded inputs; each rank of a multi-GPU run draws its own batch
+    ww = w if world == 1 else dataclasses.replace(w, seed=w.seed + 1000 * rank)
+    topk_h = torch.from_numpy(synth.topk_idx(ww)).pin_memory()
+    wts_h = torch.from_numpy(synth.topk_weights(ww)).pin_memory()
+    x_h = synth.hidden_rows(ww, pin_memory=True)
+    topk_d, wts_d, x_d = topk_h.to(dev), wts_h.to(dev), x_h.to(dev)
+
+    buf = ep.Buffer(R, E, T, H, K, C, device=dev)
+    ctx = buf.ctx
+    ntr = torch.empty((R, R), dtype=torch.int32, device=dev)
+    nte = torch.empty((R, E), dtype=torch.int32, device=dev)
+    tin = torch.empty((R, T, R), dtype=torch.uint8, device=dev)
+    ep.ep_get_dispatch_layout(ctx, topk_d, ntr, nte, tin)
+    N = int(ntr.sum().item())          # receive rows of this routing (sizing read, untimed)
+    handle = ep.Handle.empty(R, T, C, E // R, N, dev)
+    handle.is_token_in_rank = tin
+    recv_x = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
+    recv_idx = torch.empty((N, K), dtype=torch.int64, device=dev)
+    recv_w = torch.empty((N, K), dtype=torch.float32, device=dev)
+    out = torch.empty((R, T, H), dtype=torch.bfloat16, device=dev)
+    out_w = torch.empty((R, T, K), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(xd, td, wd):
+        ep.ep_get_dispatch_layout(ctx, td, ntr, nte, tin)
+        ep.ep_dispatch(ctx, xd, td, wd, ntr, nte, tin, handle, recv_x, recv_idx, recv_w, N)
+        ep.ep_combine(ctx, recv_x, N, handle, recv_w, None, None, out, out_w)
+
+    for _ in range(args.warmup):
+        step(x_d, topk_d, wts_d)
+    rc = buf.sync_status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} after warm-up")
+    _ = ep.ep_profile_read(ctx)
+
+    # ---- timed region: K steps, inputs resident in HBM (all larger than L2)
+    sampler = ClockSampler(local)
+    ep.ep_profile_enable(ctx, True)
+    launches0 = ep.kernel_launch_count()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step(x_d, topk_d, wts_d)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = sampler.stop()
+    launches = ep.kernel_launch_count() - launches0
+    ep.ep_profile_enable(ctx, False)
+    prof = ep.ep_profile_read(ctx)
+    ms_local = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms_local, world, dev)
+    rc = buf.sync_status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} after the timed region")
+
+    bytes_ = step_bytes(R, T, H, K, N)
+    total_bytes = max_over_ranks(float(bytes_["step"]), world, dev) * world * args.steps
+    gbs = total_bytes / (ms / 1e3) / 1e9
+    tokens_per_s = R * T * world * args.steps / (ms / 1e3)
+
+    # ---- per-kernel times (events around each launch on the call's stream)
+    stage_ms = {k: (v[1] / v[0] if v[0] else None) for k, v in prof.items() if v[0]}
+    peak, peak_kind = measured_peak()
+    dom = max(("dispatch", "combine"), key=lambda k: stage_ms.get(k) or 0.0)
+    dom_gbs = bytes_[dom] / (stage_ms[dom] / 1e3) / 1e9
+    traffic = ncu_traffic(dom)
+    roofline = {"bound": "hbm", "kernel": f"{dom}_kernel", "achieved": round(dom_gbs, 1),
+                "peak": peak, "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                else "fallback 6650 GB/s",
+                "traffic": traffic,
+                "algorithmic_bytes_per_launch": bytes_[dom]}
+    kernels = {k: {"ms": round(v, 4), "gbs": round(bytes_[k] / (v / 1e3) / 1e9, 1)
+                   if k in bytes_ and v else None}
+               for k, v in stage_ms.items()}
+
+    # ---- end to end through host buffers (pinned), same metric
+    out_h = torch.empty((R, T, H), dtype=torch.bfloat16, pin_memory=True)
+    out_w_h = torch.empty((R, T, K), dtype=torch.float32, pin_memory=True)
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        x_d.copy_(x_h, non_blocking=True)
+        step(x_d, topk_d, wts_d)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x_d.copy_(x_h, non_blocking=True)
+        topk_d.copy_(topk_h, non_blocking=True)
+        wts_d.copy_(wts_h, non_blocking=True)
+        step(x_d, topk_d, wts_d)
+        out_h.copy_(out, non_blocking=True)
+        out_w_h.copy_(out_w, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_gbs = max_over_ranks(float(bytes_["step"]), world, dev) * world * e2e_steps / (e2e_ms / 1e3) / 1e9
+    h2d = x_h.numel() * 2 + topk_h.numel() * 8 + wts_h.numel() * 4
+    d2h = out_h.numel() * 2 + out_w_h.numel() * 4
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, b, tok = oracle_sample(w, args.cpu_sample_tokens)
+        cpu = {"value": round(b / dt / 1e9, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "tokens_per_s": round(tok / dt, 1), "seconds": round(dt, 2),
+               "sample": f"first {args.cpu_sample_tokens} of {T} tokens of each of the {R} ranks "
+                         f"(full hidden/top-k): layout+handle+dispatch rows+combine, "
+                         f"single-threaded C++ oracle, host cores: {os.cpu_count()}"}
+
+    if rank == 0:
+        line = {
+            "metric": "dispatch+combine algorithmic HBM GB/s (tokens/s alongside)",
+            "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; DeepSeek-V3-shaped routing)",
+            "tokens_per_s": round(tokens_per_s, 1),
+            "frac_of_peak_step": round(gbs / world / peak, 4),
+            "frac_of_8tbs_step": round(gbs / world / 8000.0, 4),
+            "config": config_dict(w, l2_note=f"inputs larger than L2 (x {R*T*H*2/1e6:.0f} MB, "
+                                             f"recv {N*H*2/1e9:.2f} GB > 126 MB); no flush"),
+            "num_recv_rows": N,
+            "bytes_per_step": bytes_,
+            "kernels": kernels,
+            "roofline": roofline,
+            "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                    "ms_per_step": round(e2e_ms / e2e_steps, 3)},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    buf.destroy()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=CPU_SAMPLE_TOKENS)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

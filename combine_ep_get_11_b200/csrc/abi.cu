@@ -1,0 +1,583 @@
+// C ABI of libep.so: argument validation, the context's fixed workspace, and
+// the order of kernel launches for each entry point.  See include/ep.h for the
+// contract of every call.
+//
+// Entry point -> kernels (all on the caller's stream):
+//   ep_get_dispatch_layout : memset(histograms) + layout_kernel
+//   ep_dispatch            : [layout_kernel] + memset(scan state) + scan_kernel
+//                            [+ one host read of N] + dispatch_kernel<normal>
+//   ep_dispatch_cached     : dispatch_kernel<cached>
+//   ep_combine             : combine_kernel
+//   ep_ll_dispatch         : ll_count_kernel + dispatch_kernel<packed>
+//   ep_ll_combine          : ll_combine_kernel
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "../../include/ep.h"
+#include "kernels.h"
+
+struct ep_prof_rec {
+    int kind;
+    cudaEvent_t start, stop;
+};
+
+struct ep_ctx {
+    ep_config cfg;
+    int R, E, L, T, H, K, C, Tmax;
+    long long G;
+    int64_t ll_cap;
+    int device;
+    int num_sms;
+    // device workspace (one allocation)
+    char* ws;
+    size_t ws_bytes;
+    int* err;
+    char* scan_reset;           // status | ticket | done, zeroed before every scan
+    size_t scan_reset_bytes;
+    unsigned long long* scan_status;
+    int* scan_ticket;
+    int* scan_done;
+    int scan_tiles;
+    int* boundary;              // [R][C+1][R]
+    int* ntr_ws;                // [R][R]   (layout computed inside ep_dispatch)
+    int* nte_ws;                // [R][E]
+    int* slot_map;              // [G][K]   (low-latency slots)
+    ep::DispatchGeometry geo;
+    char last_error[256];
+    bool prof;
+    std::vector<ep_prof_rec> pending;
+    int64_t prof_launches[EP_PROFILE_KINDS];
+    double prof_ms[EP_PROFILE_KINDS];
+};
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+enum Kind { kLayout = 0, kScan = 1, kDispatch = 2, kCached = 3, kCombine = 4,
+            kLLCount = 5, kLLCopy = 6, kLLCombine = 7 };
+
+size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+int fail(ep_ctx* c, int code, const char* fmt, ...) __attribute__((format(printf, 3, 4)));
+int fail(ep_ctx* c, int code, const char* fmt, ...) {
+    if (c != nullptr) {
+        va_list ap;
+        va_start(ap, fmt);
+        vsnprintf(c->last_error, sizeof c->last_error, fmt, ap);
+        va_end(ap);
+    }
+    return code;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int validate_config(const ep_config* c) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (c->num_ranks < 1 || c->num_ranks > 32) return EP_ERR_INVALID_ARG;
+    if (c->num_experts < c->num_ranks || c->num_experts > 4096 || c->num_experts % c->num_ranks != 0)
+        return EP_ERR_INVALID_ARG;
+    if (c->num_tokens < 0) return EP_ERR_INVALID_ARG;
+    if (c->topk < 1 || c->topk > 32) return EP_ERR_INVALID_ARG;
+    if (c->hidden < 8 || c->hidden > 32768) return EP_ERR_INVALID_ARG;
+    if (c->hidden % 8 != 0) return EP_ERR_ALIGNMENT;   // rows must be whole 16-byte vectors
+    if (c->num_channels < 1 || c->num_channels > 1024) return EP_ERR_INVALID_ARG;
+    if (c->ll_max_tokens_per_rank < 0) return EP_ERR_INVALID_ARG;
+    if (c->ll_max_tokens_per_rank != 0 && c->ll_max_tokens_per_rank < c->num_tokens)
+        return EP_ERR_INVALID_ARG;
+    const long long G = (long long)c->num_ranks * c->num_tokens;
+    const long long fan = c->num_ranks > c->topk ? c->num_ranks : c->topk;
+    if (G * fan >= (1LL << 31)) return EP_ERR_INVALID_ARG;
+    const long long tmax = c->ll_max_tokens_per_rank ? c->ll_max_tokens_per_rank : c->num_tokens;
+    if ((long long)c->num_ranks * tmax >= (1LL << 31)) return EP_ERR_INVALID_ARG;
+    return EP_OK;
+}
+
+// Keep the context's device current for the duration of a call.
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = true;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
+        if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+    }
+    ~DeviceGuard() {
+        int cur;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+template <class F>
+int launch(ep_ctx* c, int kind, bool has_work, cudaStream_t s, F&& f) {
+    if (!has_work) return EP_OK;
+    cudaEvent_t a = nullptr, b = nullptr;
+    if (c->prof) {
+        if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess)
+            return fail(c, EP_ERR_CUDA, "cudaEventCreate failed");
+        cudaEventRecord(a, s);
+    }
+    const cudaError_t e = f();
+    if (e != cudaSuccess) {
+        if (a) cudaEventDestroy(a);
+        if (b) cudaEventDestroy(b);
+        return fail(c, EP_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
+    }
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (c->prof) {
+        cudaEventRecord(b, s);
+        c->pending.push_back({kind, a, b});
+    }
+    return EP_OK;
+}
+
+int cuda_check(ep_ctx* c, cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return EP_OK;
+    return fail(c, EP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int begin_call(ep_ctx* c, cudaStream_t s, cudaEvent_t wait_event) {
+    c->last_error[0] = '\0';
+    if (wait_event != nullptr) return cuda_check(c, cudaStreamWaitEvent(s, wait_event, 0), "cudaStreamWaitEvent");
+    return EP_OK;
+}
+
+int check_handle(ep_ctx* c, const ep_handle* h) {
+    if (h == nullptr || h->rank_prefix_matrix == nullptr || h->channel_prefix_matrix == nullptr ||
+        h->recv_channel_prefix_matrix == nullptr || h->is_token_in_rank == nullptr ||
+        h->send_head == nullptr || h->recv_rank_offset == nullptr ||
+        h->num_recv_tokens_per_expert == nullptr)
+        return fail(c, EP_ERR_HANDLE_MISMATCH, "handle array missing");
+    if (!aligned(h->recv_rank_offset, 8) || !aligned(h->send_head, 4) || !aligned(h->is_token_in_rank, 4))
+        return fail(c, EP_ERR_ALIGNMENT, "handle array misaligned");
+    return EP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ep_status_string(int status) {
+    switch (status) {
+        case EP_OK: return "EP_OK";
+        case EP_ERR_INVALID_ARG: return "EP_ERR_INVALID_ARG";
+        case EP_ERR_ALIGNMENT: return "EP_ERR_ALIGNMENT";
+        case EP_ERR_CAPACITY: return "EP_ERR_CAPACITY";
+        case EP_ERR_BAD_TOPK: return "EP_ERR_BAD_TOPK";
+        case EP_ERR_HANDLE_MISMATCH: return "EP_ERR_HANDLE_MISMATCH";
+        case EP_ERR_TIMEOUT: return "EP_ERR_TIMEOUT";
+        case EP_ERR_CUDA: return "EP_ERR_CUDA";
+        case EP_ERR_UNIMPLEMENTED: return "EP_ERR_UNIMPLEMENTED";
+        default: return "EP_ERR_UNKNOWN";
+    }
+}
+
+uint64_t ep_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int ep_create(const ep_config* cfg, ep_ctx** out) {
+    if (out == nullptr) return EP_ERR_INVALID_ARG;
+    *out = nullptr;
+    const int v = validate_config(cfg);
+    if (v != EP_OK) return v;
+
+    ep_ctx* c = new ep_ctx();
+    c->cfg = *cfg;
+    c->R = cfg->num_ranks;
+    c->E = cfg->num_experts;
+    c->L = c->E / c->R;
+    c->T = cfg->num_tokens;
+    c->H = cfg->hidden;
+    c->K = cfg->topk;
+    c->C = cfg->num_channels;
+    c->Tmax = cfg->ll_max_tokens_per_rank ? cfg->ll_max_tokens_per_rank : cfg->num_tokens;
+    c->G = (long long)c->R * c->T;
+    c->ll_cap = (int64_t)c->R * c->Tmax;
+
+    int rc = EP_OK;
+    cudaDeviceProp prop;
+    if (cudaGetDevice(&c->device) != cudaSuccess || cudaGetDeviceProperties(&prop, c->device) != cudaSuccess) {
+        delete c;
+        return EP_ERR_CUDA;
+    }
+    if (prop.major != 10 || prop.minor != 0) {   // built for sm_100a only
+        delete c;
+        return EP_ERR_CUDA;
+    }
+    c->num_sms = prop.multiProcessorCount;
+    c->scan_tiles = (int)((c->G + ep::kScanTile - 1) / ep::kScanTile);
+
+    // workspace layout
+    size_t off = 0;
+    const size_t off_err = off;            off += align256(sizeof(int));
+    const size_t off_scan = off;
+    const size_t status_bytes = (size_t)c->scan_tiles * c->R * sizeof(unsigned long long);
+    c->scan_reset_bytes = status_bytes + 2 * sizeof(int);
+    off += align256(c->scan_reset_bytes);
+    const size_t off_bnd = off;            off += align256((size_t)c->R * (c->C + 1) * c->R * sizeof(int));
+    const size_t off_ntr = off;            off += align256((size_t)c->R * c->R * sizeof(int));
+    const size_t off_nte = off;            off += align256((size_t)c->R * c->E * sizeof(int));
+    const size_t off_slot = off;           off += align256((size_t)c->G * c->K * sizeof(int));
+    c->ws_bytes = off;
+    if (cudaMalloc(&c->ws, c->ws_bytes) != cudaSuccess) {
+        delete c;
+        return EP_ERR_CUDA;
+    }
+    c->err = reinterpret_cast<int*>(c->ws + off_err);
+    c->scan_reset = c->ws + off_scan;
+    c->scan_status = reinterpret_cast<unsigned long long*>(c->ws + off_scan);
+    c->scan_ticket = reinterpret_cast<int*>(c->ws + off_scan + status_bytes);
+    c->scan_done = c->scan_ticket + 1;
+    c->boundary = reinterpret_cast<int*>(c->ws + off_bnd);
+    c->ntr_ws = reinterpret_cast<int*>(c->ws + off_ntr);
+    c->nte_ws = reinterpret_cast<int*>(c->ws + off_nte);
+    c->slot_map = reinterpret_cast<int*>(c->ws + off_slot);
+    if (cudaMemset(c->ws, 0, c->ws_bytes) != cudaSuccess) rc = EP_ERR_CUDA;
+    if (rc == EP_OK && ep::dispatch_prepare() != cudaSuccess) rc = EP_ERR_CUDA;
+    if (rc != EP_OK) {
+        cudaFree(c->ws);
+        delete c;
+        return rc;
+    }
+    c->geo = ep::dispatch_geometry(c->H, c->G, c->num_sms);
+    *out = c;
+    return EP_OK;
+}
+
+int ep_destroy(ep_ctx* c) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    DeviceGuard guard(c->device);
+    for (auto& r : c->pending) {
+        cudaEventDestroy(r.start);
+        cudaEventDestroy(r.stop);
+    }
+    const cudaError_t e = cudaFree(c->ws);
+    delete c;
+    return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+int ep_workspace_bytes(const ep_ctx* c, size_t* bytes) {
+    if (c == nullptr || bytes == nullptr) return EP_ERR_INVALID_ARG;
+    *bytes = c->ws_bytes;
+    return EP_OK;
+}
+
+int ep_handle_layout(const ep_ctx* c, ep_handle_sizes* s) {
+    if (c == nullptr || s == nullptr) return EP_ERR_INVALID_ARG;
+    const int64_t R = c->R, C = c->C, L = c->L, H = c->H;
+    const int64_t fan = c->R < c->K ? c->R : c->K;
+    s->rank_prefix_matrix = R * R;
+    s->channel_prefix_matrix = R * R * C;
+    s->recv_channel_prefix_matrix = R * R * C;
+    s->recv_src_idx_max = c->G * fan;
+    s->is_token_in_rank = c->G * R;
+    s->send_head = c->G * R;
+    s->recv_rank_offset = R + 1;
+    s->num_recv_tokens_per_expert = R * L;
+    s->ll_packed_recv_x = R * L * c->ll_cap * H;
+    s->ll_packed_recv_count = R * L;
+    s->ll_src_info = R * L * c->ll_cap;
+    s->ll_layout_range = R * L * R * 2;
+    return EP_OK;
+}
+
+const char* ep_last_error(const ep_ctx* c) { return c == nullptr ? "null context" : c->last_error; }
+
+int ep_sync_status(ep_ctx* c, ep_stream_t stream) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int rc = cuda_check(c, cudaStreamSynchronize(s), "cudaStreamSynchronize");
+    if (rc != EP_OK) return rc;
+    int code = 0;
+    rc = cuda_check(c, cudaMemcpy(&code, c->err, sizeof(int), cudaMemcpyDeviceToHost), "read error word");
+    if (rc != EP_OK) return rc;
+    if (code != 0) {
+        rc = cuda_check(c, cudaMemset(c->err, 0, sizeof(int)), "clear error word");
+        if (rc != EP_OK) return rc;
+        return fail(c, code, "device reported %s", ep_status_string(code));
+    }
+    return EP_OK;
+}
+
+int ep_get_dispatch_layout(ep_ctx* c, const int64_t* topk_idx, int32_t* num_tokens_per_rank,
+                           int32_t* num_tokens_per_expert, uint8_t* is_token_in_rank,
+                           ep_stream_t stream, ep_event_t wait_event) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (c->G > 0 && (topk_idx == nullptr || is_token_in_rank == nullptr))
+        return fail(c, EP_ERR_INVALID_ARG, "topk_idx / is_token_in_rank missing");
+    if (num_tokens_per_rank == nullptr || num_tokens_per_expert == nullptr)
+        return fail(c, EP_ERR_INVALID_ARG, "histogram outputs missing");
+    if (!aligned(topk_idx, 8) || !aligned(is_token_in_rank, 4))
+        return fail(c, EP_ERR_ALIGNMENT, "layout arrays misaligned");
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
+    if (rc != EP_OK) return rc;
+    rc = cuda_check(c, cudaMemsetAsync(num_tokens_per_rank, 0, sizeof(int) * c->R * c->R, s), "memset");
+    if (rc == EP_OK)
+        rc = cuda_check(c, cudaMemsetAsync(num_tokens_per_expert, 0, sizeof(int) * (size_t)c->R * c->E, s), "memset");
+    if (rc != EP_OK) return rc;
+    ep::LayoutParams p{topk_idx, is_token_in_rank, num_tokens_per_rank, num_tokens_per_expert, c->err,
+                       c->R, c->E, c->L, c->T, c->K};
+    return launch(c, kLayout, c->G > 0, s, [&] { return ep::launch_layout(p, s); });
+}
+
+int ep_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, const float* topk_weights,
+                const int32_t* num_tokens_per_rank, const int32_t* num_tokens_per_expert,
+                const uint8_t* is_token_in_rank, const ep_handle* h, uint16_t* recv_x,
+                int64_t* recv_topk_idx, float* recv_topk_weights, int64_t recv_capacity_rows,
+                int64_t* num_recv_host, ep_stream_t stream, ep_event_t wait_event) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    int rc = check_handle(c, h);
+    if (rc != EP_OK) return rc;
+    if (recv_capacity_rows < 0) return fail(c, EP_ERR_INVALID_ARG, "negative capacity");
+    if (c->G > 0 && (x == nullptr || topk_idx == nullptr)) return fail(c, EP_ERR_INVALID_ARG, "x / topk_idx missing");
+    if (recv_capacity_rows > 0 && h->recv_src_idx == nullptr)
+        return fail(c, EP_ERR_HANDLE_MISMATCH, "handle recv_src_idx missing");
+    const int given = (num_tokens_per_rank != nullptr) + (num_tokens_per_expert != nullptr) +
+                      (is_token_in_rank != nullptr);
+    if (given != 0 && given != 3) return fail(c, EP_ERR_INVALID_ARG, "pass all three layout arrays or none");
+    if (!aligned16(x) || !aligned16(recv_x)) return fail(c, EP_ERR_ALIGNMENT, "row buffers must be 16-byte aligned");
+    if (!aligned(topk_idx, 8) || !aligned(recv_topk_idx, 8) || !aligned(topk_weights, 4) ||
+        !aligned(recv_topk_weights, 4) || !aligned(is_token_in_rank, 4))
+        return fail(c, EP_ERR_ALIGNMENT, "top-k arrays misaligned");
+    if (recv_topk_weights != nullptr && topk_weights == nullptr)
+        return fail(c, EP_ERR_INVALID_ARG, "recv_topk_weights needs topk_weights");
+
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
+    if (rc != EP_OK) return rc;
+
+    // 1. layout
+    const int* nte = num_tokens_per_expert;
+    if (given == 0) {
+        rc = cuda_check(c, cudaMemsetAsync(c->ntr_ws, 0, sizeof(int) * c->R * c->R, s), "memset");
+        if (rc == EP_OK) rc = cuda_check(c, cudaMemsetAsync(c->nte_ws, 0, sizeof(int) * (size_t)c->R * c->E, s), "memset");
+        if (rc != EP_OK) return rc;
+        ep::LayoutParams lp{topk_idx, h->is_token_in_rank, c->ntr_ws, c->nte_ws, c->err, c->R, c->E, c->L, c->T, c->K};
+        rc = launch(c, kLayout, c->G > 0, s, [&] { return ep::launch_layout(lp, s); });
+        if (rc != EP_OK) return rc;
+        nte = c->nte_ws;
+    } else if (is_token_in_rank != h->is_token_in_rank && c->G > 0) {
+        rc = cuda_check(c, cudaMemcpyAsync(h->is_token_in_rank, is_token_in_rank, (size_t)c->G * c->R,
+                                           cudaMemcpyDeviceToDevice, s), "copy is_token_in_rank");
+        if (rc != EP_OK) return rc;
+    }
+
+    // 2. handle (prefix scan)
+    if (c->G == 0) {
+        // no tokens: every matrix is zero
+        const size_t rc2 = sizeof(int) * (size_t)c->R * c->R * c->C;
+        cudaError_t e = cudaMemsetAsync(h->rank_prefix_matrix, 0, sizeof(int) * c->R * c->R, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(h->channel_prefix_matrix, 0, rc2, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(h->recv_channel_prefix_matrix, 0, rc2, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(h->recv_rank_offset, 0, sizeof(int64_t) * (c->R + 1), s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(h->num_recv_tokens_per_expert, 0, sizeof(int) * (size_t)c->E, s);
+        rc = cuda_check(c, e, "zero handle");
+        if (rc != EP_OK) return rc;
+        if (num_recv_host != nullptr) *num_recv_host = 0;
+        return EP_OK;
+    }
+    rc = cuda_check(c, cudaMemsetAsync(c->scan_reset, 0, c->scan_reset_bytes, s), "memset scan state");
+    if (rc != EP_OK) return rc;
+    ep::ScanParams sp{};
+    sp.is_token_in_rank = h->is_token_in_rank;
+    sp.num_tokens_per_expert = nte;
+    sp.status = c->scan_status;
+    sp.ticket = c->scan_ticket;
+    sp.done = c->scan_done;
+    sp.boundary = c->boundary;
+    sp.send_head = h->send_head;
+    sp.rank_prefix_matrix = h->rank_prefix_matrix;
+    sp.channel_prefix_matrix = h->channel_prefix_matrix;
+    sp.recv_channel_prefix_matrix = h->recv_channel_prefix_matrix;
+    sp.recv_rank_offset = reinterpret_cast<long long*>(h->recv_rank_offset);
+    sp.num_recv_tokens_per_expert = h->num_recv_tokens_per_expert;
+    sp.err = c->err;
+    sp.G = c->G;
+    sp.R = c->R; sp.E = c->E; sp.L = c->L; sp.T = c->T; sp.C = c->C;
+    sp.q = (c->T + c->C - 1) / c->C;
+    sp.num_tiles = c->scan_tiles;
+    rc = launch(c, kScan, true, s, [&] { return ep::launch_scan(sp, s); });
+    if (rc != EP_OK) return rc;
+
+    // 3. optional host read of the receive count
+    if (num_recv_host != nullptr) {
+        int64_t n = 0;
+        rc = cuda_check(c, cudaMemcpyAsync(&n, h->recv_rank_offset + c->R, sizeof n, cudaMemcpyDeviceToHost, s), "read N");
+        if (rc == EP_OK) rc = cuda_check(c, cudaStreamSynchronize(s), "cudaStreamSynchronize");
+        if (rc != EP_OK) return rc;
+        *num_recv_host = n;
+        if (n > recv_capacity_rows)
+            return fail(c, EP_ERR_CAPACITY, "%lld receive rows, capacity %lld", (long long)n,
+                        (long long)recv_capacity_rows);
+    }
+
+    // 4. rows + metadata
+    ep::DispatchParams dp{};
+    dp.x = x;
+    dp.send_head = h->send_head;
+    dp.recv_rank_offset = reinterpret_cast<const long long*>(h->recv_rank_offset);
+    dp.recv_capacity = recv_capacity_rows;
+    dp.topk_idx = topk_idx;
+    dp.topk_weights = topk_weights;
+    dp.recv_topk_idx = recv_topk_idx;
+    dp.recv_topk_weights = recv_topk_weights;
+    dp.recv_src_idx = h->recv_src_idx;
+    dp.recv_x = recv_x;
+    dp.err = c->err;
+    dp.G = c->G;
+    dp.R = c->R; dp.E = c->E; dp.L = c->L; dp.T = c->T; dp.K = c->K; dp.H = c->H;
+    return launch(c, kDispatch, true, s, [&] { return ep::launch_dispatch(ep::kModeNormal, dp, c->geo, s); });
+}
+
+int ep_dispatch_cached(ep_ctx* c, const uint16_t* x, const ep_handle* h, uint16_t* recv_x,
+                       int64_t recv_capacity_rows, ep_stream_t stream, ep_event_t wait_event) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    int rc = check_handle(c, h);
+    if (rc != EP_OK) return rc;
+    if (recv_capacity_rows < 0) return fail(c, EP_ERR_INVALID_ARG, "negative capacity");
+    if (c->G > 0 && x == nullptr) return fail(c, EP_ERR_INVALID_ARG, "x missing");
+    if (recv_x == nullptr && recv_capacity_rows > 0) return fail(c, EP_ERR_INVALID_ARG, "recv_x missing");
+    if (!aligned16(x) || !aligned16(recv_x)) return fail(c, EP_ERR_ALIGNMENT, "row buffers must be 16-byte aligned");
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
+    if (rc != EP_OK) return rc;
+    ep::DispatchParams dp{};
+    dp.x = x;
+    dp.send_head = h->send_head;
+    dp.recv_rank_offset = reinterpret_cast<const long long*>(h->recv_rank_offset);
+    dp.recv_capacity = recv_capacity_rows;
+    dp.recv_x = recv_x;
+    dp.err = c->err;
+    dp.G = c->G;
+    dp.R = c->R; dp.E = c->E; dp.L = c->L; dp.T = c->T; dp.K = c->K; dp.H = c->H;
+    return launch(c, kCached, c->G > 0 && recv_x != nullptr, s,
+                  [&] { return ep::launch_dispatch(ep::kModeCached, dp, c->geo, s); });
+}
+
+int ep_combine(ep_ctx* c, const uint16_t* y, int64_t num_recv_rows, const ep_handle* h,
+               const float* recv_topk_weights, const uint16_t* bias0, const uint16_t* bias1,
+               uint16_t* out_x, float* out_topk_weights, ep_stream_t stream, ep_event_t wait_event) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (h == nullptr || h->send_head == nullptr || h->recv_rank_offset == nullptr)
+        return fail(c, EP_ERR_HANDLE_MISMATCH, "handle send_head / recv_rank_offset missing");
+    if (num_recv_rows < 0) return fail(c, EP_ERR_INVALID_ARG, "negative row count");
+    if (c->G > 0 && out_x == nullptr) return fail(c, EP_ERR_INVALID_ARG, "out_x missing");
+    if (num_recv_rows > 0 && y == nullptr) return fail(c, EP_ERR_INVALID_ARG, "y missing");
+    if (!aligned16(y) || !aligned16(out_x) || !aligned16(bias0) || !aligned16(bias1))
+        return fail(c, EP_ERR_ALIGNMENT, "row buffers must be 16-byte aligned");
+    if (!aligned(recv_topk_weights, 4) || !aligned(out_topk_weights, 4))
+        return fail(c, EP_ERR_ALIGNMENT, "weight arrays misaligned");
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
+    if (rc != EP_OK) return rc;
+    ep::CombineParams p{};
+    p.y = y;
+    p.y_rows = num_recv_rows;
+    p.send_head = h->send_head;
+    p.recv_rank_offset = reinterpret_cast<const long long*>(h->recv_rank_offset);
+    p.recv_topk_weights = recv_topk_weights;
+    p.bias0 = bias0;
+    p.bias1 = bias1;
+    p.out_x = out_x;
+    p.out_topk_weights = out_topk_weights;
+    p.err = c->err;
+    p.G = c->G;
+    p.R = c->R; p.K = c->K; p.H = c->H;
+    return launch(c, kCombine, c->G > 0, s, [&] { return ep::launch_combine(p, c->num_sms, s); });
+}
+
+int ep_ll_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint16_t* packed_recv_x,
+                   int32_t* packed_recv_count, int32_t* src_info, int32_t* layout_range,
+                   ep_stream_t stream, ep_event_t wait_event) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (packed_recv_count == nullptr || layout_range == nullptr || src_info == nullptr)
+        return fail(c, EP_ERR_INVALID_ARG, "low-latency outputs missing");
+    if (c->G > 0 && (x == nullptr || topk_idx == nullptr || packed_recv_x == nullptr))
+        return fail(c, EP_ERR_INVALID_ARG, "x / topk_idx / packed_recv_x missing");
+    if (!aligned16(x) || !aligned16(packed_recv_x)) return fail(c, EP_ERR_ALIGNMENT, "row buffers must be 16-byte aligned");
+    if (!aligned(topk_idx, 8)) return fail(c, EP_ERR_ALIGNMENT, "topk_idx misaligned");
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
+    if (rc != EP_OK) return rc;
+    if (c->G == 0) {
+        cudaError_t e = cudaMemsetAsync(packed_recv_count, 0, sizeof(int) * (size_t)c->E, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(layout_range, 0, sizeof(int) * 2 * (size_t)c->E * c->R, s);
+        return cuda_check(c, e, "zero low-latency counts");
+    }
+    ep::LLCountParams cp{topk_idx, c->slot_map, packed_recv_count, src_info, layout_range, c->err,
+                         c->G, c->R, c->E, c->T, c->K, c->ll_cap};
+    rc = launch(c, kLLCount, true, s, [&] { return ep::launch_ll_count(cp, s); });
+    if (rc != EP_OK) return rc;
+    ep::DispatchParams dp{};
+    dp.x = x;
+    dp.topk_idx = topk_idx;
+    dp.slot_map = c->slot_map;
+    dp.ll_capacity = c->ll_cap;
+    dp.recv_x = packed_recv_x;
+    dp.err = c->err;
+    dp.G = c->G;
+    dp.R = c->R; dp.E = c->E; dp.L = c->L; dp.T = c->T; dp.K = c->K; dp.H = c->H;
+    return launch(c, kLLCopy, true, s, [&] { return ep::launch_dispatch(ep::kModeLowLatency, dp, c->geo, s); });
+}
+
+int ep_ll_combine(ep_ctx* c, const uint16_t* y, const int64_t* topk_idx, const float* topk_weights,
+                  const int32_t* src_info, const int32_t* layout_range, uint16_t* out_x,
+                  ep_stream_t stream, ep_event_t wait_event) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (c->G > 0 && (y == nullptr || topk_idx == nullptr || topk_weights == nullptr || src_info == nullptr ||
+                     layout_range == nullptr || out_x == nullptr))
+        return fail(c, EP_ERR_INVALID_ARG, "low-latency combine argument missing");
+    if (!aligned16(y) || !aligned16(out_x)) return fail(c, EP_ERR_ALIGNMENT, "row buffers must be 16-byte aligned");
+    if (!aligned(topk_idx, 8) || !aligned(topk_weights, 4)) return fail(c, EP_ERR_ALIGNMENT, "top-k arrays misaligned");
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
+    if (rc != EP_OK) return rc;
+    ep::LLCombineParams p{y, topk_idx, topk_weights, src_info, layout_range, out_x, c->err,
+                          c->G, c->R, c->E, c->T, c->K, c->H, c->ll_cap};
+    return launch(c, kLLCombine, c->G > 0, s, [&] { return ep::launch_ll_combine(p, c->num_sms, s); });
+}
+
+int ep_profile_enable(ep_ctx* c, int enable) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    c->prof = enable != 0;
+    return EP_OK;
+}
+
+int ep_profile_read(ep_ctx* c, int64_t* launches, double* total_ms) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    DeviceGuard guard(c->device);
+    int rc = EP_OK;
+    for (auto& r : c->pending) {
+        float ms = 0.f;
+        if (rc == EP_OK && cudaEventSynchronize(r.stop) == cudaSuccess &&
+            cudaEventElapsedTime(&ms, r.start, r.stop) == cudaSuccess) {
+            c->prof_launches[r.kind] += 1;
+            c->prof_ms[r.kind] += ms;
+        } else {
+            rc = EP_ERR_CUDA;
+        }
+        cudaEventDestroy(r.start);
+        cudaEventDestroy(r.stop);
+    }
+    c->pending.clear();
+    for (int k = 0; k < EP_PROFILE_KINDS; ++k) {
+        if (launches) launches[k] = c->prof_launches[k];
+        if (total_ms) total_ms[k] = c->prof_ms[k];
+        c->prof_launches[k] = 0;
+        c->prof_ms[k] = 0.0;
+    }
+    return rc;
+}
+
+}  // extern "C"

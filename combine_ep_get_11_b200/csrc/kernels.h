@@ -1,0 +1,127 @@
+// Internal launch interface between the C ABI (abi.cu) and the kernels.
+// Plain structs of device pointers and sizes; one launcher per kernel.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace ep {
+
+// ------------------------------------------------------------------ layout
+struct LayoutParams {
+    const int64_t* topk_idx;   // [G][K]
+    uint8_t* is_token_in_rank; // [G][R]
+    int* num_tokens_per_rank;  // [R][R], zeroed before launch
+    int* num_tokens_per_expert;// [R][E], zeroed before launch
+    int* err;
+    int R, E, L, T, K;
+};
+constexpr int kLayoutThreads = 256;
+cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream);
+
+// -------------------------------------------------------------------- scan
+// Decoupled-lookback scan over the G = R*T tokens in (rank, token) order of
+// the R membership columns of is_token_in_rank.  Writes send_head and samples
+// the running counts at every channel boundary; the last tile to finish turns
+// the samples into the handle matrices.
+struct ScanParams {
+    const uint8_t* is_token_in_rank;   // [G][R]
+    const int* num_tokens_per_expert;  // [R][E]
+    unsigned long long* status;        // [num_tiles][R], zeroed before launch
+    int* ticket;                       // zeroed before launch
+    int* done;                         // zeroed before launch
+    int* boundary;                     // [R][C+1][R] workspace
+    int* send_head;                    // [G][R]
+    int* rank_prefix_matrix;           // [R][R]
+    int* channel_prefix_matrix;        // [R][R][C]
+    int* recv_channel_prefix_matrix;   // [R][R][C]
+    long long* recv_rank_offset;       // [R+1]
+    int* num_recv_tokens_per_expert;   // [R][L]
+    int* err;
+    long long G;
+    int R, E, L, T, C, q, num_tiles;
+};
+constexpr int kScanTile = 256;   // tokens per tile == threads per block
+cudaError_t launch_scan(const ScanParams& p, cudaStream_t stream);
+
+// ---------------------------------------------------- dispatch (row copies)
+enum DispatchMode { kModeNormal = 0, kModeCached = 1, kModeLowLatency = 2 };
+
+struct DispatchParams {
+    const uint16_t* x;                 // [G][H]
+    // normal / cached
+    const int* send_head;              // [G][R]
+    const long long* recv_rank_offset; // [R+1]
+    int64_t recv_capacity;             // rows of recv_x
+    // normal only (metadata rows)
+    const int64_t* topk_idx;           // [G][K]
+    const float* topk_weights;         // [G][K] or null
+    int64_t* recv_topk_idx;            // [cap][K] or null
+    float* recv_topk_weights;          // [cap][K] or null
+    int* recv_src_idx;                 // [cap] or null
+    // low latency
+    const int* slot_map;               // [G][K]
+    int64_t ll_capacity;               // R * Tmax slots per expert
+    uint16_t* recv_x;                  // normal/cached: [cap][H]; LL: [E][ll_cap][H]
+    int* err;
+    long long G;
+    int R, E, L, T, K, H;
+    // launch geometry
+    int warps_per_cta, stages;
+};
+struct DispatchGeometry {
+    int ctas, warps_per_cta, stages;
+    size_t smem_bytes;
+};
+DispatchGeometry dispatch_geometry(int H, long long G, int num_sms);
+cudaError_t dispatch_prepare();   // once per device, before the first launch
+cudaError_t launch_dispatch(int mode, const DispatchParams& p, const DispatchGeometry& geo,
+                            cudaStream_t stream);
+
+// ----------------------------------------------------------------- combine
+struct CombineParams {
+    const uint16_t* y;                 // [y_rows][H]
+    int64_t y_rows;
+    const int* send_head;              // [G][R]
+    const long long* recv_rank_offset; // [R+1]
+    const float* recv_topk_weights;    // [y_rows][K] or null
+    const uint16_t* bias0;             // [G][H] or null
+    const uint16_t* bias1;             // [G][H] or null
+    uint16_t* out_x;                   // [G][H]
+    float* out_topk_weights;           // [G][K] or null
+    int* err;
+    long long G;
+    int R, K, H;
+};
+cudaError_t launch_combine(const CombineParams& p, int num_sms, cudaStream_t stream);
+
+// ------------------------------------------------------------ low latency
+struct LLCountParams {
+    const int64_t* topk_idx;   // [G][K]
+    int* slot_map;             // [G][K]
+    int* packed_recv_count;    // [E]  (= [R][L])
+    int* src_info;             // [E][ll_cap]
+    int* layout_range;         // [E][R][2]
+    int* err;
+    long long G;
+    int R, E, T, K;
+    int64_t ll_capacity;
+};
+cudaError_t launch_ll_count(const LLCountParams& p, cudaStream_t stream);
+
+struct LLCombineParams {
+    const uint16_t* y;          // [E][ll_cap][H]
+    const int64_t* topk_idx;    // [G][K]
+    const float* topk_weights;  // [G][K]
+    const int* src_info;        // [E][ll_cap]
+    const int* layout_range;    // [E][R][2]
+    uint16_t* out_x;            // [G][H]
+    int* err;
+    long long G;
+    int R, E, T, K, H;
+    int64_t ll_capacity;
+};
+cudaError_t launch_ll_combine(const LLCombineParams& p, int num_sms, cudaStream_t stream);
+
+}  // namespace ep

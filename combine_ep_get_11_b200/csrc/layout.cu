@@ -1,0 +1,82 @@
+// Dispatch layout kernel.
+//
+// "DeepEP Buffer Class API ...", section "Configuration and Layout Helpers":
+// from topk_idx derive, before any data moves, how many tokens each rank
+// receives and which ranks each token goes to; the per-expert counts are the
+// receive counts of the "Code Examples" section.
+//
+// One thread per token.  The rank-hit set of a token is a 32-bit mask (R <= 32);
+// per-rank counts come from warp ballots + popc, per-expert counts from shared
+// memory atomics, and each block adds its counts to the global histograms.
+// The grid is (token blocks, source rank), so a block never straddles ranks.
+// Traffic: K*8 bytes read and R bytes written per token; latency-bound.
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ep {
+
+namespace {
+
+__device__ __forceinline__ uint32_t spread4(uint32_t m) {
+    // bits 0..3 of m -> bytes 0..3 (each 0 or 1)
+    return (m & 1u) | ((m & 2u) << 7) | ((m & 4u) << 14) | ((m & 8u) << 21);
+}
+
+__global__ void __launch_bounds__(kLayoutThreads)
+layout_kernel(const LayoutParams p) {
+    extern __shared__ int sh[];
+    int* sh_rank = sh;        // [32]
+    int* sh_expert = sh + 32; // [E]
+    for (int i = threadIdx.x; i < 32 + p.E; i += blockDim.x) sh[i] = 0;
+    __syncthreads();
+
+    const int s = blockIdx.y;
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    uint32_t mask = 0;
+    if (t < p.T) {
+        const int64_t g = (int64_t)s * p.T + t;
+        const int64_t* row = p.topk_idx + g * p.K;
+        bool bad = false;
+        for (int k = 0; k < p.K; ++k) {
+            const int64_t e = __ldg(row + k);
+            if (e == -1) continue;
+            if (e < -1 || e >= p.E) {
+                bad = true;
+                continue;
+            }
+            mask |= 1u << (int)(e / p.L);
+            atomicAdd(&sh_expert[e], 1);
+        }
+        if (bad) record_error(p.err, EP_ERR_BAD_TOPK);
+        uint8_t* out = p.is_token_in_rank + g * p.R;
+        if ((p.R & 3) == 0) {
+            uint32_t* o4 = reinterpret_cast<uint32_t*>(out);
+            for (int c = 0; c < p.R / 4; ++c) o4[c] = spread4(mask >> (4 * c));
+        } else {
+            for (int d = 0; d < p.R; ++d) out[d] = (mask >> d) & 1u;
+        }
+    }
+    const int lane = threadIdx.x & 31;
+    for (int d = 0; d < p.R; ++d) {
+        const unsigned b = __ballot_sync(kFullMask, (mask >> d) & 1u);
+        if (lane == 0 && b) atomicAdd(&sh_rank[d], __popc(b));
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < p.R; i += blockDim.x)
+        if (sh_rank[i]) atomicAdd(p.num_tokens_per_rank + s * p.R + i, sh_rank[i]);
+    for (int i = threadIdx.x; i < p.E; i += blockDim.x)
+        if (sh_expert[i]) atomicAdd(p.num_tokens_per_expert + (int64_t)s * p.E + i, sh_expert[i]);
+}
+
+}  // namespace
+
+cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream) {
+    if (p.T == 0) return cudaSuccess;
+    dim3 grid((p.T + kLayoutThreads - 1) / kLayoutThreads, p.R);
+    const size_t smem = (32 + (size_t)p.E) * sizeof(int);
+    layout_kernel<<<grid, kLayoutThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace ep

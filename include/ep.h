@@ -1,0 +1,277 @@
+/*
+ * ep.h -- C ABI of the B200 MoE dispatch/combine library (libep.so).
+ *
+ * Mixture-of-experts token dispatch and combine, as DeepSeek's DeepEP `Buffer`
+ * defines them, for R "virtual" expert-parallel ranks that all live on one
+ * GPU: rank s owns the token rows x[s] of one [R][T][H] tensor, so dispatch
+ * and combine are permutations of device memory.
+ *
+ * Sources of the operations (web pages about DeepEP):
+ *   [API]   "DeepEP Buffer Class API for Expert Parallel Communication:
+ *            Architecture and Usage"
+ *   [REUSE] "How DeepEP Optimizes Handle Reuse for Repeated Dispatches"
+ *   [ARCH]  "Architecture" (DeepEP-Lib)
+ *   [CORE]  "Core-Implementation" (DeepEP C++ runtime)
+ *
+ * Conventions for every call
+ *   - Tensor pointers are DEVICE memory allocated by the caller, contiguous,
+ *     row-major, 16-byte aligned.  The library never takes ownership and
+ *     allocates nothing per call (ep_create allocates a fixed workspace).
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - Every call is ordered on the caller's stream; a non-null wait_event is
+ *     waited on first (the pages' `previous_event`).
+ *   - Return value: an ep_status.  Argument errors are found on the host
+ *     before anything is launched.  Errors that only the GPU can see (an
+ *     expert id out of range, a receive buffer too small, a device wait that
+ *     ran out) are recorded in a device error word and returned by the next
+ *     ep_sync_status; kernels never trap.
+ *
+ * Notation: R = num_ranks, E = num_experts, L = E / R local experts per rank,
+ * T = num_tokens per rank, H = hidden, K = topk, C = num_channels,
+ * Tmax = ll_max_tokens_per_rank, G = R * T global tokens, g = s * T + t.
+ * Expert e lives on rank e / L as local expert e % L; -1 marks an unused slot.
+ */
+#ifndef EP_B200_H
+#define EP_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define EP_API __attribute__((visibility("default")))
+#else
+#define EP_API
+#endif
+
+/* Same types as cudaStream_t / cudaEvent_t; declared here so the header
+ * needs no CUDA include. */
+typedef struct CUstream_st* ep_stream_t;
+typedef struct CUevent_st* ep_event_t;
+
+typedef enum ep_status {
+    EP_OK = 0,
+    EP_ERR_INVALID_ARG = 1,     /* bad argument or unsupported shape */
+    EP_ERR_ALIGNMENT = 2,       /* pointer not 16-byte aligned, or H*2 not a multiple of 16 */
+    EP_ERR_CAPACITY = 3,        /* a receive buffer is too small */
+    EP_ERR_BAD_TOPK = 4,        /* an expert id outside [-1, E) */
+    EP_ERR_HANDLE_MISMATCH = 5, /* handle arrays missing or not made for this context */
+    EP_ERR_TIMEOUT = 6,         /* a bounded device wait ran out */
+    EP_ERR_CUDA = 7,            /* a CUDA runtime call failed */
+    EP_ERR_UNIMPLEMENTED = 8
+} ep_status;
+
+/* Problem shape.  [ARCH] "Configuration System" tunes kernels per rank
+ * count; here launch geometry is derived from the device, and only the
+ * channel count (which shapes the channel prefix matrices) is configurable.
+ * Limits: 1 <= R <= 32; E % R == 0, E <= 4096; T >= 0; 1 <= K <= 32;
+ * H % 8 == 0, 8 <= H <= 32768; 1 <= C <= 1024; Tmax == 0 (means T) or
+ * Tmax >= T; R * T * max(R, K) < 2^31. */
+typedef struct ep_config {
+    int32_t num_ranks;
+    int32_t num_experts;
+    int32_t num_tokens;
+    int32_t hidden;
+    int32_t topk;
+    int32_t num_channels;
+    int32_t ll_max_tokens_per_rank;
+} ep_config;
+
+typedef struct ep_ctx ep_ctx;
+
+/* The dispatch handle ([REUSE] "What the Handle Contains"): rank_prefix_matrix,
+ * channel_prefix_matrix, recv_channel_prefix_matrix, recv_src_idx,
+ * is_token_in_rank and send_head, plus two conveniences (the receive offsets
+ * and per-expert receive counts).  All arrays are caller-allocated device
+ * memory, filled by ep_dispatch and read by ep_dispatch_cached / ep_combine.
+ *
+ *   rank_prefix_matrix[i][d]         i32 [R][R]    sum_{s<=i} tokens s -> d
+ *   channel_prefix_matrix[s][d][c]   i32 [R][R][C] tokens of s for d in channels 0..c
+ *   recv_channel_prefix_matrix[d][s][c] i32 [R][R][C] first receive position of
+ *                                    block (s, c) within rank d's rows
+ *   recv_src_idx[n]                  i32 [capacity] source token t of receive row n
+ *   is_token_in_rank[s][t][d]        u8  [R][T][R]
+ *   send_head[s][t][d]               i32 [R][T][R] receive position of (s, t)
+ *                                    within rank d's rows, or -1
+ *   recv_rank_offset[d]              i64 [R+1]     first row of rank d; [R] = N
+ *   num_recv_tokens_per_expert[d][j] i32 [R][L]
+ *
+ * Receive rows of rank d are [recv_rank_offset[d], recv_rank_offset[d+1]) of
+ * one concatenated buffer, ordered by source rank, then token.  Channel c of
+ * a rank covers tokens [min(c*q, T), min((c+1)*q, T)), q = ceil(T / C).
+ * The handle stays valid only while topk_idx is unchanged ([REUSE]
+ * "Performance Contract and Constraints"). */
+typedef struct ep_handle {
+    int32_t* rank_prefix_matrix;
+    int32_t* channel_prefix_matrix;
+    int32_t* recv_channel_prefix_matrix;
+    int32_t* recv_src_idx;
+    uint8_t* is_token_in_rank;
+    int32_t* send_head;
+    int64_t* recv_rank_offset;
+    int32_t* num_recv_tokens_per_expert;
+} ep_handle;
+
+/* Element counts of each handle array (recv_src_idx: worst case R*T*min(R,K)),
+ * and of the low-latency arrays, for a context. */
+typedef struct ep_handle_sizes {
+    int64_t rank_prefix_matrix;
+    int64_t channel_prefix_matrix;
+    int64_t recv_channel_prefix_matrix;
+    int64_t recv_src_idx_max;
+    int64_t is_token_in_rank;
+    int64_t send_head;
+    int64_t recv_rank_offset;
+    int64_t num_recv_tokens_per_expert;
+    int64_t ll_packed_recv_x;     /* bf16 elements of [R][L][R*Tmax][H] */
+    int64_t ll_packed_recv_count; /* [R][L] */
+    int64_t ll_src_info;          /* [R][L][R*Tmax] */
+    int64_t ll_layout_range;      /* [R][L][R][2] */
+} ep_handle_sizes;
+
+/* Create a context on the current CUDA device: validates the shape ([CORE]
+ * "Memory Alignment and Validation": rows must be whole 16-byte vectors) and
+ * allocates the fixed device workspace (scan state, error word, internal
+ * layout arrays).  *out is set only on EP_OK.  Host-only validation runs
+ * before any CUDA call, so a bad shape fails without a GPU. */
+EP_API int ep_create(const ep_config* cfg, ep_ctx** out);
+
+/* Free the context and its workspace ([API] "Explicit Resource Cleanup").
+ * Waits for nothing: the caller must not have work in flight that uses it. */
+EP_API int ep_destroy(ep_ctx* ctx);
+
+/* Bytes of device workspace the context holds. */
+EP_API int ep_workspace_bytes(const ep_ctx* ctx, size_t* bytes);
+
+/* Sizes of the handle and low-latency arrays for this context. */
+EP_API int ep_handle_layout(const ep_ctx* ctx, ep_handle_sizes* sizes);
+
+/* Human-readable name of a status code (static string). */
+EP_API const char* ep_status_string(int status);
+
+/* Description of the last host-side error on this context (static buffer in
+ * the context; empty if none). */
+EP_API const char* ep_last_error(const ep_ctx* ctx);
+
+/* Synchronize `stream`, then return and clear the device error word (EP_OK if
+ * no kernel recorded an error since the last call).  The only blocking call
+ * besides ep_dispatch with num_recv_host. */
+EP_API int ep_sync_status(ep_ctx* ctx, ep_stream_t stream);
+
+/* Number of kernels this library has launched in this process (all contexts). */
+EP_API uint64_t ep_kernel_launch_count(void);
+
+/* Dispatch layout ([API] "Configuration and Layout Helpers", [ARCH] table
+ * "Buffer.get_dispatch_layout").
+ *   topk_idx              i64 [R][T][K]  input
+ *   num_tokens_per_rank   i32 [R][R]     out: [s][d] tokens of s with an expert on d
+ *   num_tokens_per_expert i32 [R][E]     out: [s][e] slots of s naming e
+ *   is_token_in_rank      u8  [R][T][R]  out
+ * Expert ids outside [-1, E) record EP_ERR_BAD_TOPK and count as -1. */
+EP_API int ep_get_dispatch_layout(ep_ctx* ctx, const int64_t* topk_idx,
+                           int32_t* num_tokens_per_rank, int32_t* num_tokens_per_expert,
+                           uint8_t* is_token_in_rank, ep_stream_t stream, ep_event_t wait_event);
+
+/* Dispatch ([API] "Dispatch Operation"; [REUSE] "Handle Creation").
+ * Builds the handle and scatters every token row, with its top-k ids and
+ * weights, into the receive rows of each rank that owns one of its experts.
+ *   x                 bf16 [R][T][H]
+ *   topk_idx          i64  [R][T][K]
+ *   topk_weights      f32  [R][T][K]   nullable (then recv_topk_weights is not written)
+ *   num_tokens_per_rank / num_tokens_per_expert / is_token_in_rank: the
+ *                     layout from ep_get_dispatch_layout; pass all three or
+ *                     all null (then the layout is computed here, into
+ *                     handle->is_token_in_rank)
+ *   handle            arrays to fill (see ep_handle)
+ *   recv_x            bf16 [recv_capacity_rows][H]  out; nullable together with
+ *                     capacity 0 to build only the handle
+ *   recv_topk_idx     i64  [capacity][K] out, nullable: local expert id on the
+ *                     receiving rank, -1 for slots owned elsewhere
+ *   recv_topk_weights f32  [capacity][K] out, nullable: weight, 0 elsewhere
+ *   num_recv_host     nullable host pointer: if set, the call synchronizes the
+ *                     stream once after the handle is built, stores the
+ *                     number of receive rows N there and returns
+ *                     EP_ERR_CAPACITY before writing any row if N > capacity
+ *                     (the pages' CPU-GPU sync to learn receive counts).
+ * Without num_recv_host nothing blocks; rows beyond the capacity are dropped
+ * and EP_ERR_CAPACITY is recorded for ep_sync_status. */
+EP_API int ep_dispatch(ep_ctx* ctx, const uint16_t* x, const int64_t* topk_idx, const float* topk_weights,
+                const int32_t* num_tokens_per_rank, const int32_t* num_tokens_per_expert,
+                const uint8_t* is_token_in_rank, const ep_handle* handle,
+                uint16_t* recv_x, int64_t* recv_topk_idx, float* recv_topk_weights,
+                int64_t recv_capacity_rows, int64_t* num_recv_host,
+                ep_stream_t stream, ep_event_t wait_event);
+
+/* Cached dispatch ([REUSE] "Fast Path Dispatch with Handle Reuse"): scatter
+ * new rows x with a handle from an earlier ep_dispatch of the same routing.
+ * No layout, no prefix work, no host synchronization; top-k arrays are not
+ * accepted (the handle already fixes the layout).
+ *   x       bf16 [R][T][H]; recv_x bf16 [recv_capacity_rows][H] out. */
+EP_API int ep_dispatch_cached(ep_ctx* ctx, const uint16_t* x, const ep_handle* handle,
+                       uint16_t* recv_x, int64_t recv_capacity_rows,
+                       ep_stream_t stream, ep_event_t wait_event);
+
+/* Combine ([API] "Combine Operation"): reduce by addition, back in source
+ * order, the expert outputs y that sit in the receive rows of a dispatch:
+ *   out_x[s][t] = bf16( sum over d ascending with h = send_head[s][t][d] >= 0
+ *                       of y[recv_rank_offset[d] + h]  (+ bias0[s][t] + bias1[s][t]) )
+ * accumulated in fp32 in that fixed order, rounded once to bf16 (nearest even).
+ *   y                 bf16 [num_recv_rows][H]
+ *   recv_topk_weights f32  [num_recv_rows][K] nullable; if given with
+ *                     out_topk_weights, out_topk_weights[s][t][k] is the same
+ *                     ascending-rank fp32 sum of the received weight rows
+ *   bias0, bias1      bf16 [R][T][H] nullable
+ *   out_x             bf16 [R][T][H] out
+ * A token routed nowhere gets bf16(bias0 + bias1), i.e. +0 without bias.
+ * Rows at or past num_recv_rows are never read (EP_ERR_CAPACITY recorded). */
+EP_API int ep_combine(ep_ctx* ctx, const uint16_t* y, int64_t num_recv_rows, const ep_handle* handle,
+               const float* recv_topk_weights, const uint16_t* bias0, const uint16_t* bias1,
+               uint16_t* out_x, float* out_topk_weights,
+               ep_stream_t stream, ep_event_t wait_event);
+
+/* Low-latency dispatch ([API] "IB-GDA Kernels", "Low-Latency Inference with
+ * FP8" (bf16 here)): pack tokens expert-major, bounded by Tmax per rank.
+ *   x                 bf16 [R][T][H], topk_idx i64 [R][T][K]
+ *   packed_recv_x     bf16 [R][L][R*Tmax][H] out: slot p of expert (d, j) holds
+ *                     the p-th token, in (source rank, token) order, that names
+ *                     that expert (a token counts once per expert)
+ *   packed_recv_count i32  [R][L] out
+ *   src_info          i32  [R][L][R*Tmax] out: token index t of each slot
+ *   layout_range      i32  [R][L][R][2] out: {first slot, slot count} of each
+ *                     source rank
+ * Slots at or past the count are left untouched. */
+EP_API int ep_ll_dispatch(ep_ctx* ctx, const uint16_t* x, const int64_t* topk_idx,
+                   uint16_t* packed_recv_x, int32_t* packed_recv_count,
+                   int32_t* src_info, int32_t* layout_range,
+                   ep_stream_t stream, ep_event_t wait_event);
+
+/* Low-latency combine ([API] "IB-GDA Kernels"): weighted reduction of expert
+ * outputs back to token positions,
+ *   out_x[s][t] = bf16( fp32 fused multiply-add chain, starting at 0, over the
+ *                 token's valid slots in ascending (expert id, k):
+ *                 acc = fma(topk_weights[s][t][k], y[d][j][slot], acc) )
+ * where slot is the token's position in expert (d, j)'s packed list (located
+ * through layout_range and src_info from ep_ll_dispatch of the same topk_idx).
+ *   y bf16 [R][L][R*Tmax][H]; topk_weights f32 [R][T][K]; out_x bf16 [R][T][H]. */
+EP_API int ep_ll_combine(ep_ctx* ctx, const uint16_t* y, const int64_t* topk_idx,
+                  const float* topk_weights, const int32_t* src_info,
+                  const int32_t* layout_range, uint16_t* out_x,
+                  ep_stream_t stream, ep_event_t wait_event);
+
+/* Optional per-kernel timing (CUDA events around each launch on the call's
+ * stream).  ep_profile_read synchronizes the recorded events and returns,
+ * per kernel kind, the number of launches and total milliseconds since the
+ * last read; kinds: 0 layout, 1 scan (handle), 2 dispatch, 3 cached dispatch,
+ * 4 combine, 5 ll count, 6 ll copy, 7 ll combine. */
+#define EP_PROFILE_KINDS 8
+EP_API int ep_profile_enable(ep_ctx* ctx, int enable);
+EP_API int ep_profile_read(ep_ctx* ctx, int64_t* launches, double* total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EP_B200_H */

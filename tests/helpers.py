@@ -1,0 +1,70 @@
+"""Shared test utilities: bf16 bit views, the combine tolerance, GPU runners."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import synth
+
+
+def u16(t: torch.Tensor) -> np.ndarray:
+    """bf16 tensor (any device) -> numpy uint16 bit patterns."""
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def to_bf16_tensor(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint16).view(np.int16)).view(torch.bfloat16)
+
+
+def bf16_to_f64(a: np.ndarray) -> np.ndarray:
+    return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def bf16_abs(a: np.ndarray) -> np.ndarray:
+    return (a & np.uint16(0x7FFF)).astype(np.uint16)
+
+
+def bf16_ulp(v: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 values at |v| (8 significant bits; subnormals step 2^-133)."""
+    a = np.abs(v)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -126.0)
+    return np.where(a > 0, 2.0 ** (e - 7), 2.0 ** -133)
+
+
+def combine_tolerance(ref: np.ndarray, got: np.ndarray, abs_sum: np.ndarray | None, n_terms: int):
+    """Allowed |got - ref| for an fp32 accumulation of n_terms rounded to bf16, against the
+    fp64-accumulated oracle value ref (also rounded to bf16):
+      half a bf16 ulp of each rounding + the fp32 accumulation bound n*2^-24*sum|terms|.
+    With no cancellation this is the 1 bf16 ulp bar."""
+    r, g = bf16_to_f64(ref), bf16_to_f64(got)
+    tol = 0.5 * bf16_ulp(r) + 0.5 * bf16_ulp(g)
+    if abs_sum is not None:
+        tol = tol + 1.01 * n_terms * 2.0 ** -24 * bf16_to_f64(abs_sum)
+    return np.abs(g - r), tol
+
+
+def assert_combine_close(got: np.ndarray, ref: np.ndarray, abs_sum=None, n_terms=8, what=""):
+    diff, tol = combine_tolerance(ref, got, abs_sum, n_terms)
+    bad = diff > tol
+    if bad.any():
+        i = np.argwhere(bad)[0]
+        raise AssertionError(
+            f"{what}: {bad.sum()} of {bad.size} elements outside tolerance; first at {tuple(i)}: "
+            f"got {bf16_to_f64(got)[tuple(i)]!r} ref {bf16_to_f64(ref)[tuple(i)]!r} tol {tol[tuple(i)]!r}")
+    ulps = diff / bf16_ulp(bf16_to_f64(ref))
+    return float(ulps.max()) if ulps.size else 0.0, float(diff.mean()) if diff.size else 0.0
+
+
+class Inputs:
+    """Seeded inputs of one workload, on the host (numpy / CPU torch) and on the GPU."""
+
+    def __init__(self, w: synth.Workload, device="cuda"):
+        self.w = w
+        self.topk = synth.topk_idx(w)
+        self.weights = synth.topk_weights(w)
+        self.x = synth.hidden_rows(w)
+        self.x_u16 = u16(self.x)
+        self.topk_d = torch.from_numpy(self.topk).to(device)
+        self.weights_d = torch.from_numpy(self.weights).to(device)
+        self.x_d = self.x.to(device)

@@ -1,0 +1,254 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle, element by
+element, on seeded inputs small enough for the oracle, spanning several scan tiles,
+several dispatch CTAs and ragged tails.  Integer, index and copied-row outputs must
+be bit-exact; the combines must be within one bf16 ulp plus the fp32 accumulation
+bound (see tests/helpers.py)."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import Inputs, assert_combine_close, bf16_abs, to_bf16_tensor, u16
+
+pytestmark = pytest.mark.gpu
+
+W = synth.WORKLOADS
+CASES = [
+    W["tiny"],
+    W["dsv3"].scaled(num_tokens=300),                    # 2400 tokens, H = 7168
+    W["ll"].scaled(num_tokens=77, hidden=1024),
+    W["zipf"].scaled(num_tokens=70, hidden=512),         # 32 ranks, skewed destinations
+    W["reuse"].scaled(num_tokens=260),                   # H = 4096, group-limited
+    synth.Workload("odd", 3, 9, 50, 24, 4, "uniform", 99, num_channels=7),
+    synth.Workload("top1", 4, 8, 33, 64, 1, "uniform_masked", 98, num_channels=3, mask_prob=0.3),
+    synth.Workload("one-rank", 1, 6, 40, 16, 2, "uniform_masked", 97, num_channels=4, mask_prob=0.3),
+    synth.Workload("chan>T", 2, 4, 5, 8, 2, "uniform", 96, num_channels=12),
+]
+
+
+def ids(ws):
+    return [w.name for w in ws]
+
+
+@pytest.fixture(scope="module")
+def ep(cuda_lib):
+    return cuda_lib
+
+
+def make_buffer(ep, w):
+    return ep.Buffer(w.num_ranks, w.num_experts, w.num_tokens, w.hidden, w.topk, w.num_channels,
+                     w.max_tokens_per_rank)
+
+
+def oracle_normal(inp):
+    w = inp.w
+    ntr, nte, tin = oracle.layout(inp.topk, w.num_experts)
+    h = oracle.dispatch_handle(tin, nte, w.num_channels)
+    rows = oracle.dispatch_rows(inp.x_u16, inp.topk, inp.weights, h, w.num_experts)
+    return (ntr, nte, tin), h, rows
+
+
+HANDLE_KEYS = ("rank_prefix_matrix", "channel_prefix_matrix", "recv_channel_prefix_matrix",
+               "send_head", "recv_rank_offset", "num_recv_tokens_per_expert", "is_token_in_rank")
+
+
+@pytest.mark.parametrize("w", CASES, ids=ids(CASES))
+def test_layout_handle_dispatch_combine(ep, w):
+    inp = Inputs(w)
+    buf = make_buffer(ep, w)
+    (ntr, nte, tin), h, (o_recv_x, o_idx, o_w) = oracle_normal(inp)
+    N = int(h["recv_rank_offset"][-1])
+
+    layout = buf.get_dispatch_layout(inp.topk_d)
+    for got, exp, name in zip(layout, (ntr, nte, tin), ("ntr", "nte", "is_token_in_rank")):
+        np.testing.assert_array_equal(got.cpu().numpy(), exp, err_msg=name)
+
+    recv_x, recv_idx, recv_w, handle = buf.dispatch(inp.x_d, inp.topk_d, inp.weights_d, layout=layout)
+    assert buf.sync_status() == 0
+    assert handle.num_recv_rows == N
+    for key in HANDLE_KEYS:
+        np.testing.assert_array_equal(getattr(handle, key).cpu().numpy(), h[key], err_msg=key)
+    np.testing.assert_array_equal(handle.recv_src_idx.cpu().numpy()[:N], h["recv_src_idx"])
+    np.testing.assert_array_equal(u16(recv_x), o_recv_x)
+    np.testing.assert_array_equal(recv_idx.cpu().numpy(), o_idx)
+    np.testing.assert_array_equal(recv_w.cpu().numpy(), o_w)
+
+    # identity experts: every sum is exact, so the combine is bit-exact
+    out, out_w = buf.combine(recv_x, handle, recv_w)
+    e_out, e_w = oracle.combine(o_recv_x, h, o_w)
+    np.testing.assert_array_equal(u16(out), e_out)
+    np.testing.assert_array_equal(out_w.cpu().numpy(), e_w)
+
+    # independent expert outputs and two bias terms
+    y = synth.expert_rows(w.seed + 1, N, w.hidden)
+    b0, b1 = synth.bias_rows(w, 0), synth.bias_rows(w, 1)
+    out2, _ = buf.combine(y.cuda(), handle, None, bias=(b0.cuda(), b1.cuda()))
+    ref, _ = oracle.combine(u16(y), h, bias0=u16(b0), bias1=u16(b1))
+    abs_sum, _ = oracle.combine(bf16_abs(u16(y)), h, bias0=bf16_abs(u16(b0)), bias1=bf16_abs(u16(b1)))
+    assert_combine_close(u16(out2), ref, abs_sum, min(w.num_ranks, w.topk) + 2, "combine")
+
+    # cached dispatch of new rows with the same handle
+    x2 = synth.hidden_rows(dataclasses.replace(w, seed=w.seed + 17))
+    recv_x2 = buf.dispatch_cached(x2.cuda(), handle)
+    e_x2, _, _ = oracle.dispatch_rows(u16(x2), inp.topk, None, h, w.num_experts)
+    np.testing.assert_array_equal(u16(recv_x2), e_x2)
+    assert buf.sync_status() == 0
+    buf.destroy()
+
+
+@pytest.mark.parametrize("w", CASES[:5], ids=ids(CASES[:5]))
+def test_dispatch_computes_layout_itself(ep, w):
+    """ep_dispatch without a precomputed layout builds the same handle and rows."""
+    inp = Inputs(w)
+    buf = make_buffer(ep, w)
+    _, h, (o_recv_x, _, _) = oracle_normal(inp)
+    N = int(h["recv_rank_offset"][-1])
+    handle = ep.Handle.empty(w.num_ranks, w.num_tokens, w.num_channels, w.local_experts, N, "cuda")
+    recv_x = torch.empty((N, w.hidden), dtype=torch.bfloat16, device="cuda")
+    n = ep.ep_dispatch(buf.ctx, inp.x_d, inp.topk_d, None, None, None, None, handle, recv_x, None,
+                       None, N, want_num_recv=True)
+    assert n == N
+    for key in HANDLE_KEYS:
+        np.testing.assert_array_equal(getattr(handle, key).cpu().numpy(), h[key], err_msg=key)
+    np.testing.assert_array_equal(u16(recv_x), o_recv_x)
+    assert buf.sync_status() == 0
+    buf.destroy()
+
+
+LL_CASES = [
+    W["ll"].scaled(num_tokens=40, hidden=1024),
+    W["tiny"],
+    dataclasses.replace(W["ll"].scaled(num_tokens=50, hidden=256), max_tokens_per_rank=64,
+                        name="ll-tmax64"),
+    synth.Workload("ll-odd", 3, 12, 30, 40, 5, "uniform_masked", 95, mask_prob=0.2),
+]
+
+
+@pytest.mark.parametrize("w", LL_CASES, ids=ids(LL_CASES))
+def test_low_latency(ep, w):
+    inp = Inputs(w)
+    buf = make_buffer(ep, w)
+    packed, count, (src_info, layout_range) = buf.low_latency_dispatch(inp.x_d, inp.topk_d)
+    assert buf.sync_status() == 0
+    ll = oracle.ll_dispatch(inp.x_u16, inp.topk, w.num_experts, w.tmax)
+    np.testing.assert_array_equal(count.cpu().numpy(), ll["packed_recv_count"])
+    np.testing.assert_array_equal(layout_range.cpu().numpy(), ll["layout_range"])
+    p = u16(packed)
+    si = src_info.cpu().numpy()
+    R, L = w.num_ranks, w.local_experts
+    for d in range(R):
+        for j in range(L):
+            n = int(ll["packed_recv_count"][d, j])
+            np.testing.assert_array_equal(si[d, j, :n], ll["src_info"][d, j, :n])
+            np.testing.assert_array_equal(p[d, j, :n], ll["packed_recv_x"][d, j, :n])
+    # identity experts and independent expert outputs
+    for y_u16 in (p, u16(synth.expert_rows(w.seed + 3, R * L * w.tmax * w.num_ranks, w.hidden)
+                         ).reshape(p.shape)):
+        y_d = to_bf16_tensor(y_u16).cuda()
+        out = buf.low_latency_combine(y_d, inp.topk_d, inp.weights_d, (src_info, layout_range))
+        ref = oracle.ll_combine(y_u16, inp.topk, inp.weights, ll["src_info"], ll["layout_range"],
+                                w.num_experts, w.tmax)
+        abs_ref = oracle.ll_combine(bf16_abs(y_u16), inp.topk, np.abs(inp.weights), ll["src_info"],
+                                    ll["layout_range"], w.num_experts, w.tmax)
+        assert_combine_close(u16(out), ref, abs_ref, w.topk, "ll combine")
+    assert buf.sync_status() == 0
+    buf.destroy()
+
+
+# ----------------------------------------------------------------------------- edge cases
+
+def test_no_tokens(ep):
+    w = synth.Workload("empty", 4, 16, 0, 64, 2, "uniform", 1)
+    buf = make_buffer(ep, w)
+    topk = torch.empty((4, 0, 2), dtype=torch.int64, device="cuda")
+    x = torch.empty((4, 0, 64), dtype=torch.bfloat16, device="cuda")
+    recv_x, recv_idx, _, handle = buf.dispatch(x, topk)
+    assert recv_x.shape[0] == 0
+    assert handle.recv_rank_offset.cpu().tolist() == [0] * 5
+    assert not handle.rank_prefix_matrix.any() and not handle.channel_prefix_matrix.any()
+    out, _ = buf.combine(recv_x, handle)
+    assert out.numel() == 0
+    assert buf.sync_status() == 0
+    buf.destroy()
+
+
+def test_all_slots_masked(ep):
+    w = synth.Workload("masked", 2, 8, 100, 64, 2, "uniform", 2)
+    buf = make_buffer(ep, w)
+    topk = torch.full((2, 100, 2), -1, dtype=torch.int64, device="cuda")
+    x = torch.randn((2, 100, 64), device="cuda").to(torch.bfloat16)
+    recv_x, _, _, handle = buf.dispatch(x, topk)
+    assert recv_x.shape[0] == 0
+    assert (handle.send_head == -1).all()
+    out, _ = buf.combine(recv_x, handle)
+    assert (out == 0).all()
+    assert buf.sync_status() == 0
+    buf.destroy()
+
+
+def test_capacity_overflow_is_reported_not_written(ep):
+    w = W["tiny"]
+    inp = Inputs(w)
+    buf = make_buffer(ep, w)
+    _, h, (o_recv_x, _, _) = oracle_normal(inp)
+    N = int(h["recv_rank_offset"][-1])
+    cap = N - 7
+    # host-checked: the count is read back and nothing is written
+    handle = ep.Handle.empty(w.num_ranks, w.num_tokens, w.num_channels, w.local_experts, cap, "cuda")
+    recv_x = torch.zeros((cap, w.hidden), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ep.EpError) as e:
+        ep.ep_dispatch(buf.ctx, inp.x_d, inp.topk_d, None, None, None, None, handle, recv_x, None,
+                       None, cap, want_num_recv=True)
+    assert e.value.status == 3
+    assert not recv_x.any()
+    # device-checked: rows below the capacity land, the rest are dropped and reported
+    ep.ep_dispatch(buf.ctx, inp.x_d, inp.topk_d, None, None, None, None, handle, recv_x, None,
+                   None, cap)
+    assert buf.sync_status() == 3
+    assert buf.sync_status() == 0          # the error word is cleared once read
+    np.testing.assert_array_equal(u16(recv_x), o_recv_x[:cap])
+    buf.destroy()
+
+
+def test_bad_expert_id_is_reported(ep):
+    w = W["tiny"]
+    buf = make_buffer(ep, w)
+    topk = torch.from_numpy(synth.topk_idx(w)).cuda()
+    topk[1, 5, 0] = w.num_experts + 3
+    buf.get_dispatch_layout(topk)
+    assert buf.sync_status() == 4
+    buf.destroy()
+
+
+def test_misaligned_rows_are_rejected(ep):
+    w = W["tiny"]
+    inp = Inputs(w)
+    buf = make_buffer(ep, w)
+    flat = torch.empty(inp.x_d.numel() + 8, dtype=torch.bfloat16, device="cuda")
+    x_bad = flat[1:1 + inp.x_d.numel()].view(inp.x_d.shape)
+    with pytest.raises(ep.EpError) as e:
+        buf.dispatch(x_bad, inp.topk_d)
+    assert e.value.status == 2
+    buf.destroy()
+
+
+def test_profile_counts_every_kernel(ep):
+    w = W["tiny"]
+    inp = Inputs(w)
+    buf = make_buffer(ep, w)
+    ep.ep_profile_enable(buf.ctx, True)
+    before = ep.kernel_launch_count()
+    recv_x, _, recv_w, handle = buf.dispatch(inp.x_d, inp.topk_d, inp.weights_d)
+    buf.combine(recv_x, handle, recv_w)
+    buf.dispatch_cached(inp.x_d, handle)
+    packed, _, llh = buf.low_latency_dispatch(inp.x_d, inp.topk_d)
+    buf.low_latency_combine(packed, inp.topk_d, inp.weights_d, llh)
+    prof = ep.ep_profile_read(buf.ctx)
+    assert ep.kernel_launch_count() - before == 8
+    for kind in ep.PROFILE_KINDS:
+        n, ms = prof[kind]
+        assert n == 1 and ms > 0, kind
+    buf.destroy()
