@@ -172,6 +172,26 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def aggregate(ms_local: float, bytes_per_step: int, tokens_per_step: int, steps: int, world: int,
+              device=None):
+    """Whole-job numbers of a weak-scaling run: every rank moves its own batch, the
+    job time is the slowest rank's.  Returns (ms, GB/s, tokens/s)."""
+    ms = max_over_ranks(ms_local, world, device)
+    total_bytes = sum_over_ranks(float(bytes_per_step) * steps, world, device)
+    total_tokens = sum_over_ranks(float(tokens_per_step) * steps, world, device)
+    return ms, total_bytes / (ms / 1e3) / 1e9, total_tokens / (ms / 1e3)
+
+
+def sum_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -309,16 +329,13 @@ def run_ours(args):
     launches = ep.kernel_launch_count() - launches0
     ep.ep_profile_enable(ctx, False)
     prof = ep.ep_profile_read(ctx)
-    ms_local = ev0.elapsed_time(ev1)
-    ms = max_over_ranks(ms_local, world, dev)
     rc = buf.sync_status()
     if rc != 0:
         raise RuntimeError(f"device status {rc} after the timed region")
 
     bytes_ = step_bytes(R, T, H, K, N)
-    total_bytes = max_over_ranks(float(bytes_["step"]), world, dev) * world * args.steps
-    gbs = total_bytes / (ms / 1e3) / 1e9
-    tokens_per_s = R * T * world * args.steps / (ms / 1e3)
+    ms, gbs, tokens_per_s = aggregate(ev0.elapsed_time(ev1), bytes_["step"], R * T, args.steps,
+                                      world, dev)
 
     # ---- per-kernel times (events around each launch on the call's stream)
     stage_ms = {k: (v[1] / v[0] if v[0] else None) for k, v in prof.items() if v[0]}
@@ -356,8 +373,7 @@ def run_ours(args):
         out_w_h.copy_(out_w, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    e2e_gbs = max_over_ranks(float(bytes_["step"]), world, dev) * world * e2e_steps / (e2e_ms / 1e3) / 1e9
+    e2e_ms, e2e_gbs, _ = aggregate(e0.elapsed_time(e1), bytes_["step"], R * T, e2e_steps, world, dev)
     h2d = x_h.numel() * 2 + topk_h.numel() * 8 + wts_h.numel() * 4
     d2h = out_h.numel() * 2 + out_w_h.numel() * 4
 

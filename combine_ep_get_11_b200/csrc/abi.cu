@@ -147,9 +147,11 @@ int begin_call(ep_ctx* c, cudaStream_t s, cudaEvent_t wait_event) {
 }
 
 int check_handle(ep_ctx* c, const ep_handle* h) {
+    // per-token arrays are empty (and may be null) when there are no tokens
+    const bool tokens = c->G > 0;
     if (h == nullptr || h->rank_prefix_matrix == nullptr || h->channel_prefix_matrix == nullptr ||
-        h->recv_channel_prefix_matrix == nullptr || h->is_token_in_rank == nullptr ||
-        h->send_head == nullptr || h->recv_rank_offset == nullptr ||
+        h->recv_channel_prefix_matrix == nullptr || (tokens && h->is_token_in_rank == nullptr) ||
+        (tokens && h->send_head == nullptr) || h->recv_rank_offset == nullptr ||
         h->num_recv_tokens_per_expert == nullptr)
         return fail(c, EP_ERR_HANDLE_MISMATCH, "handle array missing");
     if (!aligned(h->recv_rank_offset, 8) || !aligned(h->send_head, 4) || !aligned(h->is_token_in_rank, 4))
@@ -466,7 +468,7 @@ int ep_combine(ep_ctx* c, const uint16_t* y, int64_t num_recv_rows, const ep_han
                const float* recv_topk_weights, const uint16_t* bias0, const uint16_t* bias1,
                uint16_t* out_x, float* out_topk_weights, ep_stream_t stream, ep_event_t wait_event) {
     if (c == nullptr) return EP_ERR_INVALID_ARG;
-    if (h == nullptr || h->send_head == nullptr || h->recv_rank_offset == nullptr)
+    if (h == nullptr || (c->G > 0 && h->send_head == nullptr) || h->recv_rank_offset == nullptr)
         return fail(c, EP_ERR_HANDLE_MISMATCH, "handle send_head / recv_rank_offset missing");
     if (num_recv_rows < 0) return fail(c, EP_ERR_INVALID_ARG, "negative row count");
     if (c->G > 0 && out_x == nullptr) return fail(c, EP_ERR_INVALID_ARG, "out_x missing");

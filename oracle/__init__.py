@@ -115,15 +115,20 @@ def dispatch_handle(is_token_in_rank: np.ndarray, num_tokens_per_expert: np.ndar
     return h
 
 
-def dispatch_rows(x: np.ndarray, topk_idx: np.ndarray, topk_weights, handle: dict, num_experts: int):
+def dispatch_rows(x, topk_idx: np.ndarray, topk_weights, handle: dict, num_experts: int):
     """x [R,T,H] uint16 (bf16 bits) -> recv_x [N,H] u16, recv_topk_idx [N,K] i64,
-    recv_topk_weights [N,K] f32 (None if topk_weights is None)."""
-    x = np.ascontiguousarray(x, dtype=np.uint16)
+    recv_topk_weights [N,K] f32 (None if topk_weights is None).  With x=None only the
+    top-k rows are produced (recv_x is None)."""
     topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int64)
-    R, T, H = x.shape
-    K = topk_idx.shape[2]
+    R, T, K = topk_idx.shape
     N = int(handle["recv_rank_offset"][-1])
-    recv_x = np.empty((N, H), np.uint16)
+    if x is not None:
+        x = np.ascontiguousarray(x, dtype=np.uint16)
+        H = x.shape[2]
+        recv_x = np.empty((N, H), np.uint16)
+    else:
+        H = 1
+        recv_x = None
     recv_idx = np.empty((N, K), np.int64)
     w = None if topk_weights is None else np.ascontiguousarray(topk_weights, dtype=np.float32)
     recv_w = None if w is None else np.empty((N, K), np.float32)

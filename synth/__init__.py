@@ -192,3 +192,17 @@ def bias_rows(w: Workload, which: int):
     b = torch.empty((w.num_ranks, w.num_tokens, w.hidden), dtype=torch.bfloat16)
     return _normal_bf16_rows(w.seed + 7919 * (which + 1), _KIND_BIAS,
                              (w.num_tokens, w.hidden), w.num_ranks, b)
+
+
+def expert_rows_device(seed: int, num_rows: int, hidden: int, device="cuda", chunk_rows: int = 1 << 16):
+    """An independent N(0,1) bf16 tensor [num_rows, H] drawn on the GPU with torch's
+    seeded generator (for full-size workloads whose expert outputs are too large to
+    draw on the host).  Deterministic for a given seed, device type and torch build."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    y = torch.empty((num_rows, hidden), dtype=torch.bfloat16, device=device)
+    for lo in range(0, num_rows, chunk_rows):
+        hi = min(num_rows, lo + chunk_rows)
+        y[lo:hi] = torch.randn((hi - lo, hidden), generator=gen, device=device, dtype=torch.float32)
+    return y

@@ -1,0 +1,230 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration the benchmark
+uses (same library calls, same geometry).  Where the oracle cannot hold every
+output, it is checked on sampled rows/tokens, and properties that hold at any
+size are checked everywhere:
+
+* layout, handle matrices, send_head, recv_src_idx, receive top-k rows: complete,
+  bit-exact against the oracle;
+* received hidden rows: sampled, bit-exact against the source rows the oracle
+  names;
+* combine of identity experts (y = received rows): every token, bit-exact
+  against the closed form bf16(fan-out * x);
+* combine of independent expert outputs: sampled tokens against the oracle,
+  within the combine tolerance;
+* handle reuse: 100 iterations of cached dispatch + combine replayed from one
+  CUDA graph (so no host synchronisation can happen inside an iteration).
+"""
+import numpy as np
+import psutil
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import Inputs, assert_combine_close, bf16_abs, bf16_to_f64, u16
+
+pytestmark = pytest.mark.gpu
+
+W = synth.WORKLOADS
+SAMPLE_ROWS = 4096
+SAMPLE_TOKENS = 768
+
+
+@pytest.fixture(scope="module")
+def ep(cuda_lib):
+    return cuda_lib
+
+
+def make_buffer(ep, w):
+    return ep.Buffer(w.num_ranks, w.num_experts, w.num_tokens, w.hidden, w.topk, w.num_channels,
+                     w.max_tokens_per_rank)
+
+
+def row_sources(h):
+    """(s, t) of every receive row, from the oracle handle."""
+    off = h["recv_rank_offset"]
+    rp = h["rank_prefix_matrix"]
+    N = int(off[-1])
+    rows = np.arange(N)
+    d = np.searchsorted(off[1:], rows, side="right")
+    p = rows - off[d]
+    s = np.empty(N, np.int64)
+    for dd in range(rp.shape[0]):
+        m = d == dd
+        s[m] = np.searchsorted(rp[:, dd], p[m], side="right")
+    return s, h["recv_src_idx"].astype(np.int64)
+
+
+def closed_form_identity(x_u16, tin):
+    """bf16(fan-out * x) per token: exact product in fp32, one rounding (torch CPU)."""
+    fan = torch.from_numpy(tin.sum(-1).astype(np.float32))
+    out = torch.empty(x_u16.shape, dtype=torch.bfloat16)
+    xb = torch.from_numpy(x_u16.view(np.int16)).view(torch.bfloat16)
+    for s in range(x_u16.shape[0]):
+        out[s] = (fan[s][:, None] * xb[s].float()).to(torch.bfloat16)
+    return out.view(torch.int16).numpy().view(np.uint16)
+
+
+def check_normal_full(ep, w, y_source):
+    inp = Inputs(w)
+    buf = make_buffer(ep, w)
+    ntr, nte, tin = oracle.layout(inp.topk, w.num_experts)
+    layout = buf.get_dispatch_layout(inp.topk_d)
+    for got, exp, name in zip(layout, (ntr, nte, tin), ("ntr", "nte", "is_token_in_rank")):
+        np.testing.assert_array_equal(got.cpu().numpy(), exp, err_msg=name)
+    h = oracle.dispatch_handle(tin, nte, w.num_channels)
+    N = int(h["recv_rank_offset"][-1])
+
+    recv_x, recv_idx, recv_w, handle = buf.dispatch(inp.x_d, inp.topk_d, inp.weights_d, layout=layout)
+    assert buf.sync_status() == 0
+    for key in ("rank_prefix_matrix", "channel_prefix_matrix", "recv_channel_prefix_matrix",
+                "send_head", "recv_rank_offset", "num_recv_tokens_per_expert"):
+        np.testing.assert_array_equal(getattr(handle, key).cpu().numpy(), h[key], err_msg=key)
+    np.testing.assert_array_equal(handle.recv_src_idx.cpu().numpy()[:N], h["recv_src_idx"])
+    _, o_idx, o_w = oracle.dispatch_rows(None, inp.topk, inp.weights, h, w.num_experts)
+    np.testing.assert_array_equal(recv_idx.cpu().numpy(), o_idx)
+    np.testing.assert_array_equal(recv_w.cpu().numpy(), o_w)
+
+    rng = np.random.default_rng(w.seed)
+    s_of, t_of = row_sources(h)
+    rows = rng.choice(N, size=min(SAMPLE_ROWS, N), replace=False)
+    got_rows = u16(recv_x[torch.from_numpy(rows).cuda()])
+    np.testing.assert_array_equal(got_rows, inp.x_u16[s_of[rows], t_of[rows]])
+
+    out, out_w = buf.combine(recv_x, handle, recv_w)
+    np.testing.assert_array_equal(u16(out), closed_form_identity(inp.x_u16, tin))
+    np.testing.assert_array_equal(out_w.cpu().numpy(),
+                                  np.where(inp.topk != -1, inp.weights, 0).astype(np.float32))
+
+    # independent expert outputs: sampled tokens against the oracle
+    G = w.num_ranks * w.num_tokens
+    tokens = np.sort(rng.choice(G, size=min(SAMPLE_TOKENS, G), replace=False))
+    if y_source == "host":
+        y_host = synth.expert_rows(w.seed + 5, N, w.hidden)
+        y_d = y_host.cuda()
+    else:
+        need = N * w.hidden * 2 * 1.2
+        if psutil.virtual_memory().available < need + 8e9:
+            pytest.skip("not enough host memory to hold the expert outputs for the oracle")
+        y_d = synth.expert_rows_device(w.seed + 5, N, w.hidden)
+        y_host = y_d.cpu()
+    del recv_x
+    out2, _ = buf.combine(y_d, handle)
+    got = u16(out2).reshape(G, w.hidden)[tokens]
+    y_u = u16(y_host)
+    ref, _ = oracle.combine(y_u, h, tokens=tokens)
+    abs_ref, _ = oracle.combine(bf16_abs(y_u), h, tokens=tokens)
+    assert_combine_close(got, ref, abs_ref, min(w.num_ranks, w.topk), f"{w.name} combine")
+    assert buf.sync_status() == 0
+    buf.destroy()
+
+
+def test_dsv3_full(ep):
+    check_normal_full(ep, W["dsv3"], "host")
+
+
+def test_zipf_full(ep):
+    check_normal_full(ep, W["zipf"], "device")
+
+
+def test_reuse_handle_100_iterations_in_a_graph(ep):
+    w = W["reuse"]
+    inp = Inputs(w)
+    buf = make_buffer(ep, w)
+    ntr, nte, tin = oracle.layout(inp.topk, w.num_experts)
+    h = oracle.dispatch_handle(tin, nte, w.num_channels)
+    N = int(h["recv_rank_offset"][-1])
+    recv_x, _, _, handle = buf.dispatch(inp.x_d, inp.topk_d, inp.weights_d)
+    assert buf.sync_status() == 0
+    np.testing.assert_array_equal(handle.send_head.cpu().numpy(), h["send_head"])
+
+    x_static = inp.x_d.clone()
+    recv_static = torch.empty_like(recv_x)
+    out_static = torch.empty_like(inp.x_d)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):      # warm the calls once outside capture
+        ep.ep_dispatch_cached(buf.ctx, x_static, handle, recv_static, N)
+        ep.ep_combine(buf.ctx, recv_static, N, handle, None, None, None, out_static, None)
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    launches0 = ep.kernel_launch_count()
+    with torch.cuda.graph(graph):
+        ep.ep_dispatch_cached(buf.ctx, x_static, handle, recv_static, N)
+        ep.ep_combine(buf.ctx, recv_static, N, handle, None, None, None, out_static, None)
+    assert ep.kernel_launch_count() - launches0 == 2
+
+    s_of, t_of = row_sources(h)
+    rng = np.random.default_rng(5)
+    G = w.num_ranks * w.num_tokens
+    fan = tin.sum(-1).reshape(-1).astype(np.float32)
+    for it in range(100):
+        x_static.copy_(torch.roll(inp.x_d, shifts=it, dims=1))   # new rows, same routing
+        graph.replay()
+        if it in (0, 1, 37, 99):
+            torch.cuda.synchronize()
+            x_it = np.roll(inp.x_u16, it, axis=1)
+            rows = rng.choice(N, size=2048, replace=False)
+            np.testing.assert_array_equal(u16(recv_static[torch.from_numpy(rows).cuda()]),
+                                          x_it[s_of[rows], t_of[rows]])
+            toks = rng.choice(G, size=512, replace=False)
+            xs = torch.from_numpy(x_it.reshape(G, -1)[toks].view(np.int16)).view(torch.bfloat16)
+            exp = (torch.from_numpy(fan[toks])[:, None] * xs.float()).to(torch.bfloat16)
+            got = u16(out_static.reshape(G, -1)[torch.from_numpy(toks).cuda()])
+            np.testing.assert_array_equal(got, exp.view(torch.int16).numpy().view(np.uint16))
+    assert buf.sync_status() == 0
+    del graph
+    buf.destroy()
+
+
+def test_low_latency_full(ep):
+    w = W["ll"]
+    inp = Inputs(w)
+    buf = make_buffer(ep, w)
+    R, L, T, K, H = w.num_ranks, w.local_experts, w.num_tokens, w.topk, w.hidden
+    cap = R * w.tmax
+    packed, count, (src_info, layout_range) = buf.low_latency_dispatch(inp.x_d, inp.topk_d)
+    assert buf.sync_status() == 0
+    ll = oracle.ll_dispatch(None, inp.topk, w.num_experts, w.tmax, with_rows=False)
+    np.testing.assert_array_equal(count.cpu().numpy(), ll["packed_recv_count"])
+    np.testing.assert_array_equal(layout_range.cpu().numpy(), ll["layout_range"])
+    si = src_info.cpu().numpy()
+    cnt = ll["packed_recv_count"]
+    for d in range(R):
+        for j in range(L):
+            np.testing.assert_array_equal(si[d, j, :cnt[d, j]], ll["src_info"][d, j, :cnt[d, j]])
+    # sampled packed rows
+    rng = np.random.default_rng(3)
+    lr = ll["layout_range"]
+    for _ in range(1024):
+        d, j = rng.integers(R), rng.integers(L)
+        if cnt[d, j] == 0:
+            continue
+        slot = int(rng.integers(cnt[d, j]))
+        s = int(np.searchsorted(lr[d, j, :, 0], slot, side="right") - 1)
+        while lr[d, j, s, 1] == 0 or slot >= lr[d, j, s, 0] + lr[d, j, s, 1]:
+            s -= 1
+        t = int(ll["src_info"][d, j, slot])
+        np.testing.assert_array_equal(u16(packed[d, j, slot]), inp.x_u16[s, t])
+    # identity experts, every token: out ~ x * sum of valid weights
+    out = buf.low_latency_combine(packed, inp.topk_d, inp.weights_d, (src_info, layout_range))
+    wsum = np.where(inp.topk != -1, inp.weights.astype(np.float64), 0.0).sum(-1)
+    wabs = np.where(inp.topk != -1, np.abs(inp.weights.astype(np.float64)), 0.0).sum(-1)
+    xf = bf16_to_f64(inp.x_u16)
+    ref = oracle.round_bf16(xf * wsum[..., None])
+    abs_sum = oracle.round_bf16(np.abs(xf) * wabs[..., None])
+    assert_combine_close(u16(out), ref, abs_sum, K, "ll identity combine")
+    # independent expert outputs, sampled tokens
+    y_d = synth.expert_rows_device(w.seed + 9, R * L * cap, H).view(R, L, cap, H)
+    out2 = buf.low_latency_combine(y_d, inp.topk_d, inp.weights_d, (src_info, layout_range))
+    G = R * T
+    tokens = np.sort(rng.choice(G, size=512, replace=False))
+    y_u = u16(y_d)
+    ref2 = oracle.ll_combine(y_u, inp.topk, inp.weights, ll["src_info"], ll["layout_range"],
+                             w.num_experts, w.tmax, tokens=tokens)
+    abs2 = oracle.ll_combine(bf16_abs(y_u), inp.topk, np.abs(inp.weights), ll["src_info"],
+                             ll["layout_range"], w.num_experts, w.tmax, tokens=tokens)
+    got = u16(out2).reshape(G, H)[tokens]
+    assert_combine_close(got, ref2, abs2, K, "ll combine")
+    assert buf.sync_status() == 0
+    buf.destroy()
