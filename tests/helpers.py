@@ -68,3 +68,15 @@ class Inputs:
         self.topk_d = torch.from_numpy(self.topk).to(device)
         self.weights_d = torch.from_numpy(self.weights).to(device)
         self.x_d = self.x.to(device)
+
+
+def identity_combine_closed_form(fan: np.ndarray, x_u16: np.ndarray) -> np.ndarray:
+    """Combine of identity experts, token by token: fan copies of x summed from +0.
+    The sum is exact (fan * x fits in fp32), so it is bf16(fan * x) with one rounding --
+    except for zeros: +0 plus any number of signed zeros is +0 under round-to-nearest."""
+    xb = torch.from_numpy(np.ascontiguousarray(x_u16).view(np.int16)).view(torch.bfloat16)
+    f = torch.from_numpy(np.ascontiguousarray(fan, dtype=np.float32))
+    out = (f[..., None] * xb.float()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    out = out.copy()
+    out[out == 0x8000] = 0
+    return out

@@ -21,7 +21,8 @@ import torch
 
 import oracle
 import synth
-from helpers import Inputs, assert_combine_close, bf16_abs, bf16_to_f64, u16
+from helpers import (Inputs, assert_combine_close, bf16_abs, bf16_to_f64,
+                     identity_combine_closed_form, u16)
 
 pytestmark = pytest.mark.gpu
 
@@ -56,13 +57,8 @@ def row_sources(h):
 
 
 def closed_form_identity(x_u16, tin):
-    """bf16(fan-out * x) per token: exact product in fp32, one rounding (torch CPU)."""
-    fan = torch.from_numpy(tin.sum(-1).astype(np.float32))
-    out = torch.empty(x_u16.shape, dtype=torch.bfloat16)
-    xb = torch.from_numpy(x_u16.view(np.int16)).view(torch.bfloat16)
-    for s in range(x_u16.shape[0]):
-        out[s] = (fan[s][:, None] * xb[s].float()).to(torch.bfloat16)
-    return out.view(torch.int16).numpy().view(np.uint16)
+    fan = tin.sum(-1).astype(np.float32)
+    return np.stack([identity_combine_closed_form(fan[s], x_u16[s]) for s in range(x_u16.shape[0])])
 
 
 def check_normal_full(ep, w, y_source):
@@ -168,10 +164,9 @@ def test_reuse_handle_100_iterations_in_a_graph(ep):
             np.testing.assert_array_equal(u16(recv_static[torch.from_numpy(rows).cuda()]),
                                           x_it[s_of[rows], t_of[rows]])
             toks = rng.choice(G, size=512, replace=False)
-            xs = torch.from_numpy(x_it.reshape(G, -1)[toks].view(np.int16)).view(torch.bfloat16)
-            exp = (torch.from_numpy(fan[toks])[:, None] * xs.float()).to(torch.bfloat16)
+            exp = identity_combine_closed_form(fan[toks], x_it.reshape(G, -1)[toks])
             got = u16(out_static.reshape(G, -1)[torch.from_numpy(toks).cuda()])
-            np.testing.assert_array_equal(got, exp.view(torch.int16).numpy().view(np.uint16))
+            np.testing.assert_array_equal(got, exp)
     assert buf.sync_status() == 0
     del graph
     buf.destroy()

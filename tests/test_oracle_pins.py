@@ -242,12 +242,16 @@ def test_combine_identity_experts_closed_form():
     """y = recv_x  =>  out = bf16(fan-out * x) (exact: fan-out * x fits in fp32)."""
     w_ = synth.WORKLOADS["dsv3"].scaled(num_tokens=40, hidden=64)
     topk = synth.topk_idx(w_)
-    x = synth.hidden_rows(w_).view(torch.int16).numpy().view(np.uint16)
+    x = synth.hidden_rows(w_).view(torch.int16).numpy().view(np.uint16).copy()
+    x[0, :5, :3] = 0x8000          # negative zeros: a sum that starts at +0 stays +0
+    x[1, :5, :3] = 0x0000
     _, _, tin, h, (recv_x, _, _) = run_oracle_dispatch(topk, w_.num_experts, w_.num_channels, x)
     out, _ = oracle.combine(recv_x, h)
     fan = tin.sum(-1).astype(np.float32)
     exp = f32_to_bf16_torch(fan[..., None] * bf16_to_f64(x).astype(np.float32))
+    exp[exp == 0x8000] = 0
     np.testing.assert_array_equal(out, exp)
+    assert (out[0, :5, :3] == 0).all()
 
 
 def test_combine_bias_closed_form():
