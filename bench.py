@@ -275,6 +275,8 @@ def run_ours(args):
     torch.cuda.set_device(dev)
     ep.load()
     w = synth.WORKLOADS[WORKLOAD]
+    if args.tokens and args.tokens != w.num_tokens:
+        w = w.scaled(num_tokens=args.tokens)          # same shape, fewer tokens per rank
     R, E, T, H, K, C = w.num_ranks, w.num_experts, w.num_tokens, w.hidden, w.topk, w.num_channels
 
     # seeded inputs; each rank of a multi-GPU run draws its own batch
@@ -425,6 +427,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-sample-tokens", type=int, default=CPU_SAMPLE_TOKENS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="tokens per rank (default: the workload's 4096); smaller runs are for profiling")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
     if args.impl == "reference":

@@ -340,8 +340,9 @@ int ep_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, const flo
     if (c->G > 0 && (x == nullptr || topk_idx == nullptr)) return fail(c, EP_ERR_INVALID_ARG, "x / topk_idx missing");
     if (recv_capacity_rows > 0 && h->recv_src_idx == nullptr)
         return fail(c, EP_ERR_HANDLE_MISMATCH, "handle recv_src_idx missing");
+    // (with no tokens, is_token_in_rank is empty and may be null)
     const int given = (num_tokens_per_rank != nullptr) + (num_tokens_per_expert != nullptr) +
-                      (is_token_in_rank != nullptr);
+                      (is_token_in_rank != nullptr || (c->G == 0 && num_tokens_per_rank != nullptr));
     if (given != 0 && given != 3) return fail(c, EP_ERR_INVALID_ARG, "pass all three layout arrays or none");
     if (!aligned16(x) || !aligned16(recv_x)) return fail(c, EP_ERR_ALIGNMENT, "row buffers must be 16-byte aligned");
     if (!aligned(topk_idx, 8) || !aligned(recv_topk_idx, 8) || !aligned(topk_weights, 4) ||
@@ -355,6 +356,19 @@ int ep_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, const flo
     rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
     if (rc != EP_OK) return rc;
 
+    if (c->G == 0) {
+        // no tokens: every matrix is zero
+        const size_t rc2 = sizeof(int) * (size_t)c->R * c->R * c->C;
+        cudaError_t e = cudaMemsetAsync(h->rank_prefix_matrix, 0, sizeof(int) * c->R * c->R, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(h->channel_prefix_matrix, 0, rc2, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(h->recv_channel_prefix_matrix, 0, rc2, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(h->recv_rank_offset, 0, sizeof(int64_t) * (c->R + 1), s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(h->num_recv_tokens_per_expert, 0, sizeof(int) * (size_t)c->E, s);
+        rc = cuda_check(c, e, "zero handle");
+        if (rc != EP_OK) return rc;
+        if (num_recv_host != nullptr) *num_recv_host = 0;
+        return EP_OK;
+    }
     // 1. layout
     const int* nte = num_tokens_per_expert;
     if (given == 0) {
@@ -372,19 +386,6 @@ int ep_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, const flo
     }
 
     // 2. handle (prefix scan)
-    if (c->G == 0) {
-        // no tokens: every matrix is zero
-        const size_t rc2 = sizeof(int) * (size_t)c->R * c->R * c->C;
-        cudaError_t e = cudaMemsetAsync(h->rank_prefix_matrix, 0, sizeof(int) * c->R * c->R, s);
-        if (e == cudaSuccess) e = cudaMemsetAsync(h->channel_prefix_matrix, 0, rc2, s);
-        if (e == cudaSuccess) e = cudaMemsetAsync(h->recv_channel_prefix_matrix, 0, rc2, s);
-        if (e == cudaSuccess) e = cudaMemsetAsync(h->recv_rank_offset, 0, sizeof(int64_t) * (c->R + 1), s);
-        if (e == cudaSuccess) e = cudaMemsetAsync(h->num_recv_tokens_per_expert, 0, sizeof(int) * (size_t)c->E, s);
-        rc = cuda_check(c, e, "zero handle");
-        if (rc != EP_OK) return rc;
-        if (num_recv_host != nullptr) *num_recv_host = 0;
-        return EP_OK;
-    }
     rc = cuda_check(c, cudaMemsetAsync(c->scan_reset, 0, c->scan_reset_bytes, s), "memset scan state");
     if (rc != EP_OK) return rc;
     ep::ScanParams sp{};
