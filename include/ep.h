@@ -261,6 +261,41 @@ EP_API int ep_ll_combine(ep_ctx* ctx, const uint16_t* y, const int64_t* topk_idx
                   const int32_t* layout_range, uint16_t* out_x,
                   ep_stream_t stream, ep_event_t wait_event);
 
+/* Size of the library's static device scratch array (512 KiB on every GPU that
+ * loads the library, held until the process exits). */
+#define EP_STATIC_SCRATCH_BYTES (512u * 1024u)
+
+/* Dispatch-handle build that allocates nothing.  No counterpart on the pages:
+ * this is a convenience of this library for callers that cannot call
+ * cudaMalloc -- for example a process whose device memory is all reserved by a
+ * framework's caching allocator or a fixed serving budget, or code that must
+ * not risk the device-wide synchronisation cudaMalloc/cudaFree can cause.  It
+ * needs no ep_ctx (ep_create allocates) and uses the library's static scratch
+ * array instead of a workspace.
+ *
+ * Computes what ep_dispatch's handle step computes, from a layout:
+ *   is_token_in_rank      u8  [R][T][R] input (4-byte aligned)
+ *   num_tokens_per_expert i32 [R][E]    input
+ *   handle                outputs: send_head, rank_prefix_matrix,
+ *                         channel_prefix_matrix, recv_channel_prefix_matrix,
+ *                         recv_rank_offset, num_recv_tokens_per_expert
+ *                         (recv_src_idx and is_token_in_rank are not touched)
+ *   error_word            nullable device int32, zeroed by the caller; a device
+ *                         wait that runs out stores EP_ERR_TIMEOUT there
+ * Limits as for ep_config; in addition the scratch it needs,
+ *   256 + round_up(8 * R * ceil(R*T / 256), 256) + 4 * R * R * (C + 1) bytes,
+ * must fit in EP_STATIC_SCRATCH_BYTES, or the call returns EP_ERR_CAPACITY
+ * before launching anything (R = 32, T = 8192, C = 10 needs about 300 KiB).
+ * The first call on a device looks up the array's device address (once, with
+ * that device current); make that first call before any stream capture.
+ * Every call shares the one array, and each call clears what must start at
+ * zero: calls that may overlap on the GPU (other streams, other threads) race
+ * and must be serialised by the caller. */
+EP_API int ep_dispatch_handle_static(int32_t num_ranks, int32_t num_experts, int32_t num_tokens,
+                                     int32_t num_channels, const uint8_t* is_token_in_rank,
+                                     const int32_t* num_tokens_per_expert, const ep_handle* handle,
+                                     int32_t* error_word, ep_stream_t stream);
+
 /* Optional per-kernel timing (CUDA events around each launch on the call's
  * stream).  ep_profile_read synchronizes the recorded events and returns,
  * per kernel kind, the number of launches and total milliseconds since the
