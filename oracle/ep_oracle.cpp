@@ -269,8 +269,9 @@ int oracle_dispatch_rows(int32_t R, int32_t E, int32_t T, int32_t K, int32_t H,
 
 // Combine.  [API] "Combine Operation": the handle maps received rows back to
 // their source tokens and the rows are reduced by addition, with optional bias
-// terms; the example `combine(recv_tokens, handle, recv_weights)` returns the
-// combined tokens and combined weights.  Readings: the hidden rows are summed
+// terms; in the usage example the call takes the received rows, the handle and
+// the received weights and gives back combined rows and combined weights.
+// Readings: the hidden rows are summed
 // unweighted over destination ranks in ascending order, then bias0 and bias1
 // ([R][T][H] each, optional) are added; the combined weights are the sum over
 // destinations of the received weight rows.
