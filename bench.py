@@ -265,6 +265,75 @@ def config_dict(w, l2_note):
 
 # ---------------------------------------------------------------- GPU arm
 
+class Path:
+    """One workload's timed step: buffers, the step itself and its algorithmic bytes."""
+
+    def __init__(self, ep, w, dev, topk_d, wts_d, x_d):
+        import torch
+        self.ep, self.w, self.dev = ep, w, dev
+        R, E, T, H, K, C = w.num_ranks, w.num_experts, w.num_tokens, w.hidden, w.topk, w.num_channels
+        self.buf = ep.Buffer(R, E, T, H, K, C, w.max_tokens_per_rank, device=dev)
+        ctx = self.ctx = self.buf.ctx
+        X, G = R * T * H * 2, R * T
+        self.out = torch.empty((R, T, H), dtype=torch.bfloat16, device=dev)
+        self.out_w = None
+        if w.name == "ll":
+            L, cap = E // R, R * w.tmax
+            self.packed = torch.empty((R, L, cap, H), dtype=torch.bfloat16, device=dev)
+            self.count = torch.empty((R, L), dtype=torch.int32, device=dev)
+            self.src_info = torch.empty((R, L, cap), dtype=torch.int32, device=dev)
+            self.layout_range = torch.empty((R, L, R, 2), dtype=torch.int32, device=dev)
+            valid = topk_d >= 0
+            S = int(torch.stack([(topk_d == e).any(-1) for e in range(E)]).sum().item()) \
+                if E <= 1024 else int(valid.sum().item())
+            self.N = S
+            self.bytes = {"ll_count": G * K * 12 + S * 4 + E * R * 8,
+                          "ll_copy": X + G * K * 12 + S * H * 2,
+                          "ll_combine": S * H * 2 + S * 4 + X + G * K * 12}
+            self.dominant = ("ll_copy", "ll_combine")
+            self.inputs = ("x", "topk", "weights")
+
+            def step(xd, td, wd):
+                ep.ep_ll_dispatch(ctx, xd, td, self.packed, self.count, self.src_info, self.layout_range)
+                ep.ep_ll_combine(ctx, self.packed, td, wd, self.src_info, self.layout_range, self.out)
+            self.step = step
+            return
+        ntr = torch.empty((R, R), dtype=torch.int32, device=dev)
+        nte = torch.empty((R, E), dtype=torch.int32, device=dev)
+        tin = torch.empty((R, T, R), dtype=torch.uint8, device=dev)
+        ep.ep_get_dispatch_layout(ctx, topk_d, ntr, nte, tin)
+        N = self.N = int(ntr.sum().item())    # receive rows of this routing (sizing read, untimed)
+        handle = ep.Handle.empty(R, T, C, E // R, N, dev)
+        handle.is_token_in_rank = tin
+        recv_x = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
+        Y = N * H * 2
+        if w.name == "reuse":
+            # handle built once (untimed); each step reuses it: cached dispatch + combine
+            ep.ep_dispatch(ctx, x_d, topk_d, wts_d, ntr, nte, tin, handle, recv_x, None, None, N)
+            self.bytes = {"dispatch_cached": X + G * R * 4 + Y, "combine": Y + G * R * 4 + X}
+            self.dominant = ("dispatch_cached", "combine")
+            self.inputs = ("x",)
+
+            def step(xd, td, wd):
+                ep.ep_dispatch_cached(ctx, xd, handle, recv_x, N)
+                ep.ep_combine(ctx, recv_x, N, handle, None, None, None, self.out, None)
+            self.step = step
+            return
+        recv_idx = torch.empty((N, K), dtype=torch.int64, device=dev)
+        recv_w = torch.empty((N, K), dtype=torch.float32, device=dev)
+        self.out_w = torch.empty((R, T, K), dtype=torch.float32, device=dev)
+        self.bytes = step_bytes(R, T, H, K, N)
+        del self.bytes["step"]
+        self.dominant = ("dispatch", "combine")
+        self.inputs = ("x", "topk", "weights")
+
+        def step(xd, td, wd):
+            ep.ep_get_dispatch_layout(ctx, td, ntr, nte, tin)
+            ep.ep_dispatch(ctx, xd, td, wd, ntr, nte, tin, handle, recv_x, recv_idx, recv_w, N)
+            ep.ep_combine(ctx, recv_x, N, handle, recv_w, None, None, self.out, self.out_w)
+        self.step = step
+
+
 def run_ours(args):
     import torch
 
@@ -274,10 +343,10 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     ep.load()
-    w = synth.WORKLOADS[WORKLOAD]
+    w = synth.WORKLOADS[args.workload]
     if args.tokens and args.tokens != w.num_tokens:
-        w = w.scaled(num_tokens=args.tokens)          # same shape, fewer tokens per rank
-    R, E, T, H, K, C = w.num_ranks, w.num_experts, w.num_tokens, w.hidden, w.topk, w.num_channels
+        w = dataclasses.replace(w.scaled(num_tokens=args.tokens), name=w.name)   # profiling runs
+    R, E, T, H, K = w.num_ranks, w.num_experts, w.num_tokens, w.hidden, w.topk
 
     # seeded inputs; each rank of a multi-GPU run draws its own batch
     ww = w if world == 1 else dataclasses.replace(w, seed=w.seed + 1000 * rank)
@@ -285,27 +354,17 @@ def run_ours(args):
     wts_h = torch.from_numpy(synth.topk_weights(ww)).pin_memory()
     x_h = synth.hidden_rows(ww, pin_memory=True)
     topk_d, wts_d, x_d = topk_h.to(dev), wts_h.to(dev), x_h.to(dev)
-
-    buf = ep.Buffer(R, E, T, H, K, C, device=dev)
-    ctx = buf.ctx
-    ntr = torch.empty((R, R), dtype=torch.int32, device=dev)
-    nte = torch.empty((R, E), dtype=torch.int32, device=dev)
-    tin = torch.empty((R, T, R), dtype=torch.uint8, device=dev)
-    ep.ep_get_dispatch_layout(ctx, topk_d, ntr, nte, tin)
-    N = int(ntr.sum().item())          # receive rows of this routing (sizing read, untimed)
-    handle = ep.Handle.empty(R, T, C, E // R, N, dev)
-    handle.is_token_in_rank = tin
-    recv_x = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
-    recv_idx = torch.empty((N, K), dtype=torch.int64, device=dev)
-    recv_w = torch.empty((N, K), dtype=torch.float32, device=dev)
-    out = torch.empty((R, T, H), dtype=torch.bfloat16, device=dev)
-    out_w = torch.empty((R, T, K), dtype=torch.float32, device=dev)
+    path = Path(ep, w, dev, topk_d, wts_d, x_d)
+    buf, ctx, step = path.buf, path.ctx, path.step
+    step_total = sum(path.bytes.values())
     stream = torch.cuda.current_stream(dev)
 
-    def step(xd, td, wd):
-        ep.ep_get_dispatch_layout(ctx, td, ntr, nte, tin)
-        ep.ep_dispatch(ctx, xd, td, wd, ntr, nte, tin, handle, recv_x, recv_idx, recv_w, N)
-        ep.ep_combine(ctx, recv_x, N, handle, recv_w, None, None, out, out_w)
+    # inputs smaller than L2 are re-read from L2 across steps: flush between steps then
+    input_bytes = R * T * H * 2
+    flush = input_bytes < 2 * L2_BYTES
+    # flush by reading (a written scrub leaves ~L2 of dirty lines whose write-back
+    # would overlap the next timed kernel)
+    scrub = torch.ones(L2_BYTES, dtype=torch.float16, device=dev) if flush else None
 
     for _ in range(args.warmup):
         step(x_d, topk_d, wts_d)
@@ -314,81 +373,117 @@ def run_ours(args):
         raise RuntimeError(f"device status {rc} after warm-up")
     _ = ep.ep_profile_read(ctx)
 
-    # ---- timed region: K steps, inputs resident in HBM (all larger than L2)
+    # ---- timed region: K steps, inputs resident in HBM.  By default the K steps are
+    # captured once into a CUDA graph and replayed (no host launch overhead between
+    # kernels); the library's per-kernel events are captured with them.
+    evs = [(torch.cuda.Event(enable_timing=True, external=True),
+            torch.cuda.Event(enable_timing=True, external=True))
+           for _ in range(args.steps)] if flush else None
+
+    def timed_body():
+        s = torch.cuda.current_stream(dev)
+        for i in range(args.steps):
+            if flush:
+                scrub.sum()              # L2 flush (reads 2 x L2), outside the timed pair
+                evs[i][0].record(s)
+            step(x_d, topk_d, wts_d)
+            if flush:
+                evs[i][1].record(s)
+
     sampler = ClockSampler(local)
     ep.ep_profile_enable(ctx, True)
     launches0 = ep.kernel_launch_count()
+    if args.graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            timed_body()
+        launches = ep.kernel_launch_count() - launches0    # kernels in one replay
+        ep.ep_profile_enable(ctx, False)
     barrier(world)
     torch.cuda.synchronize(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
-    for _ in range(args.steps):
-        step(x_d, topk_d, wts_d)
+    if args.graph:
+        graph.replay()
+    else:
+        timed_body()
     ev1.record(stream)
     torch.cuda.synchronize(dev)
+    if not args.graph:
+        launches = ep.kernel_launch_count() - launches0
+    ms_local = sum(a.elapsed_time(b) for a, b in evs) if flush else ev0.elapsed_time(ev1)
     barrier(world)
     clocks = sampler.stop()
-    launches = ep.kernel_launch_count() - launches0
     ep.ep_profile_enable(ctx, False)
     prof = ep.ep_profile_read(ctx)
+    if args.graph:
+        del graph
     rc = buf.sync_status()
     if rc != 0:
         raise RuntimeError(f"device status {rc} after the timed region")
 
-    bytes_ = step_bytes(R, T, H, K, N)
-    ms, gbs, tokens_per_s = aggregate(ev0.elapsed_time(ev1), bytes_["step"], R * T, args.steps,
-                                      world, dev)
+    ms, gbs, tokens_per_s = aggregate(ms_local, step_total, R * T, args.steps, world, dev)
 
     # ---- per-kernel times (events around each launch on the call's stream)
-    stage_ms = {k: (v[1] / v[0] if v[0] else None) for k, v in prof.items() if v[0]}
+    stage_ms = {k: (v[1] / v[0]) for k, v in prof.items() if v[0]}
     peak, peak_kind = measured_peak()
-    dom = max(("dispatch", "combine"), key=lambda k: stage_ms.get(k) or 0.0)
-    dom_gbs = bytes_[dom] / (stage_ms[dom] / 1e3) / 1e9
-    traffic = ncu_traffic(dom)
-    roofline = {"bound": "hbm", "kernel": f"{dom}_kernel", "achieved": round(dom_gbs, 1),
+    dom = max(path.dominant, key=lambda k: stage_ms.get(k) or 0.0)
+    dom_gbs = path.bytes[dom] / (stage_ms[dom] / 1e3) / 1e9
+    traffic = ncu_traffic(dom) if (w.name == WORKLOAD and not args.tokens) else None
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1),
                 "peak": peak, "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                 else "fallback 6650 GB/s",
                 "traffic": traffic,
-                "algorithmic_bytes_per_launch": bytes_[dom]}
-    kernels = {k: {"ms": round(v, 4), "gbs": round(bytes_[k] / (v / 1e3) / 1e9, 1)
-                   if k in bytes_ and v else None}
+                "algorithmic_bytes_per_launch": path.bytes[dom]}
+    kernels = {k: {"ms": round(v, 4), "gbs": round(path.bytes[k] / (v / 1e3) / 1e9, 1)
+                   if k in path.bytes and v else None}
                for k, v in stage_ms.items()}
 
     # ---- end to end through host buffers (pinned), same metric
     out_h = torch.empty((R, T, H), dtype=torch.bfloat16, pin_memory=True)
-    out_w_h = torch.empty((R, T, K), dtype=torch.float32, pin_memory=True)
+    out_w_h = torch.empty((R, T, K), dtype=torch.float32, pin_memory=True) if path.out_w is not None else None
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        if "topk" in path.inputs:
+            topk_d.copy_(topk_h, non_blocking=True)
+        if "weights" in path.inputs:
+            wts_d.copy_(wts_h, non_blocking=True)
+        step(x_d, topk_d, wts_d)
+        out_h.copy_(path.out, non_blocking=True)
+        if out_w_h is not None:
+            out_w_h.copy_(path.out_w, non_blocking=True)
+
     e2e_steps = max(3, min(args.steps, 20))
     for _ in range(2):
-        x_d.copy_(x_h, non_blocking=True)
-        step(x_d, topk_d, wts_d)
+        e2e_step()
     barrier(world)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        x_d.copy_(x_h, non_blocking=True)
-        topk_d.copy_(topk_h, non_blocking=True)
-        wts_d.copy_(wts_h, non_blocking=True)
-        step(x_d, topk_d, wts_d)
-        out_h.copy_(out, non_blocking=True)
-        out_w_h.copy_(out_w, non_blocking=True)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms, e2e_gbs, _ = aggregate(e0.elapsed_time(e1), bytes_["step"], R * T, e2e_steps, world, dev)
-    h2d = x_h.numel() * 2 + topk_h.numel() * 8 + wts_h.numel() * 4
-    d2h = out_h.numel() * 2 + out_w_h.numel() * 4
+    e2e_ms, e2e_gbs, _ = aggregate(e0.elapsed_time(e1), step_total, R * T, e2e_steps, world, dev)
+    h2d = x_h.numel() * 2 + ((topk_h.numel() * 8) if "topk" in path.inputs else 0) + \
+        ((wts_h.numel() * 4) if "weights" in path.inputs else 0)
+    d2h = out_h.numel() * 2 + (out_w_h.numel() * 4 if out_w_h is not None else 0)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, b, tok = oracle_sample(w, args.cpu_sample_tokens)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and w.name == WORKLOAD:
+        dt, b, tok = oracle_sample(w, min(args.cpu_sample_tokens, T))
         cpu = {"value": round(b / dt / 1e9, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
                "tokens_per_s": round(tok / dt, 1), "seconds": round(dt, 2),
-               "sample": f"first {args.cpu_sample_tokens} of {T} tokens of each of the {R} ranks "
-                         f"(full hidden/top-k): layout+handle+dispatch rows+combine, "
+               "sample": f"first {min(args.cpu_sample_tokens, T)} of {T} tokens of each of the {R} "
+                         f"ranks (full hidden/top-k): layout+handle+dispatch rows+combine, "
                          f"single-threaded C++ oracle, host cores: {os.cpu_count()}"}
 
     if rank == 0:
+        l2 = (f"L2 flushed between steps (read of {2 * L2_BYTES >> 20} MB, outside the timed pairs)"
+              if flush else f"inputs larger than L2 (x {R*T*H*2/1e6:.0f} MB, received rows "
+                            f"{path.N*H*2/1e9:.2f} GB > 126 MB); no flush")
         line = {
             "metric": "dispatch+combine algorithmic HBM GB/s (tokens/s alongside)",
             "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -396,18 +491,19 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; DeepSeek-V3-shaped routing)",
             "tokens_per_s": round(tokens_per_s, 1),
+            "us_per_step": round(ms / args.steps * 1e3, 2),
             "frac_of_peak_step": round(gbs / world / peak, 4),
             "frac_of_8tbs_step": round(gbs / world / 8000.0, 4),
-            "config": config_dict(w, l2_note=f"inputs larger than L2 (x {R*T*H*2/1e6:.0f} MB, "
-                                             f"recv {N*H*2/1e9:.2f} GB > 126 MB); no flush"),
-            "num_recv_rows": N,
-            "bytes_per_step": bytes_,
+            "config": config_dict(w, l2_note=l2),
+            "num_recv_rows": path.N,
+            "bytes_per_step": dict(path.bytes, step=step_total),
             "kernels": kernels,
             "roofline": roofline,
             "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                     "ms_per_step": round(e2e_ms / e2e_steps, 3)},
             "gpu_launches": launches,
+            "timed_as": "one CUDA graph replay of the K steps" if args.graph else "eager launches",
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
@@ -427,6 +523,10 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-sample-tokens", type=int, default=CPU_SAMPLE_TOKENS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="enqueue the timed steps eagerly instead of replaying one CUDA graph")
+    ap.add_argument("--workload", choices=sorted(synth.WORKLOADS), default=WORKLOAD,
+                    help="default dsv3 (the headline); the others are extra measurements")
     ap.add_argument("--tokens", type=int, default=0,
                     help="tokens per rank (default: the workload's 4096); smaller runs are for profiling")
     args = ap.parse_args(argv)

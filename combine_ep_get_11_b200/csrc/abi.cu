@@ -8,7 +8,7 @@
 //                            [+ one host read of N] + dispatch_kernel<normal>
 //   ep_dispatch_cached     : dispatch_kernel<cached>
 //   ep_combine             : combine_kernel
-//   ep_ll_dispatch         : ll_count_kernel + dispatch_kernel<packed>
+//   ep_ll_dispatch         : memset(LL scan state) + ll_scan_kernel + dispatch_kernel<packed>
 //   ep_ll_combine          : ll_combine_kernel
 
 #include <atomic>
@@ -46,7 +46,13 @@ struct ep_ctx {
     int* ntr_ws;                // [R][R]   (layout computed inside ep_dispatch)
     int* nte_ws;                // [R][E]
     int* slot_map;              // [G][K]   (low-latency slots)
-    ep::DispatchGeometry geo;
+    char* ll_reset;             // LL scan: status | ticket | done, zeroed before every LL scan
+    size_t ll_reset_bytes;
+    unsigned long long* ll_status;
+    int* ll_ticket;
+    int* ll_done;
+    int ll_tiles;
+    int* ll_boundary;           // [R+1][E]
     char last_error[256];
     bool prof;
     std::vector<ep_prof_rec> pending;
@@ -112,6 +118,15 @@ struct DeviceGuard {
     }
 };
 
+// Record a profiling event; inside a stream capture it becomes an event-record
+// node of the graph (so it is recorded each time the graph runs).
+cudaError_t record_event(cudaEvent_t ev, cudaStream_t s) {
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &st) == cudaSuccess && st == cudaStreamCaptureStatusActive)
+        return cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+    return cudaEventRecord(ev, s);
+}
+
 template <class F>
 int launch(ep_ctx* c, int kind, bool has_work, cudaStream_t s, F&& f) {
     if (!has_work) return EP_OK;
@@ -119,7 +134,7 @@ int launch(ep_ctx* c, int kind, bool has_work, cudaStream_t s, F&& f) {
     if (c->prof) {
         if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess)
             return fail(c, EP_ERR_CUDA, "cudaEventCreate failed");
-        cudaEventRecord(a, s);
+        record_event(a, s);
     }
     const cudaError_t e = f();
     if (e != cudaSuccess) {
@@ -129,7 +144,7 @@ int launch(ep_ctx* c, int kind, bool has_work, cudaStream_t s, F&& f) {
     }
     g_launches.fetch_add(1, std::memory_order_relaxed);
     if (c->prof) {
-        cudaEventRecord(b, s);
+        record_event(b, s);
         c->pending.push_back({kind, a, b});
     }
     return EP_OK;
@@ -223,6 +238,11 @@ int ep_create(const ep_config* cfg, ep_ctx** out) {
     const size_t off_ntr = off;            off += align256((size_t)c->R * c->R * sizeof(int));
     const size_t off_nte = off;            off += align256((size_t)c->R * c->E * sizeof(int));
     const size_t off_slot = off;           off += align256((size_t)c->G * c->K * sizeof(int));
+    c->ll_tiles = (int)((c->G + ep::kLLTile - 1) / ep::kLLTile);
+    const size_t ll_status_bytes = (size_t)c->ll_tiles * c->E * sizeof(unsigned long long);
+    c->ll_reset_bytes = ll_status_bytes + 2 * sizeof(int);
+    const size_t off_ll = off;             off += align256(c->ll_reset_bytes);
+    const size_t off_llb = off;            off += align256((size_t)(c->R + 1) * c->E * sizeof(int));
     c->ws_bytes = off;
     if (cudaMalloc(&c->ws, c->ws_bytes) != cudaSuccess) {
         delete c;
@@ -237,14 +257,18 @@ int ep_create(const ep_config* cfg, ep_ctx** out) {
     c->ntr_ws = reinterpret_cast<int*>(c->ws + off_ntr);
     c->nte_ws = reinterpret_cast<int*>(c->ws + off_nte);
     c->slot_map = reinterpret_cast<int*>(c->ws + off_slot);
+    c->ll_reset = c->ws + off_ll;
+    c->ll_status = reinterpret_cast<unsigned long long*>(c->ws + off_ll);
+    c->ll_ticket = reinterpret_cast<int*>(c->ws + off_ll + ll_status_bytes);
+    c->ll_done = c->ll_ticket + 1;
+    c->ll_boundary = reinterpret_cast<int*>(c->ws + off_llb);
     if (cudaMemset(c->ws, 0, c->ws_bytes) != cudaSuccess) rc = EP_ERR_CUDA;
-    if (rc == EP_OK && ep::dispatch_prepare() != cudaSuccess) rc = EP_ERR_CUDA;
+    if (rc == EP_OK && ep::ll_prepare(c->E) != cudaSuccess) rc = EP_ERR_CUDA;
     if (rc != EP_OK) {
         cudaFree(c->ws);
         delete c;
         return rc;
     }
-    c->geo = ep::dispatch_geometry(c->H, c->G, c->num_sms);
     *out = c;
     return EP_OK;
 }
@@ -436,7 +460,8 @@ int ep_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, const flo
     dp.err = c->err;
     dp.G = c->G;
     dp.R = c->R; dp.E = c->E; dp.L = c->L; dp.T = c->T; dp.K = c->K; dp.H = c->H;
-    return launch(c, kDispatch, true, s, [&] { return ep::launch_dispatch(ep::kModeNormal, dp, c->geo, s); });
+    dp.splits = ep::dispatch_splits(c->H);
+    return launch(c, kDispatch, true, s, [&] { return ep::launch_dispatch(ep::kModeNormal, dp, s); });
 }
 
 int ep_dispatch_cached(ep_ctx* c, const uint16_t* x, const ep_handle* h, uint16_t* recv_x,
@@ -461,8 +486,9 @@ int ep_dispatch_cached(ep_ctx* c, const uint16_t* x, const ep_handle* h, uint16_
     dp.err = c->err;
     dp.G = c->G;
     dp.R = c->R; dp.E = c->E; dp.L = c->L; dp.T = c->T; dp.K = c->K; dp.H = c->H;
+    dp.splits = ep::dispatch_splits(c->H);
     return launch(c, kCached, c->G > 0 && recv_x != nullptr, s,
-                  [&] { return ep::launch_dispatch(ep::kModeCached, dp, c->geo, s); });
+                  [&] { return ep::launch_dispatch(ep::kModeCached, dp, s); });
 }
 
 int ep_combine(ep_ctx* c, const uint16_t* y, int64_t num_recv_rows, const ep_handle* h,
@@ -495,6 +521,7 @@ int ep_combine(ep_ctx* c, const uint16_t* y, int64_t num_recv_rows, const ep_han
     p.err = c->err;
     p.G = c->G;
     p.R = c->R; p.K = c->K; p.H = c->H;
+    p.splits = ep::combine_splits(c->H);
     return launch(c, kCombine, c->G > 0, s, [&] { return ep::launch_combine(p, c->num_sms, s); });
 }
 
@@ -517,8 +544,11 @@ int ep_ll_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint16
         if (e == cudaSuccess) e = cudaMemsetAsync(layout_range, 0, sizeof(int) * 2 * (size_t)c->E * c->R, s);
         return cuda_check(c, e, "zero low-latency counts");
     }
-    ep::LLCountParams cp{topk_idx, c->slot_map, packed_recv_count, src_info, layout_range, c->err,
-                         c->G, c->R, c->E, c->T, c->K, c->ll_cap};
+    rc = cuda_check(c, cudaMemsetAsync(c->ll_reset, 0, c->ll_reset_bytes, s), "memset low-latency scan state");
+    if (rc != EP_OK) return rc;
+    ep::LLCountParams cp{topk_idx, c->slot_map, packed_recv_count, src_info, layout_range,
+                         c->ll_status, c->ll_ticket, c->ll_done, c->ll_boundary, c->err,
+                         c->G, c->R, c->E, c->T, c->K, c->ll_cap, c->ll_tiles};
     rc = launch(c, kLLCount, true, s, [&] { return ep::launch_ll_count(cp, s); });
     if (rc != EP_OK) return rc;
     ep::DispatchParams dp{};
@@ -530,7 +560,8 @@ int ep_ll_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint16
     dp.err = c->err;
     dp.G = c->G;
     dp.R = c->R; dp.E = c->E; dp.L = c->L; dp.T = c->T; dp.K = c->K; dp.H = c->H;
-    return launch(c, kLLCopy, true, s, [&] { return ep::launch_dispatch(ep::kModeLowLatency, dp, c->geo, s); });
+    dp.splits = ep::dispatch_splits(c->H);
+    return launch(c, kLLCopy, true, s, [&] { return ep::launch_dispatch(ep::kModeLowLatency, dp, s); });
 }
 
 int ep_ll_combine(ep_ctx* c, const uint16_t* y, const int64_t* topk_idx, const float* topk_weights,
@@ -547,7 +578,8 @@ int ep_ll_combine(ep_ctx* c, const uint16_t* y, const int64_t* topk_idx, const f
     int rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
     if (rc != EP_OK) return rc;
     ep::LLCombineParams p{y, topk_idx, topk_weights, src_info, layout_range, out_x, c->err,
-                          c->G, c->R, c->E, c->T, c->K, c->H, c->ll_cap};
+                          c->G, c->R, c->E, c->T, c->K, c->H, c->ll_cap,
+                          ep::combine_splits(c->H)};
     return launch(c, kLLCombine, c->G > 0, s, [&] { return ep::launch_ll_combine(p, c->num_sms, s); });
 }
 

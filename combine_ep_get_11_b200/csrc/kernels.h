@@ -8,6 +8,13 @@
 
 namespace ep {
 
+// Warps per token for the row kernels: a token's row may be cut into column
+// slices (whole 512-byte warp strides) handled by separate warps.  Measured on
+// B200: the fan-out copy gains ~2% from two warps per row (more stores in
+// flight per row); the gather-reduce kernels do best with one.
+inline int dispatch_splits(int H) { return (H / 8) >= 64 ? 2 : 1; }
+inline int combine_splits(int) { return 1; }
+
 // ------------------------------------------------------------------ layout
 struct LayoutParams {
     const int64_t* topk_idx;   // [G][K]
@@ -67,17 +74,9 @@ struct DispatchParams {
     int* err;
     long long G;
     int R, E, L, T, K, H;
-    // launch geometry
-    int warps_per_cta, stages;
+    int splits;                        // warps per token (column slices of the row)
 };
-struct DispatchGeometry {
-    int ctas, warps_per_cta, stages;
-    size_t smem_bytes;
-};
-DispatchGeometry dispatch_geometry(int H, long long G, int num_sms);
-cudaError_t dispatch_prepare();   // once per device, before the first launch
-cudaError_t launch_dispatch(int mode, const DispatchParams& p, const DispatchGeometry& geo,
-                            cudaStream_t stream);
+cudaError_t launch_dispatch(int mode, const DispatchParams& p, cudaStream_t stream);
 
 // ----------------------------------------------------------------- combine
 struct CombineParams {
@@ -93,22 +92,32 @@ struct CombineParams {
     int* err;
     long long G;
     int R, K, H;
+    int splits;                        // warps per token (column slices of the row)
 };
 cudaError_t launch_combine(const CombineParams& p, int num_sms, cudaStream_t stream);
 
 // ------------------------------------------------------------ low latency
+// Low-latency slot assignment: a decoupled-lookback scan over 256-token tiles
+// whose columns are the E experts (the same scheme as the handle scan).
 struct LLCountParams {
     const int64_t* topk_idx;   // [G][K]
     int* slot_map;             // [G][K]
     int* packed_recv_count;    // [E]  (= [R][L])
     int* src_info;             // [E][ll_cap]
     int* layout_range;         // [E][R][2]
+    unsigned long long* status;// [num_tiles][E], zeroed before launch
+    int* ticket;               // zeroed before launch
+    int* done;                 // zeroed before launch
+    int* boundary;             // [R+1][E] workspace
     int* err;
     long long G;
     int R, E, T, K;
     int64_t ll_capacity;
+    int num_tiles;
 };
+constexpr int kLLTile = 256;   // tokens per tile == threads per block
 cudaError_t launch_ll_count(const LLCountParams& p, cudaStream_t stream);
+cudaError_t ll_prepare(int E);   // once per device: shared-memory opt-in
 
 struct LLCombineParams {
     const uint16_t* y;          // [E][ll_cap][H]
@@ -121,6 +130,7 @@ struct LLCombineParams {
     long long G;
     int R, E, T, K, H;
     int64_t ll_capacity;
+    int splits;                 // warps per token (column slices of the row)
 };
 cudaError_t launch_ll_combine(const LLCombineParams& p, int num_sms, cudaStream_t stream);
 

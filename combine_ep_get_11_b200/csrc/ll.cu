@@ -8,13 +8,12 @@
 // handle.
 //
 // Slot order: the tokens of expert e are packed in (source rank, token) order,
-// so slot(s, t, e) = #{(s', t') < (s, t) naming e}.  ll_count_kernel computes
-// it with one CTA per expert: the CTA sweeps all G tokens in order, a block
-// scan of the membership flags gives each member its slot, and it writes
-// src_info (token index per slot), layout_range (first slot and count per
-// source rank), the count, and a [G][K] slot map for the copy kernel (the
-// dispatch kernel's packed mode).  No atomics touch the order, so the packing
-// is deterministic.
+// so slot(s, t, e) = #{(s', t') < (s, t) naming e}: an exclusive running count
+// over the G tokens, one column per expert.  ll_scan_kernel computes all E
+// columns in one decoupled-lookback pass and writes src_info (token index per
+// slot), layout_range (first slot and count per source rank), the counts and a
+// [G][K] slot map for the copy kernel (the dispatch kernel's packed mode).  No
+// atomic decides an order, so the packing is deterministic.
 //
 // ll_combine_kernel: one warp per token.  Lane k finds the slot of its expert
 // by binary search in src_info inside layout_range[e][s] (ascending token
@@ -28,70 +27,159 @@ namespace ep {
 
 namespace {
 
-constexpr int kCountThreads = 512;
-constexpr int kCountWarps = kCountThreads / 32;
 constexpr int kLLCombineThreads = 256;
 constexpr int kLLCombineWarps = kLLCombineThreads / 32;
-constexpr int kRowsPerGroup = 8;
+constexpr int kLLRowsPerGroup = 8;
+constexpr int kLLWords = kLLTile / 32;
+constexpr int kLLStride = kLLWords + 1;   // odd row stride: no shared-memory bank conflicts
+constexpr unsigned long long kLLFlagAggregate = 1ull << 62;
+constexpr unsigned long long kLLFlagInclusive = 2ull << 62;
 
-__global__ void __launch_bounds__(kCountThreads)
-ll_count_kernel(const LLCountParams p) {
-    __shared__ int s_warp_total[kCountWarps];
-    __shared__ int s_base;
-    __shared__ int s_begin[33];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int e = blockIdx.x;
-    const long long cap = p.ll_capacity;
-    int* src_info = p.src_info + (long long)e * cap;
-    if (tid == 0) s_base = 0;
+__host__ __device__ inline size_t ll_scan_smem(int E) {
+    return (size_t)E * kLLStride * sizeof(uint32_t) + (size_t)E * sizeof(int);
+}
+
+// One 256-token tile per block (ticket order).  Each thread owns one token:
+// its experts set one bit each in the tile's [E][8]-word membership bitmap (a
+// token naming an expert twice sets the same bit).  Thread e then publishes
+// expert e's tile count and looks back over earlier tiles for the exclusive
+// prefix (bounded wait); a member's slot is that prefix plus the members of the
+// expert earlier in the tile.  Samples of the running counts at each source
+// rank's first token go to `boundary`; the last tile to finish turns them into
+// layout_range and the per-expert counts.
+template <int kMaxK>
+__global__ void __launch_bounds__(kLLTile)
+ll_scan_kernel(const LLCountParams p) {
+    extern __shared__ uint32_t ll_smem[];
+    uint32_t* bits = ll_smem;                                       // [E][kLLStride]
+    int* s_excl = reinterpret_cast<int*>(ll_smem + (size_t)p.E * kLLStride);  // [E]
+    __shared__ int s_tile, s_last;
+    const int tid = threadIdx.x;
+    const int E = p.E;
+    if (tid == 0) s_tile = atomicAdd(p.ticket, 1);
+    for (int i = tid; i < E * kLLStride; i += kLLTile) bits[i] = 0;
+    __syncthreads();
+    const int tile = s_tile;
+    const long long g0 = (long long)tile * kLLTile;
+    const long long g = g0 + tid;
+    const int w = tid >> 5, b = tid & 31;
+
+    int64_t ids[kMaxK];
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k) ids[k] = (g < p.G && k < p.K) ? __ldg(p.topk_idx + g * p.K + k) : -1;
+    bool bad = false;
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k) {
+        const int64_t e = ids[k];
+        if (e < -1 || e >= E) { bad = true; ids[k] = -1; continue; }
+        if (e >= 0) atomicOr(&bits[e * kLLStride + w], 1u << b);
+    }
+    if (bad) record_error(p.err, EP_ERR_BAD_TOPK);
     __syncthreads();
 
-    for (long long c0 = 0; c0 < p.G; c0 += kCountThreads) {
-        const long long g = c0 + tid;
-        uint32_t kmask = 0;
-        if (g < p.G) {
-            const int64_t* row = p.topk_idx + g * p.K;
-            for (int k = 0; k < p.K; ++k) {
-                const int64_t v = __ldg(row + k);
-                if (v == e) kmask |= 1u << k;
-                if (e == 0 && (v < -1 || v >= p.E)) record_error(p.err, EP_ERR_BAD_TOPK);
-            }
-        }
-        const bool member = kmask != 0;
-        const uint32_t b = __ballot_sync(kFullMask, member);
-        if (lane == 0) s_warp_total[warp] = __popc(b);
-        __syncthreads();
-        int warp_off = 0, block_total = 0;
-        for (int w = 0; w < kCountWarps; ++w) {
-            const int v = s_warp_total[w];
-            warp_off += (w < warp) ? v : 0;
-            block_total += v;
-        }
-        const int slot = s_base + warp_off + __popc(b & lanemask_lt());
-        if (g < p.G) {
-            const int t = (int)(g % p.T);
-            if (t == 0) s_begin[g / p.T] = slot;   // slots before this rank's first token
-            if (member) {
-                if (slot < cap) {
-                    src_info[slot] = t;
-                    for (int k = 0; k < p.K; ++k)
-                        if ((kmask >> k) & 1u) p.slot_map[g * p.K + k] = slot;
-                } else {
-                    record_error(p.err, EP_ERR_CAPACITY);
+    for (int e = tid; e < E; e += kLLTile) {
+        int agg = 0;
+#pragma unroll
+        for (int q = 0; q < kLLWords; ++q) agg += __popc(bits[e * kLLStride + q]);
+        unsigned long long* mine = p.status + (size_t)tile * E + e;
+        int excl = 0;
+        if (tile == 0) {
+            st_relaxed_u64(mine, kLLFlagInclusive | (unsigned)agg);
+        } else {
+            st_relaxed_u64(mine, kLLFlagAggregate | (unsigned)agg);
+            int j = tile - 1;
+            uint64_t t0 = 0;
+            uint32_t spins = 0;
+            while (j >= 0) {
+                const unsigned long long v = ld_relaxed_u64(p.status + (size_t)j * E + e);
+                const unsigned long long flag = v & (3ull << 62);
+                if (flag == 0) {
+                    if (spins == 0) t0 = globaltimer_ns();
+                    ++spins;
+                    if (spins > kWaitLimitIters ||
+                        ((spins & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs)) {
+                        record_error(p.err, EP_ERR_TIMEOUT);
+                        break;
+                    }
+                    continue;
                 }
+                excl += (int)(uint32_t)v;
+                if (flag == kLLFlagInclusive) break;
+                --j;
+            }
+            st_relaxed_u64(mine, kLLFlagInclusive | (unsigned)(excl + agg));
+        }
+        s_excl[e] = excl;
+    }
+    __syncthreads();
+
+    const long long cap = p.ll_capacity;
+    if (g < p.G) {
+        const int t = (int)(g % p.T);
+#pragma unroll
+        for (int k = 0; k < kMaxK; ++k) {
+            const int64_t e = ids[k];
+            if (e < 0) continue;
+            const uint32_t* be = bits + e * kLLStride;
+            int slot = s_excl[e] + __popc(be[w] & ((1u << b) - 1u));
+            for (int q = 0; q < w; ++q) slot += __popc(be[q]);
+            if (slot < cap) {
+                p.slot_map[g * p.K + k] = slot;
+                p.src_info[e * cap + slot] = t;
+            } else {
+                record_error(p.err, EP_ERR_CAPACITY);
             }
         }
-        __syncthreads();
-        if (tid == 0) s_base += block_total;
-        __syncthreads();
     }
-    if (tid == 0) s_begin[p.R] = s_base;
+
+    // running counts at source starts s*T (s = 0..R; s*T == G belongs to the last tile)
+    const bool last_tile = tile == p.num_tiles - 1;
+    const int s_lo = (int)((g0 + p.T - 1) / p.T);
+    const int s_hi = (int)min((long long)p.R, (g0 + kLLTile) / p.T);
+    for (int s = s_lo; s <= s_hi; ++s) {
+        const long long gb = (long long)s * p.T;
+        const bool mine = (gb >= g0 && gb < g0 + kLLTile && gb < p.G) || (gb == p.G && last_tile);
+        if (!mine) continue;
+        const int rel = (int)(gb - g0);    // 0..256
+        for (int e = tid; e < E; e += kLLTile) {
+            const uint32_t* be = bits + e * kLLStride;
+            int cnt = 0;
+            for (int q = 0; q < (rel >> 5); ++q) cnt += __popc(be[q]);
+            if ((rel >> 5) < kLLWords) cnt += __popc(be[rel >> 5] & ((1u << (rel & 31)) - 1u));
+            p.boundary[(long long)s * E + e] = s_excl[e] + cnt;
+        }
+    }
+
+    __threadfence();
     __syncthreads();
-    for (int s = tid; s < p.R; s += kCountThreads) {
-        p.layout_range[((long long)e * p.R + s) * 2 + 0] = s_begin[s];
-        p.layout_range[((long long)e * p.R + s) * 2 + 1] = s_begin[s + 1] - s_begin[s];
+    if (tid == 0) s_last = atomicAdd(p.done, 1) == p.num_tiles - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    // loads of each batch before its stores, so the L2 round trips overlap
+    constexpr int kBatch = 8;
+    const int nr = E * p.R;
+    for (int i0 = 0; i0 < nr; i0 += kLLTile * kBatch) {
+        int vb[kBatch], vn[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int i = i0 + u * kLLTile + tid;   // i = e*R + s
+            if (i < nr) {
+                const int e = i / p.R, s = i % p.R;
+                vb[u] = __ldcg(p.boundary + (long long)s * E + e);
+                vn[u] = __ldcg(p.boundary + (long long)(s + 1) * E + e);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int i = i0 + u * kLLTile + tid;
+            if (i < nr) {
+                p.layout_range[(long long)i * 2 + 0] = vb[u];
+                p.layout_range[(long long)i * 2 + 1] = vn[u] - vb[u];
+            }
+        }
     }
-    if (tid == 0) p.packed_recv_count[e] = s_base;
+    for (int e = tid; e < E; e += kLLTile) p.packed_recv_count[e] = __ldcg(p.boundary + (long long)p.R * E + e);
 }
 
 __device__ __forceinline__ void fma_bf16x8(float* acc, float w, const uint4& v) {
@@ -105,7 +193,7 @@ __device__ __forceinline__ void fma_bf16x8(float* acc, float w, const uint4& v) 
     acc[7] = __fmaf_rn(w, bf16_hi(v.w), acc[7]);
 }
 
-template <int U>
+template <int U, int kGroup = kLLRowsPerGroup>
 __global__ void __launch_bounds__(kLLCombineThreads)
 ll_combine_kernel(const LLCombineParams p) {
     __shared__ long long s_rows[kLLCombineWarps][32];
@@ -114,8 +202,11 @@ ll_combine_kernel(const LLCombineParams p) {
     const int nvec = p.H / 8;
     const long long cap = p.ll_capacity;
 
-    const long long stride = (long long)gridDim.x * kLLCombineWarps;
-    for (long long g = (long long)blockIdx.x * kLLCombineWarps + warp; g < p.G; g += stride) {
+    const long long wid = (long long)blockIdx.x * kLLCombineWarps + warp;
+    const long long g = wid / p.splits;          // token
+    const int part = (int)(wid % p.splits);      // column slice of its row
+    if (g >= p.G) return;   // whole warp
+    {
         const int s = (int)(g / p.T), t = (int)(g % p.T);
         long long e = -1;
         float w = 0.f;
@@ -157,39 +248,41 @@ ll_combine_kernel(const LLCombineParams p) {
         __syncwarp();
 
         uint4* out = reinterpret_cast<uint4*>(p.out_x + g * p.H);
-        for (int c0 = 0; c0 < nvec; c0 += 32 * U) {
+        const int per = ((nvec + p.splits - 1) / p.splits + 31) / 32 * 32;
+        const int clo = part * per, chi = min(nvec, clo + per);
+        for (int c0 = clo; c0 < chi; c0 += 32 * U) {
             float acc[U][8];
 #pragma unroll
             for (int u = 0; u < U; ++u)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
-            for (int i0 = 0; i0 < nv; i0 += kRowsPerGroup) {
-                uint4 v[kRowsPerGroup][U];
+            for (int i0 = 0; i0 < nv; i0 += kGroup) {
+                uint4 v[kGroup][U];
 #pragma unroll
-                for (int i = 0; i < kRowsPerGroup; ++i) {
+                for (int i = 0; i < kGroup; ++i) {
                     if (i0 + i < nv) {
                         const uint4* src = reinterpret_cast<const uint4*>(p.y + s_rows[warp][i0 + i] * p.H);
 #pragma unroll
                         for (int u = 0; u < U; ++u) {
                             const int c = c0 + lane + 32 * u;
-                            if (c < nvec) v[i][u] = ld_stream_v4(src + c);
+                            if (c < chi) v[i][u] = ld_stream_v4(src + c);
                         }
                     }
                 }
 #pragma unroll
-                for (int i = 0; i < kRowsPerGroup; ++i) {
+                for (int i = 0; i < kGroup; ++i) {
                     if (i0 + i < nv) {
                         const float wi = s_w[warp][i0 + i];
 #pragma unroll
                         for (int u = 0; u < U; ++u)
-                            if (c0 + lane + 32 * u < nvec) fma_bf16x8(acc[u], wi, v[i][u]);
+                            if (c0 + lane + 32 * u < chi) fma_bf16x8(acc[u], wi, v[i][u]);
                     }
                 }
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int c = c0 + lane + 32 * u;
-                if (c >= nvec) continue;
+                if (c >= chi) continue;
                 uint4 o;
                 o.x = pack_bf16x2_rn(acc[u][0], acc[u][1]);
                 o.y = pack_bf16x2_rn(acc[u][2], acc[u][3]);
@@ -204,19 +297,36 @@ ll_combine_kernel(const LLCombineParams p) {
 
 }  // namespace
 
+cudaError_t ll_prepare(int E) {
+    // opt in to large dynamic shared memory when E needs it
+    const size_t smem = ll_scan_smem(E);
+    if (smem <= 48 * 1024) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(ll_scan_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(ll_scan_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(ll_scan_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    return e;
+}
+
 cudaError_t launch_ll_count(const LLCountParams& p, cudaStream_t stream) {
     if (p.G == 0 || p.E == 0) return cudaSuccess;
-    ll_count_kernel<<<p.E, kCountThreads, 0, stream>>>(p);
+    const size_t smem = ll_scan_smem(p.E);
+    if (p.K <= 8)
+        ll_scan_kernel<8><<<p.num_tiles, kLLTile, smem, stream>>>(p);
+    else if (p.K <= 16)
+        ll_scan_kernel<16><<<p.num_tiles, kLLTile, smem, stream>>>(p);
+    else
+        ll_scan_kernel<32><<<p.num_tiles, kLLTile, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_ll_combine(const LLCombineParams& p, int num_sms, cudaStream_t stream) {
     if (p.G == 0) return cudaSuccess;
-    constexpr int U = 2;
-    long long blocks = (p.G + kLLCombineWarps - 1) / kLLCombineWarps;
-    const long long cap = (long long)num_sms * 4;
-    if (blocks > cap) blocks = cap;
-    ll_combine_kernel<U><<<(int)blocks, kLLCombineThreads, 0, stream>>>(p);
+    (void)num_sms;
+    const long long blocks = (p.G * p.splits + kLLCombineWarps - 1) / kLLCombineWarps;
+    // 4 x 16-byte vectors per lane per row, groups of 4 rows (measured best on B200)
+    ll_combine_kernel<4, 4><<<(unsigned)blocks, kLLCombineThreads, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -17,7 +17,10 @@
 // Each 256-token tile turns its tokens' membership into per-column bit words
 // (warp ballots), publishes its column counts, and finds its exclusive prefix
 // by looking back over earlier tiles (flags: aggregate / inclusive), one lane
-// per column.  Tiles are numbered by an atomic ticket in start order, so a
+// per column.  A flag and its count share one 64-bit word, and nothing else is
+// read on the strength of a flag, so relaxed (not acquire/release) accesses
+// suffice; the finishing tile's reads of the boundary samples are ordered by
+// a fence and the finish counter.  Tiles are numbered by an atomic ticket in start order, so a
 // tile only ever waits on tiles that are already running; every wait is
 // bounded (EP_ERR_TIMEOUT).  The tile then writes send_head and the channel
 // boundary samples; the last tile to finish (atomic counter) assembles the
@@ -84,14 +87,14 @@ scan_kernel(const ScanParams p) {
         unsigned long long* mine = p.status + (size_t)tile * R + lane;
         int excl = 0;
         if (tile == 0) {
-            st_release_u64(mine, kFlagInclusive | (unsigned)agg);
+            st_relaxed_u64(mine, kFlagInclusive | (unsigned)agg);
         } else {
-            st_release_u64(mine, kFlagAggregate | (unsigned)agg);
+            st_relaxed_u64(mine, kFlagAggregate | (unsigned)agg);
             int j = tile - 1;
             uint64_t t0 = 0;
             uint32_t spins = 0;
             while (j >= 0) {
-                const unsigned long long v = ld_acquire_u64(p.status + (size_t)j * R + lane);
+                const unsigned long long v = ld_relaxed_u64(p.status + (size_t)j * R + lane);
                 const unsigned long long flag = v & (3ull << 62);
                 if (flag == 0) {
                     if (spins == 0) t0 = globaltimer_ns();
@@ -107,7 +110,7 @@ scan_kernel(const ScanParams p) {
                 if (flag == kFlagInclusive) break;
                 --j;
             }
-            st_release_u64(mine, kFlagInclusive | (unsigned)(excl + agg));
+            st_relaxed_u64(mine, kFlagInclusive | (unsigned)(excl + agg));
         }
         s_excl[lane] = excl;
     }
@@ -154,31 +157,61 @@ scan_kernel(const ScanParams p) {
     if (!s_last) return;
     __threadfence();
 
+    // Loads of each batch are issued before its stores (independent L2 round
+    // trips overlap; a store between loads would serialise them).
     const int C = p.C;
     const int* bp = p.boundary;
     auto B = [&](int s, int c, int d) { return __ldcg(bp + ((long long)s * (C + 1) + c) * R + d); };
-    for (int i = tid; i < R * R * C; i += kScanTile) {
-        // i enumerates [d][s][c]
-        const int c = i % C, s = (i / C) % R, d = i / (C * R);
-        p.recv_channel_prefix_matrix[i] = B(s, c, d);
-        p.channel_prefix_matrix[((long long)s * R + d) * C + c] = B(s, c + 1, d) - B(s, 0, d);
+    constexpr int kBatch = 8;
+    const int nm = R * R * C;
+    for (int i0 = 0; i0 < nm; i0 += kScanTile * kBatch) {
+        int vc[kBatch], vn[kBatch], v0[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int i = i0 + u * kScanTile + tid;   // i enumerates [d][s][c]
+            if (i < nm) {
+                const int c = i % C, s = (i / C) % R, d = i / (C * R);
+                vc[u] = B(s, c, d);
+                vn[u] = B(s, c + 1, d);
+                v0[u] = B(s, 0, d);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int i = i0 + u * kScanTile + tid;
+            if (i < nm) {
+                const int c = i % C, s = (i / C) % R, d = i / (C * R);
+                p.recv_channel_prefix_matrix[i] = vc[u];
+                p.channel_prefix_matrix[((long long)s * R + d) * C + c] = vn[u] - v0[u];
+            }
+        }
     }
     for (int i = tid; i < R * R; i += kScanTile) {
         const int s = i / R, d = i % R;
         p.rank_prefix_matrix[i] = B(s, C, d);
     }
+    __shared__ long long s_total[32];
+    if (tid < R) s_total[tid] = B(R - 1, C, tid);
+    __syncthreads();
     if (tid == 0) {
         long long off = 0;
         for (int d = 0; d < R; ++d) {
             p.recv_rank_offset[d] = off;
-            off += B(R - 1, C, d);
+            off += s_total[d];
         }
         p.recv_rank_offset[R] = off;
     }
     for (int i = tid; i < p.E; i += kScanTile) {
-        // i = d*L + j
+        // i = d*L + j: sum over sources, 8 independent loads per round
+        int part[kBatch] = {0, 0, 0, 0, 0, 0, 0, 0};
+        for (int s0 = 0; s0 < R; s0 += kBatch) {
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u)
+                if (s0 + u < R) part[u] += __ldcg(p.num_tokens_per_expert + (long long)(s0 + u) * p.E + i);
+        }
         int sum = 0;
-        for (int s = 0; s < R; ++s) sum += __ldcg(p.num_tokens_per_expert + (long long)s * p.E + i);
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) sum += part[u];
         p.num_recv_tokens_per_expert[i] = sum;
     }
 }

@@ -297,7 +297,8 @@ EP_API int ep_dispatch_handle_static(int32_t num_ranks, int32_t num_experts, int
                                      int32_t* error_word, ep_stream_t stream);
 
 /* Optional per-kernel timing (CUDA events around each launch on the call's
- * stream).  ep_profile_read synchronizes the recorded events and returns,
+ * stream; inside a stream capture they become event-record nodes, recorded
+ * each time the graph runs).  ep_profile_read synchronizes the recorded events and returns,
  * per kernel kind, the number of launches and total milliseconds since the
  * last read; kinds: 0 layout, 1 scan (handle), 2 dispatch, 3 cached dispatch,
  * 4 combine, 5 ll count, 6 ll copy, 7 ll combine. */

@@ -29,28 +29,33 @@ class OracleError(RuntimeError):
     pass
 
 
+def load_library(path: str):
+    """Load an oracle build from `path` and declare its C signatures."""
+    L = ctypes.CDLL(path)
+    L.oracle_round_bf16.argtypes = [_ptr, _ptr, _c_i64]
+    L.oracle_round_bf16.restype = None
+    L.oracle_layout.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _ptr, _ptr, _ptr, _ptr]
+    L.oracle_dispatch_handle.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _ptr, _ptr,
+                                             _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _c_i64]
+    L.oracle_dispatch_rows.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
+                                           _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr]
+    L.oracle_combine.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _ptr, _c_i64, _ptr, _ptr,
+                                     _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _c_i64]
+    L.oracle_ll_dispatch.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
+                                         _ptr, _ptr, _ptr, _ptr, _ptr, _ptr]
+    L.oracle_ll_combine.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
+                                        _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _c_i64]
+    for name in ("oracle_layout", "oracle_dispatch_handle", "oracle_dispatch_rows",
+                 "oracle_combine", "oracle_ll_dispatch", "oracle_ll_combine"):
+        getattr(L, name).restype = ctypes.c_int
+    return L
+
+
 def lib():
+    """The oracle library (EP_ORACLE_LIB may name another build, e.g. a planted mutant)."""
     global _LIB
     if _LIB is None:
-        path = _build.build()
-        L = ctypes.CDLL(path)
-        L.oracle_round_bf16.argtypes = [_ptr, _ptr, _c_i64]
-        L.oracle_round_bf16.restype = None
-        L.oracle_layout.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _ptr, _ptr, _ptr, _ptr]
-        L.oracle_dispatch_handle.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _ptr, _ptr,
-                                             _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _c_i64]
-        L.oracle_dispatch_rows.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
-                                           _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr]
-        L.oracle_combine.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _ptr, _c_i64, _ptr, _ptr,
-                                     _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _c_i64]
-        L.oracle_ll_dispatch.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
-                                         _ptr, _ptr, _ptr, _ptr, _ptr, _ptr]
-        L.oracle_ll_combine.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
-                                        _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _c_i64]
-        for name in ("oracle_layout", "oracle_dispatch_handle", "oracle_dispatch_rows",
-                     "oracle_combine", "oracle_ll_dispatch", "oracle_ll_combine"):
-            getattr(L, name).restype = ctypes.c_int
-        _LIB = L
+        _LIB = load_library(os.environ.get("EP_ORACLE_LIB") or _build.build())
     return _LIB
 
 

@@ -124,6 +124,9 @@ LL_CASES = [
     dataclasses.replace(W["ll"].scaled(num_tokens=50, hidden=256), max_tokens_per_rank=64,
                         name="ll-tmax64"),
     synth.Workload("ll-odd", 3, 12, 30, 40, 5, "uniform_masked", 95, mask_prob=0.2),
+    # more than 4096 tokens, and more than 16 slots: the tiled lookback slot scan
+    synth.Workload("ll-big", 32, 256, 160, 64, 8, "uniform", 94),
+    synth.Workload("ll-k20", 4, 64, 50, 32, 20, "uniform_masked", 93, mask_prob=0.1),
 ]
 
 
