@@ -283,9 +283,10 @@ class Path:
             self.count = torch.empty((R, L), dtype=torch.int32, device=dev)
             self.src_info = torch.empty((R, L, cap), dtype=torch.int32, device=dev)
             self.layout_range = torch.empty((R, L, R, 2), dtype=torch.int32, device=dev)
-            valid = topk_d >= 0
-            S = int(torch.stack([(topk_d == e).any(-1) for e in range(E)]).sum().item()) \
-                if E <= 1024 else int(valid.sum().item())
+            # valid (token, expert) pairs, a token counted once per expert (host-side count)
+            t = np.sort(topk_d.cpu().numpy().reshape(-1, K), axis=1)
+            S = int(((t >= 0) & np.concatenate([np.ones((t.shape[0], 1), bool),
+                                                t[:, 1:] != t[:, :-1]], axis=1)).sum())
             self.N = S
             self.bytes = {"ll_count": G * K * 12 + S * 4 + E * R * 8,
                           "ll_copy": X + G * K * 12 + S * H * 2,
