@@ -45,8 +45,12 @@ def load_library(path: str):
                                          _ptr, _ptr, _ptr, _ptr, _ptr, _ptr]
     L.oracle_ll_combine.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
                                         _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _c_i64]
+    L.oracle_fp8_e4m3_encode.argtypes = [_ptr, _ptr, _c_i64]
+    L.oracle_fp8_e4m3_encode.restype = None
+    L.oracle_quantize_e4m3_blocks.argtypes = [_ptr, _c_i64, _c_i32, _c_i32, _ptr, _ptr]
     for name in ("oracle_layout", "oracle_dispatch_handle", "oracle_dispatch_rows",
-                 "oracle_combine", "oracle_ll_dispatch", "oracle_ll_combine"):
+                 "oracle_combine", "oracle_ll_dispatch", "oracle_ll_combine",
+                 "oracle_quantize_e4m3_blocks"):
         getattr(L, name).restype = ctypes.c_int
     return L
 
@@ -210,3 +214,22 @@ def ll_combine(y, topk_idx, topk_weights, src_info, layout_range, num_experts: i
         _p(np.ascontiguousarray(layout_range, dtype=np.int32)), _p(out), _p(tok),
         0 if tok is None else tok.size), "oracle_ll_combine")
     return out.reshape(R, T, H) if tok is None else out
+
+
+def fp8_e4m3_encode(values: np.ndarray) -> np.ndarray:
+    v = np.ascontiguousarray(values, dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().oracle_fp8_e4m3_encode(_p(v), _p(out), v.size)
+    return out
+
+
+def quantize_e4m3_blocks(rows: np.ndarray, block: int = 128):
+    """rows [..., H] uint16 (bf16 bits) -> (codes [..., H] u8, scales [..., H/block] f32)."""
+    r = np.ascontiguousarray(rows, dtype=np.uint16)
+    H = r.shape[-1]
+    n = r.size // H
+    codes = np.empty(r.shape, np.uint8)
+    scales = np.empty(r.shape[:-1] + (H // block,), np.float32)
+    _check(lib().oracle_quantize_e4m3_blocks(_p(r), n, H, block, _p(codes), _p(scales)),
+           "oracle_quantize_e4m3_blocks")
+    return codes, scales

@@ -421,4 +421,69 @@ int oracle_ll_combine(int32_t R, int32_t E, int32_t T, int32_t K, int32_t H, int
     return ORACLE_OK;
 }
 
+// ---------------------------------------------------------------- FP8 (LL)
+//
+// [API] "IB-GDA Kernels" / "Low-Latency Inference with FP8": the low-latency
+// path can quantise to FP8 (use_fp8), and the packed result becomes a tuple
+// (the example indexes packed_x[0]).  The pages give no format; the reading
+// taken: OCP FP8 E4M3 (bias 7, 3 mantissa bits, largest finite 448, no
+// infinities), one fp32 scale per token per block of 128 hidden channels,
+//   scale = amax(|x| over the block) / 448      (fp32 division, nearest even;
+//                                                 1 when the block is all zero)
+//   code  = e4m3(x / scale)                       (fp32 division, then nearest
+//                                                 even, saturating at +-448)
+// so x ~= value(code) * scale.
+
+// E4M3 code of a finite value, round to nearest even, saturating at +-448.
+static uint8_t e4m3_encode(double v) {
+    const uint8_t sign = std::signbit(v) ? 0x80 : 0x00;
+    double a = std::fabs(v);
+    if (a == 0.0) return sign;
+    // spacing of E4M3 values at a: 2^(e-3) for a in [2^e, 2^(e+1)), e >= -6;
+    // subnormals (a < 2^-6) step by 2^-9
+    int e;
+    std::frexp(a, &e);                   // a = m * 2^e, m in [0.5, 1): leading bit 2^(e-1)
+    int qexp = (e - 1) - 3;
+    if (qexp < -9) qexp = -9;
+    double r = std::ldexp(std::nearbyint(std::ldexp(a, -qexp)), qexp);
+    if (r > 448.0) r = 448.0;            // saturate to the largest finite value
+    if (r == 0.0) return sign;
+    if (r < std::ldexp(1.0, -6)) {       // subnormal: exponent field 0
+        const int m = (int)std::ldexp(r, 9);
+        return (uint8_t)(sign | m);
+    }
+    int re;
+    std::frexp(r, &re);                  // r in [2^(re-1), 2^re)
+    const int E = (re - 1) + 7;
+    const int m = (int)(std::ldexp(r, -(re - 1)) * 8.0) - 8;
+    return (uint8_t)(sign | (E << 3) | m);
+}
+
+void oracle_fp8_e4m3_encode(const double* in, uint8_t* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_encode(in[i]);
+}
+
+// Quantise n bf16 rows of H channels in blocks of `block` channels:
+//   codes[r][c] (u8), scales[r][c / block] (f32).
+int oracle_quantize_e4m3_blocks(const uint16_t* rows, int64_t n, int32_t H, int32_t block,
+                                uint8_t* codes, float* scales) {
+    if (H < 1 || block < 1 || H % block != 0) return ORACLE_BAD_ARG;
+    const int32_t nb = H / block;
+    for (int64_t r = 0; r < n; ++r) {
+        for (int32_t b = 0; b < nb; ++b) {
+            float amax = 0.0f;
+            for (int32_t i = 0; i < block; ++i)
+                amax = std::max(amax, (float)std::fabs(bf16_bits_to_double(rows[r * H + b * block + i])));
+            const float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+            scales[r * nb + b] = scale;
+            for (int32_t i = 0; i < block; ++i) {
+                const float x = (float)bf16_bits_to_double(rows[r * H + b * block + i]);
+                const float q = x / scale;
+                codes[r * H + b * block + i] = e4m3_encode((double)q);
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
 }  // extern "C"

@@ -56,6 +56,11 @@ MUTANTS = {
     "ll layout range shifted": ("const int64_t begin = slot;", "const int64_t begin = slot + (s > 0);"),
     "expert count per token": (
         "num_tokens_per_expert[(int64_t)s * E + e] += 1;", "num_tokens_per_expert[(int64_t)s * E + e] = 1;"),
+    "fp8 scale uses the wrong range": (
+        "amax > 0.0f ? amax / 448.0f : 1.0f", "amax > 0.0f ? amax / 240.0f : 1.0f"),
+    "fp8 rounding truncates": (
+        "double r = std::ldexp(std::nearbyint(std::ldexp(a, -qexp)), qexp);",
+        "double r = std::ldexp(std::trunc(std::ldexp(a, -qexp)), qexp);"),
     "weights leak to other ranks": (
         "here ? topk_weights[g * K + k] : 0.0f;", "topk_weights[g * K + k];"),
 }

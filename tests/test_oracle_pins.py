@@ -504,3 +504,64 @@ def test_round_bf16_against_exact_and_torch():
     np.testing.assert_array_equal(got, exp)
     assert struct.pack(">H", int(oracle.round_bf16(np.array([1.0 + 2.0 ** -8 + 2.0 ** -40]))[0])) \
         == b"\x3f\x81"
+
+
+# ----------------------------------------------------------------------------
+# FP8 (E4M3) block quantisation of the low-latency path
+
+def _e4m3_values():
+    codes = np.arange(256, dtype=np.uint8)
+    vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    return codes, vals
+
+
+def test_e4m3_encoder_against_torch_and_ties():
+    rng = np.random.default_rng(4)
+    v32 = np.concatenate([rng.uniform(-448, 448, 50000), rng.standard_normal(50000) * 0.02]).astype(np.float32)
+    np.testing.assert_array_equal(oracle.fp8_e4m3_encode(v32.astype(np.float64)),
+                                  torch.from_numpy(v32).to(torch.float8_e4m3fn).view(torch.uint8).numpy())
+    codes, vals = _e4m3_values()
+    finite = ~np.isnan(vals)
+    np.testing.assert_array_equal(oracle.fp8_e4m3_encode(vals[finite]), codes[finite])
+    # exact midpoints between neighbouring positive values round to the even code
+    pos = np.sort(vals[finite & (vals > 0)])
+    mids = (pos[:-1] + pos[1:]) / 2
+    got = oracle.fp8_e4m3_encode(mids)
+    lo = oracle.fp8_e4m3_encode(pos[:-1])
+    hi = oracle.fp8_e4m3_encode(pos[1:])
+    np.testing.assert_array_equal(got, np.where(lo % 2 == 0, lo, hi))
+    # saturation at the largest finite value, both signs
+    assert oracle.fp8_e4m3_encode(np.array([448.0, 463.9, 1e6, -1e6])).tolist() == [0x7E, 0x7E, 0x7E, 0xFE]
+
+
+def test_block_quantisation_closed_forms():
+    H = 256
+    # block 0: amax 56 -> scale 0.125 exactly; codes are e4m3(8 x) with 8 x exact in E4M3
+    b0 = np.array([56.0, -56.0, 1.0, -0.5, 0.25, 3.0, 0.0, 7.0] * 16, np.float32)
+    # block 1: all zero -> scale 1, codes 0
+    b1 = np.zeros(128, np.float32)
+    x = f32_to_bf16_torch(np.concatenate([b0, b1])[None, :])
+    codes, scales = oracle.quantize_e4m3_blocks(x, 128)
+    assert scales.tolist() == [[0.125, 1.0]]
+    np.testing.assert_array_equal(codes[0, :128], oracle.fp8_e4m3_encode(8.0 * b0.astype(np.float64)))
+    assert codes[0, 0] == 0x7E and codes[0, 1] == 0xFE          # amax maps to +-448
+    assert not codes[0, 128:].any()
+
+
+def test_block_quantisation_error_bound():
+    rng = np.random.default_rng(9)
+    x = f32_to_bf16_torch(rng.standard_normal((64, 512)).astype(np.float32))
+    codes, scales = oracle.quantize_e4m3_blocks(x, 128)
+    _, vals = _e4m3_values()
+    deq = vals[codes] * np.repeat(scales.astype(np.float64), 128, axis=1)
+    xf = bf16_to_f64(x)
+    q = np.abs(xf) / np.repeat(scales.astype(np.float64), 128, axis=1)
+    e = np.floor(np.log2(np.maximum(q, 2.0 ** -6)))
+    half_step = 2.0 ** (e - 3) / 2 * np.repeat(scales.astype(np.float64), 128, axis=1)
+    assert (np.abs(deq - xf) <= half_step * (1 + 1e-6) + 1e-30).all()
+    # the largest element of each block is encoded as +-448
+    blocks = np.abs(xf).reshape(64, 4, 128)
+    arg = blocks.argmax(-1)
+    c = codes.reshape(64, 4, 128)
+    picked = np.take_along_axis(c, arg[..., None], -1)[..., 0]
+    assert np.isin(picked, [0x7E, 0xFE]).all()
