@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "EP_OK", 1: "EP_ERR_INVALID_ARG", 2: "EP_ERR_ALIGNMENT", 3: "
                 4: "EP_ERR_BAD_TOPK", 5: "EP_ERR_HANDLE_MISMATCH", 6: "EP_ERR_TIMEOUT",
                 7: "EP_ERR_CUDA", 8: "EP_ERR_UNIMPLEMENTED"}
 PROFILE_KINDS = ["layout", "scan", "dispatch", "dispatch_cached", "combine", "ll_count",
-                 "ll_copy", "ll_combine"]
+                 "ll_copy", "ll_combine", "ll_copy_fp8"]
 
 _vp = ctypes.c_void_p
 _i32 = ctypes.c_int32
@@ -75,6 +75,7 @@ _SIGNATURES = {
     "ep_combine": (ctypes.c_int, [_vp, _vp, _i64, ctypes.POINTER(ep_handle), _vp, _vp, _vp, _vp,
                                   _vp, _vp, _vp]),
     "ep_ll_dispatch": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "ep_ll_dispatch_fp8": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "ep_ll_combine": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "ep_profile_enable": (ctypes.c_int, [_vp, ctypes.c_int]),
     "ep_profile_read": (ctypes.c_int, [_vp, ctypes.POINTER(_i64), ctypes.POINTER(ctypes.c_double)]),
@@ -222,6 +223,14 @@ def ep_ll_dispatch(ctx, x, topk_idx, packed_recv_x, packed_recv_count, src_info,
                                  _stream(stream), _event(wait_event)), "ep_ll_dispatch", ctx)
 
 
+def ep_ll_dispatch_fp8(ctx, x, topk_idx, packed_recv_x_fp8, packed_recv_scales, packed_recv_count,
+                       src_info, layout_range, stream=None, wait_event=None):
+    _check(load().ep_ll_dispatch_fp8(ctx, _ptr(x), _ptr(topk_idx), _ptr(packed_recv_x_fp8),
+                                     _ptr(packed_recv_scales), _ptr(packed_recv_count), _ptr(src_info),
+                                     _ptr(layout_range), _stream(stream), _event(wait_event)),
+           "ep_ll_dispatch_fp8", ctx)
+
+
 def ep_ll_combine(ctx, y, topk_idx, topk_weights, src_info, layout_range, out_x, stream=None,
                   wait_event=None):
     _check(load().ep_ll_combine(ctx, _ptr(y), _ptr(topk_idx), _ptr(topk_weights), _ptr(src_info),
@@ -234,8 +243,8 @@ def ep_profile_enable(ctx, enable: bool = True):
 
 
 def ep_profile_read(ctx) -> dict:
-    n = (_i64 * 8)()
-    ms = (ctypes.c_double * 8)()
+    n = (_i64 * len(PROFILE_KINDS))()
+    ms = (ctypes.c_double * len(PROFILE_KINDS))()
     _check(load().ep_profile_read(ctx, n, ms), "ep_profile_read", ctx)
     return {k: (int(n[i]), float(ms[i])) for i, k in enumerate(PROFILE_KINDS)}
 
@@ -326,12 +335,18 @@ class Buffer:
                    stream)
         return out, out_w
 
-    def low_latency_dispatch(self, x, topk_idx, stream=None):
+    def low_latency_dispatch(self, x, topk_idx, use_fp8=False, stream=None):
+        """Returns (packed, count, handle); with use_fp8, packed is (codes u8, scales f32)."""
         cap = self.R * self.Tmax
-        packed = torch.empty((self.R, self.L, cap, self.H), dtype=torch.bfloat16, device=self.device)
         count = torch.empty((self.R, self.L), dtype=torch.int32, device=self.device)
         src_info = torch.empty((self.R, self.L, cap), dtype=torch.int32, device=self.device)
         layout_range = torch.empty((self.R, self.L, self.R, 2), dtype=torch.int32, device=self.device)
+        if use_fp8:
+            codes = torch.empty((self.R, self.L, cap, self.H), dtype=torch.uint8, device=self.device)
+            scales = torch.empty((self.R, self.L, cap, self.H // 128), dtype=torch.float32, device=self.device)
+            ep_ll_dispatch_fp8(self.ctx, x, topk_idx, codes, scales, count, src_info, layout_range, stream)
+            return (codes, scales), count, (src_info, layout_range)
+        packed = torch.empty((self.R, self.L, cap, self.H), dtype=torch.bfloat16, device=self.device)
         ep_ll_dispatch(self.ctx, x, topk_idx, packed, count, src_info, layout_range, stream)
         return packed, count, (src_info, layout_range)
 

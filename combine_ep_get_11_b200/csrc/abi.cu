@@ -8,7 +8,7 @@
 //                            [+ one host read of N] + dispatch_kernel<normal>
 //   ep_dispatch_cached     : dispatch_kernel<cached>
 //   ep_combine             : combine_kernel
-//   ep_ll_dispatch         : memset(LL scan state) + ll_scan_kernel + dispatch_kernel<packed>
+//   ep_ll_dispatch[_fp8]   : memset(LL scan state) + ll_scan_kernel + dispatch_kernel<packed[, FP8]>
 //   ep_ll_combine          : ll_combine_kernel
 
 #include <atomic>
@@ -65,7 +65,7 @@ namespace {
 std::atomic<uint64_t> g_launches{0};
 
 enum Kind { kLayout = 0, kScan = 1, kDispatch = 2, kCached = 3, kCombine = 4,
-            kLLCount = 5, kLLCopy = 6, kLLCombine = 7 };
+            kLLCount = 5, kLLCopy = 6, kLLCombine = 7, kLLCopyFp8 = 8 };
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
@@ -525,16 +525,25 @@ int ep_combine(ep_ctx* c, const uint16_t* y, int64_t num_recv_rows, const ep_han
     return launch(c, kCombine, c->G > 0, s, [&] { return ep::launch_combine(p, c->num_sms, s); });
 }
 
-int ep_ll_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint16_t* packed_recv_x,
-                   int32_t* packed_recv_count, int32_t* src_info, int32_t* layout_range,
-                   ep_stream_t stream, ep_event_t wait_event) {
+}  // extern "C"
+
+namespace {
+
+int ll_dispatch_impl(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint16_t* packed_recv_x,
+                     uint8_t* packed_fp8, float* packed_scales, int32_t* packed_recv_count,
+                     int32_t* src_info, int32_t* layout_range, ep_stream_t stream, ep_event_t wait_event) {
     if (c == nullptr) return EP_ERR_INVALID_ARG;
+    const bool fp8 = packed_fp8 != nullptr || packed_scales != nullptr;
     if (packed_recv_count == nullptr || layout_range == nullptr || src_info == nullptr)
         return fail(c, EP_ERR_INVALID_ARG, "low-latency outputs missing");
-    if (c->G > 0 && (x == nullptr || topk_idx == nullptr || packed_recv_x == nullptr))
-        return fail(c, EP_ERR_INVALID_ARG, "x / topk_idx / packed_recv_x missing");
-    if (!aligned16(x) || !aligned16(packed_recv_x)) return fail(c, EP_ERR_ALIGNMENT, "row buffers must be 16-byte aligned");
-    if (!aligned(topk_idx, 8)) return fail(c, EP_ERR_ALIGNMENT, "topk_idx misaligned");
+    if (fp8 && c->H % ep::kFp8Block != 0)
+        return fail(c, EP_ERR_INVALID_ARG, "FP8 packing needs hidden %% 128 == 0");
+    if (c->G > 0 && (x == nullptr || topk_idx == nullptr ||
+                     (fp8 ? (packed_fp8 == nullptr || packed_scales == nullptr) : packed_recv_x == nullptr)))
+        return fail(c, EP_ERR_INVALID_ARG, "x / topk_idx / packed outputs missing");
+    if (!aligned16(x) || !aligned16(packed_recv_x) || !aligned16(packed_fp8))
+        return fail(c, EP_ERR_ALIGNMENT, "row buffers must be 16-byte aligned");
+    if (!aligned(topk_idx, 8) || !aligned(packed_scales, 4)) return fail(c, EP_ERR_ALIGNMENT, "array misaligned");
     DeviceGuard guard(c->device);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     int rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
@@ -557,11 +566,36 @@ int ep_ll_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint16
     dp.slot_map = c->slot_map;
     dp.ll_capacity = c->ll_cap;
     dp.recv_x = packed_recv_x;
+    dp.recv_fp8 = packed_fp8;
+    dp.recv_scales = packed_scales;
     dp.err = c->err;
     dp.G = c->G;
     dp.R = c->R; dp.E = c->E; dp.L = c->L; dp.T = c->T; dp.K = c->K; dp.H = c->H;
     dp.splits = ep::dispatch_splits(c->H);
-    return launch(c, kLLCopy, true, s, [&] { return ep::launch_dispatch(ep::kModeLowLatency, dp, s); });
+    const int mode = fp8 ? ep::kModeLowLatencyFp8 : ep::kModeLowLatency;
+    return launch(c, fp8 ? kLLCopyFp8 : kLLCopy, true, s, [&] { return ep::launch_dispatch(mode, dp, s); });
+}
+
+}  // namespace
+
+extern "C" {
+
+int ep_ll_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint16_t* packed_recv_x,
+                   int32_t* packed_recv_count, int32_t* src_info, int32_t* layout_range,
+                   ep_stream_t stream, ep_event_t wait_event) {
+    if (c != nullptr && c->G > 0 && packed_recv_x == nullptr)
+        return fail(c, EP_ERR_INVALID_ARG, "packed_recv_x missing");
+    return ll_dispatch_impl(c, x, topk_idx, packed_recv_x, nullptr, nullptr, packed_recv_count, src_info,
+                            layout_range, stream, wait_event);
+}
+
+int ep_ll_dispatch_fp8(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint8_t* packed_recv_x_fp8,
+                       float* packed_recv_scales, int32_t* packed_recv_count, int32_t* src_info,
+                       int32_t* layout_range, ep_stream_t stream, ep_event_t wait_event) {
+    if (c != nullptr && c->G > 0 && (packed_recv_x_fp8 == nullptr || packed_recv_scales == nullptr))
+        return fail(c, EP_ERR_INVALID_ARG, "FP8 outputs missing");
+    return ll_dispatch_impl(c, x, topk_idx, nullptr, packed_recv_x_fp8, packed_recv_scales, packed_recv_count,
+                            src_info, layout_range, stream, wait_event);
 }
 
 int ep_ll_combine(ep_ctx* c, const uint16_t* y, const int64_t* topk_idx, const float* topk_weights,

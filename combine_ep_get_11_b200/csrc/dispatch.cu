@@ -26,9 +26,12 @@
 //     resolves its destination row; a ballot compacts the rows in lane order;
 //   * in the normal form the destination lanes also write the receive
 //     metadata: local top-k ids, weights, and recv_src_idx.
-// Per token the HBM traffic is H*2 bytes read + fan-out * H*2 bytes written.
+// Per token the HBM traffic is H*2 bytes read + fan-out * H*2 bytes written
+// (fan-out * (H + H/32) bytes in the FP8 packed form).
 
 #include <algorithm>
+
+#include <cuda_fp8.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -51,8 +54,9 @@ dispatch_kernel(const DispatchParams p) {
     const int part = (int)(wid % p.splits);      // column slice of its row
     if (g >= p.G) return;   // whole warp
 
+    constexpr bool kPacked = kMode == kModeLowLatency || kMode == kModeLowLatencyFp8;
     long long row = -1;
-    if (kMode == kModeLowLatency) {
+    if (kPacked) {
         long long e = -1;
         if (lane < p.K) e = p.topk_idx[g * p.K + lane];
         bool valid = e >= 0 && e < p.E;
@@ -110,6 +114,62 @@ dispatch_kernel(const DispatchParams p) {
     const int per = ((nvec + p.splits - 1) / p.splits + 31) / 32 * 32;
     const int lo = part * per, hi = min(nvec, lo + per);
     const uint4* src = reinterpret_cast<const uint4*>(p.x + g * p.H);
+    if (kMode == kModeLowLatencyFp8) {
+        // Each half-warp holds 16 vectors = one 128-channel block: amax by xor
+        // shuffles within the half, scale = amax / 448, codes = E4M3(x / scale)
+        // (round to nearest even, saturating), 8 code bytes per lane per vector.
+        const int nblk = p.H / kFp8Block;
+        for (int c0 = lo; c0 < hi; c0 += 32 * kVec) {
+            uint4 v[kVec];
+#pragma unroll
+            for (int u = 0; u < kVec; ++u) {
+                const int c = c0 + lane + 32 * u;
+                if (c < hi) v[u] = ld_nc_v4(src + c);
+            }
+#pragma unroll
+            for (int u = 0; u < kVec; ++u) {
+                const int c = c0 + lane + 32 * u;
+                if (c0 + 32 * u >= hi) break;               // warp-uniform
+                float xs[8];
+                xs[0] = bf16_lo(v[u].x); xs[1] = bf16_hi(v[u].x);
+                xs[2] = bf16_lo(v[u].y); xs[3] = bf16_hi(v[u].y);
+                xs[4] = bf16_lo(v[u].z); xs[5] = bf16_hi(v[u].z);
+                xs[6] = bf16_lo(v[u].w); xs[7] = bf16_hi(v[u].w);
+                float m = 0.f;
+                if (c < hi) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(xs[i]));
+                }
+                m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 8));
+                m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 4));
+                m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 2));
+                m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 1));
+                const float scale = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
+                uint32_t packed[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t word = 0;
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const float2 q = make_float2(__fdiv_rn(xs[4 * h + 2 * i], scale),
+                                                     __fdiv_rn(xs[4 * h + 2 * i + 1], scale));
+                        const __nv_fp8x2_storage_t pair = __nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
+                        word |= (uint32_t)pair << (16 * i);
+                    }
+                    packed[h] = word;
+                }
+                if (c < hi) {
+                    const uint2 codes = make_uint2(packed[0], packed[1]);
+                    for (int i = 0; i < f; ++i) {
+                        const long long r = s_rows[warp][i];
+                        *reinterpret_cast<uint2*>(p.recv_fp8 + r * p.H + (long long)c * 8) = codes;
+                        if ((lane & 15) == 0) p.recv_scales[r * nblk + c / 16] = scale;
+                    }
+                }
+            }
+        }
+        return;
+    }
     for (int c0 = lo; c0 < hi; c0 += 32 * kVec) {
         uint4 v[kVec];
 #pragma unroll
@@ -131,7 +191,9 @@ dispatch_kernel(const DispatchParams p) {
 template <int kMode>
 cudaError_t launch_mode(const DispatchParams& p, cudaStream_t stream) {
     const long long blocks = (p.G * p.splits + kDispatchWarps - 1) / kDispatchWarps;
-    dispatch_kernel<kMode><<<(unsigned)blocks, kDispatchThreads, 0, stream>>>(p);
+    // the FP8 form also keeps the codes and scales live: hold 14 vectors per pass
+    constexpr int kVec = kMode == kModeLowLatencyFp8 ? 14 : kVecPerLane;
+    dispatch_kernel<kMode, kVec><<<(unsigned)blocks, kDispatchThreads, 0, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -143,6 +205,7 @@ cudaError_t launch_dispatch(int mode, const DispatchParams& p, cudaStream_t stre
         case kModeNormal: return launch_mode<kModeNormal>(p, stream);
         case kModeCached: return launch_mode<kModeCached>(p, stream);
         case kModeLowLatency: return launch_mode<kModeLowLatency>(p, stream);
+        case kModeLowLatencyFp8: return launch_mode<kModeLowLatencyFp8>(p, stream);
         default: return cudaErrorInvalidValue;
     }
 }

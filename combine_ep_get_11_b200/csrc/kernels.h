@@ -53,7 +53,8 @@ constexpr int kScanTile = 256;   // tokens per tile == threads per block
 cudaError_t launch_scan(const ScanParams& p, cudaStream_t stream);
 
 // ---------------------------------------------------- dispatch (row copies)
-enum DispatchMode { kModeNormal = 0, kModeCached = 1, kModeLowLatency = 2 };
+enum DispatchMode { kModeNormal = 0, kModeCached = 1, kModeLowLatency = 2, kModeLowLatencyFp8 = 3 };
+constexpr int kFp8Block = 128;   // hidden channels per FP8 scale
 
 struct DispatchParams {
     const uint16_t* x;                 // [G][H]
@@ -71,6 +72,9 @@ struct DispatchParams {
     const int* slot_map;               // [G][K]
     int64_t ll_capacity;               // R * Tmax slots per expert
     uint16_t* recv_x;                  // normal/cached: [cap][H]; LL: [E][ll_cap][H]
+    // low latency, FP8 form (recv_x unused)
+    uint8_t* recv_fp8;                 // [E][ll_cap][H] E4M3 codes
+    float* recv_scales;                // [E][ll_cap][H/128]
     int* err;
     long long G;
     int R, E, L, T, K, H;

@@ -248,6 +248,21 @@ EP_API int ep_ll_dispatch(ep_ctx* ctx, const uint16_t* x, const int64_t* topk_id
                    int32_t* src_info, int32_t* layout_range,
                    ep_stream_t stream, ep_event_t wait_event);
 
+/* Low-latency dispatch with FP8 packing ([API] "IB-GDA Kernels", "Low-Latency
+ * Inference with FP8": use_fp8, the packed result becomes a pair).  Same
+ * packing, counts, src_info and layout_range as ep_ll_dispatch; each packed row
+ * is stored as OCP E4M3 codes with one fp32 scale per 128 hidden channels:
+ *   scale = amax(|x| over the block) / 448 (fp32, nearest even; 1 for an all-zero
+ *           block),  code = E4M3(x / scale) (fp32 division, nearest even,
+ *           saturating at +-448), so x ~= value(code) * scale.
+ *   packed_recv_x_fp8   u8  [R][L][R*Tmax][H]      out (16-byte aligned)
+ *   packed_recv_scales  f32 [R][L][R*Tmax][H/128]  out
+ * Requires H % 128 == 0 (EP_ERR_INVALID_ARG otherwise). */
+EP_API int ep_ll_dispatch_fp8(ep_ctx* ctx, const uint16_t* x, const int64_t* topk_idx,
+                              uint8_t* packed_recv_x_fp8, float* packed_recv_scales,
+                              int32_t* packed_recv_count, int32_t* src_info, int32_t* layout_range,
+                              ep_stream_t stream, ep_event_t wait_event);
+
 /* Low-latency combine ([API] "IB-GDA Kernels"): weighted reduction of expert
  * outputs back to token positions,
  *   out_x[s][t] = bf16( fp32 fused multiply-add chain, starting at 0, over the
@@ -301,8 +316,8 @@ EP_API int ep_dispatch_handle_static(int32_t num_ranks, int32_t num_experts, int
  * each time the graph runs).  ep_profile_read synchronizes the recorded events and returns,
  * per kernel kind, the number of launches and total milliseconds since the
  * last read; kinds: 0 layout, 1 scan (handle), 2 dispatch, 3 cached dispatch,
- * 4 combine, 5 ll count, 6 ll copy, 7 ll combine. */
-#define EP_PROFILE_KINDS 8
+ * 4 combine, 5 ll slots, 6 ll copy, 7 ll combine, 8 ll copy (FP8). */
+#define EP_PROFILE_KINDS 9
 EP_API int ep_profile_enable(ep_ctx* ctx, int enable);
 EP_API int ep_profile_read(ep_ctx* ctx, int64_t* launches, double* total_ms);
 

@@ -201,6 +201,22 @@ def test_low_latency_full(ep):
             s -= 1
         t = int(ll["src_info"][d, j, slot])
         np.testing.assert_array_equal(u16(packed[d, j, slot]), inp.x_u16[s, t])
+    # FP8 packing of the same slots: codes and scales of every valid slot bit-exact
+    (codes, scales), count8, (src8, lr8) = buf.low_latency_dispatch(inp.x_d, inp.topk_d, use_fp8=True)
+    assert buf.sync_status() == 0
+    np.testing.assert_array_equal(count8.cpu().numpy(), cnt)
+    np.testing.assert_array_equal(lr8.cpu().numpy(), lr)
+    cd, sc = codes.cpu().numpy(), scales.cpu().numpy()
+    for d in range(R):
+        for j in range(L):
+            n = int(cnt[d, j])
+            # the rows the oracle's lists name: slot p holds x[s][src_info[p]]
+            s_of = np.repeat(np.arange(R), lr[d, j, :, 1])
+            rows = inp.x_u16[s_of, ll["src_info"][d, j, :n]]
+            e_codes, e_scales = oracle.quantize_e4m3_blocks(rows, 128)
+            np.testing.assert_array_equal(cd[d, j, :n], e_codes)
+            np.testing.assert_array_equal(sc[d, j, :n], e_scales)
+    del codes, scales
     # identity experts, every token: out ~ x * sum of valid weights
     out = buf.low_latency_combine(packed, inp.topk_d, inp.weights_d, (src_info, layout_range))
     wsum = np.where(inp.topk != -1, inp.weights.astype(np.float64), 0.0).sum(-1)

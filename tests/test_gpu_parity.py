@@ -249,9 +249,48 @@ def test_profile_counts_every_kernel(ep):
     buf.dispatch_cached(inp.x_d, handle)
     packed, _, llh = buf.low_latency_dispatch(inp.x_d, inp.topk_d)
     buf.low_latency_combine(packed, inp.topk_d, inp.weights_d, llh)
+    buf.low_latency_dispatch(inp.x_d, inp.topk_d, use_fp8=True)
     prof = ep.ep_profile_read(buf.ctx)
-    assert ep.kernel_launch_count() - before == 8
+    assert ep.kernel_launch_count() - before == 10
     for kind in ep.PROFILE_KINDS:
         n, ms = prof[kind]
-        assert n == 1 and ms > 0, kind
+        assert n == (2 if kind == "ll_count" else 1) and ms > 0, kind
+    buf.destroy()
+
+
+FP8_CASES = [w for w in LL_CASES if w.hidden % 128 == 0]
+
+
+@pytest.mark.parametrize("w", FP8_CASES, ids=ids(FP8_CASES))
+def test_low_latency_fp8(ep, w):
+    """FP8 packing: same slots as the bf16 form; codes and scales bit-exact."""
+    inp = Inputs(w)
+    buf = make_buffer(ep, w)
+    (codes, scales), count, (src_info, layout_range) = buf.low_latency_dispatch(
+        inp.x_d, inp.topk_d, use_fp8=True)
+    assert buf.sync_status() == 0
+    ll = oracle.ll_dispatch(inp.x_u16, inp.topk, w.num_experts, w.tmax)
+    np.testing.assert_array_equal(count.cpu().numpy(), ll["packed_recv_count"])
+    np.testing.assert_array_equal(layout_range.cpu().numpy(), ll["layout_range"])
+    c, sc, si = codes.cpu().numpy(), scales.cpu().numpy(), src_info.cpu().numpy()
+    for d in range(w.num_ranks):
+        for j in range(w.local_experts):
+            n = int(ll["packed_recv_count"][d, j])
+            if n == 0:
+                continue
+            np.testing.assert_array_equal(si[d, j, :n], ll["src_info"][d, j, :n])
+            e_codes, e_scales = oracle.quantize_e4m3_blocks(ll["packed_recv_x"][d, j, :n], 128)
+            np.testing.assert_array_equal(c[d, j, :n], e_codes, err_msg=f"codes of expert ({d},{j})")
+            np.testing.assert_array_equal(sc[d, j, :n], e_scales, err_msg=f"scales of expert ({d},{j})")
+    buf.destroy()
+
+
+def test_low_latency_fp8_rejects_unaligned_hidden(ep):
+    w = LL_CASES[-3]            # hidden 40: not a multiple of 128
+    assert w.hidden % 128 != 0
+    inp = Inputs(w)
+    buf = make_buffer(ep, w)
+    with pytest.raises(ep.EpError) as e:
+        buf.low_latency_dispatch(inp.x_d, inp.topk_d, use_fp8=True)
+    assert e.value.status == 1
     buf.destroy()
