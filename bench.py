@@ -268,7 +268,7 @@ def config_dict(w, l2_note):
 class Path:
     """One workload's timed step: buffers, the step itself and its algorithmic bytes."""
 
-    def __init__(self, ep, w, dev, topk_d, wts_d, x_d):
+    def __init__(self, ep, w, dev, topk_d, wts_d, x_d, fp8=False):
         import torch
         self.ep, self.w, self.dev = ep, w, dev
         R, E, T, H, K, C = w.num_ranks, w.num_experts, w.num_tokens, w.hidden, w.topk, w.num_channels
@@ -278,6 +278,7 @@ class Path:
         self.out = torch.empty((R, T, H), dtype=torch.bfloat16, device=dev)
         self.out_w = None
         if w.name == "ll":
+            self.fp8 = fp8
             L, cap = E // R, R * w.tmax
             self.packed = torch.empty((R, L, cap, H), dtype=torch.bfloat16, device=dev)
             self.count = torch.empty((R, L), dtype=torch.int32, device=dev)
@@ -288,14 +289,25 @@ class Path:
             S = int(((t >= 0) & np.concatenate([np.ones((t.shape[0], 1), bool),
                                                 t[:, 1:] != t[:, :-1]], axis=1)).sum())
             self.N = S
+            copy_key = "ll_copy_fp8" if fp8 else "ll_copy"
+            row_bytes = H + (H // 128) * 4 if fp8 else H * 2
             self.bytes = {"ll_count": G * K * 12 + S * 4 + E * R * 8,
-                          "ll_copy": X + G * K * 12 + S * H * 2,
+                          copy_key: X + G * K * 12 + S * row_bytes,
                           "ll_combine": S * H * 2 + S * 4 + X + G * K * 12}
-            self.dominant = ("ll_copy", "ll_combine")
+            self.dominant = (copy_key, "ll_combine")
             self.inputs = ("x", "topk", "weights")
+            if fp8:
+                self.codes = torch.empty((R, L, cap, H), dtype=torch.uint8, device=dev)
+                self.scales = torch.empty((R, L, cap, H // 128), dtype=torch.float32, device=dev)
 
             def step(xd, td, wd):
-                ep.ep_ll_dispatch(ctx, xd, td, self.packed, self.count, self.src_info, self.layout_range)
+                if fp8:
+                    # experts would read the FP8 rows; their bf16 outputs sit in `packed`
+                    ep.ep_ll_dispatch_fp8(ctx, xd, td, self.codes, self.scales, self.count,
+                                          self.src_info, self.layout_range)
+                else:
+                    ep.ep_ll_dispatch(ctx, xd, td, self.packed, self.count, self.src_info,
+                                      self.layout_range)
                 ep.ep_ll_combine(ctx, self.packed, td, wd, self.src_info, self.layout_range, self.out)
             self.step = step
             return
@@ -355,7 +367,9 @@ def run_ours(args):
     wts_h = torch.from_numpy(synth.topk_weights(ww)).pin_memory()
     x_h = synth.hidden_rows(ww, pin_memory=True)
     topk_d, wts_d, x_d = topk_h.to(dev), wts_h.to(dev), x_h.to(dev)
-    path = Path(ep, w, dev, topk_d, wts_d, x_d)
+    if args.fp8 and w.name != "ll":
+        raise SystemExit("--fp8 applies to the low-latency workload only")
+    path = Path(ep, w, dev, topk_d, wts_d, x_d, fp8=args.fp8)
     buf, ctx, step = path.buf, path.ctx, path.step
     step_total = sum(path.bytes.values())
     stream = torch.cuda.current_stream(dev)
@@ -495,7 +509,8 @@ def run_ours(args):
             "us_per_step": round(ms / args.steps * 1e3, 2),
             "frac_of_peak_step": round(gbs / world / peak, 4),
             "frac_of_8tbs_step": round(gbs / world / 8000.0, 4),
-            "config": config_dict(w, l2_note=l2),
+            "config": dict(config_dict(w, l2_note=l2), **({"ll_packing": "fp8 e4m3, 128-channel fp32 scales"}
+                                                           if args.fp8 else {})),
             "num_recv_rows": path.N,
             "bytes_per_step": dict(path.bytes, step=step_total),
             "kernels": kernels,
@@ -524,6 +539,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-sample-tokens", type=int, default=CPU_SAMPLE_TOKENS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fp8", action="store_true",
+                    help="low-latency workload: FP8 (E4M3 + scales) dispatch packing")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="enqueue the timed steps eagerly instead of replaying one CUDA graph")
     ap.add_argument("--workload", choices=sorted(synth.WORKLOADS), default=WORKLOAD,

@@ -116,8 +116,9 @@ dispatch_kernel(const DispatchParams p) {
     const uint4* src = reinterpret_cast<const uint4*>(p.x + g * p.H);
     if (kMode == kModeLowLatencyFp8) {
         // Each half-warp holds 16 vectors = one 128-channel block: amax by xor
-        // shuffles within the half, scale = amax / 448, codes = E4M3(x / scale)
-        // (round to nearest even, saturating), 8 code bytes per lane per vector.
+        // shuffles within the half, scale = amax / 448, codes = E4M3(x * (448 /
+        // amax)) (round to nearest even, saturating), 8 code bytes per lane per
+        // vector.
         const int nblk = p.H / kFp8Block;
         for (int c0 = lo; c0 < hi; c0 += 32 * kVec) {
             uint4 v[kVec];
@@ -145,14 +146,15 @@ dispatch_kernel(const DispatchParams p) {
                 m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 2));
                 m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 1));
                 const float scale = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
+                const float inv = m > 0.f ? __fdiv_rn(448.f, m) : 0.f;
                 uint32_t packed[2];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     uint32_t word = 0;
 #pragma unroll
                     for (int i = 0; i < 2; ++i) {
-                        const float2 q = make_float2(__fdiv_rn(xs[4 * h + 2 * i], scale),
-                                                     __fdiv_rn(xs[4 * h + 2 * i + 1], scale));
+                        const float2 q = make_float2(__fmul_rn(xs[4 * h + 2 * i], inv),
+                                                     __fmul_rn(xs[4 * h + 2 * i + 1], inv));
                         const __nv_fp8x2_storage_t pair = __nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
                         word |= (uint32_t)pair << (16 * i);
                     }
@@ -168,21 +170,21 @@ dispatch_kernel(const DispatchParams p) {
                 }
             }
         }
-        return;
-    }
-    for (int c0 = lo; c0 < hi; c0 += 32 * kVec) {
-        uint4 v[kVec];
-#pragma unroll
-        for (int u = 0; u < kVec; ++u) {
-            const int c = c0 + lane + 32 * u;
-            if (c < hi) v[u] = ld_nc_v4(src + c);
-        }
-        for (int i = 0; i < f; ++i) {
-            uint4* dst = reinterpret_cast<uint4*>(p.recv_x + s_rows[warp][i] * p.H);
+    } else {
+        for (int c0 = lo; c0 < hi; c0 += 32 * kVec) {
+            uint4 v[kVec];
 #pragma unroll
             for (int u = 0; u < kVec; ++u) {
                 const int c = c0 + lane + 32 * u;
-                if (c < hi) st_stream_v4(dst + c, v[u]);
+                if (c < hi) v[u] = ld_nc_v4(src + c);
+            }
+            for (int i = 0; i < f; ++i) {
+                uint4* dst = reinterpret_cast<uint4*>(p.recv_x + s_rows[warp][i] * p.H);
+#pragma unroll
+                for (int u = 0; u < kVec; ++u) {
+                    const int c = c0 + lane + 32 * u;
+                    if (c < hi) st_stream_v4(dst + c, v[u]);
+                }
             }
         }
     }

@@ -252,9 +252,10 @@ EP_API int ep_ll_dispatch(ep_ctx* ctx, const uint16_t* x, const int64_t* topk_id
  * Inference with FP8": use_fp8, the packed result becomes a pair).  Same
  * packing, counts, src_info and layout_range as ep_ll_dispatch; each packed row
  * is stored as OCP E4M3 codes with one fp32 scale per 128 hidden channels:
- *   scale = amax(|x| over the block) / 448 (fp32, nearest even; 1 for an all-zero
- *           block),  code = E4M3(x / scale) (fp32 division, nearest even,
- *           saturating at +-448), so x ~= value(code) * scale.
+ *   scale = amax(|x| over the block) / 448 (fp32, nearest even),
+ *   code  = E4M3(x * (448 / amax)) (fp32 quotient and product, each nearest
+ *           even; E4M3 nearest even, saturating at +-448);
+ * an all-zero block has scale 1 and zero codes; x ~= value(code) * scale.
  *   packed_recv_x_fp8   u8  [R][L][R*Tmax][H]      out (16-byte aligned)
  *   packed_recv_scales  f32 [R][L][R*Tmax][H/128]  out
  * Requires H % 128 == 0 (EP_ERR_INVALID_ARG otherwise). */

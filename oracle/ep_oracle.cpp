@@ -428,11 +428,11 @@ int oracle_ll_combine(int32_t R, int32_t E, int32_t T, int32_t K, int32_t H, int
 // (the example indexes packed_x[0]).  The pages give no format; the reading
 // taken: OCP FP8 E4M3 (bias 7, 3 mantissa bits, largest finite 448, no
 // infinities), one fp32 scale per token per block of 128 hidden channels,
-//   scale = amax(|x| over the block) / 448      (fp32 division, nearest even;
-//                                                 1 when the block is all zero)
-//   code  = e4m3(x / scale)                       (fp32 division, then nearest
-//                                                 even, saturating at +-448)
-// so x ~= value(code) * scale.
+//   scale = amax(|x| over the block) / 448       (fp32 division, nearest even)
+//   code  = e4m3(x * (448 / amax))                (fp32 division and product,
+//                                                  each nearest even; then E4M3
+//                                                  nearest even, saturating)
+// with scale = 1 and all codes 0 for an all-zero block; x ~= value(code) * scale.
 
 // E4M3 code of a finite value, round to nearest even, saturating at +-448.
 static uint8_t e4m3_encode(double v) {
@@ -475,10 +475,11 @@ int oracle_quantize_e4m3_blocks(const uint16_t* rows, int64_t n, int32_t H, int3
             for (int32_t i = 0; i < block; ++i)
                 amax = std::max(amax, (float)std::fabs(bf16_bits_to_double(rows[r * H + b * block + i])));
             const float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+            const float inv = amax > 0.0f ? 448.0f / amax : 0.0f;
             scales[r * nb + b] = scale;
             for (int32_t i = 0; i < block; ++i) {
                 const float x = (float)bf16_bits_to_double(rows[r * H + b * block + i]);
-                const float q = x / scale;
+                const float q = x * inv;
                 codes[r * H + b * block + i] = e4m3_encode((double)q);
             }
         }

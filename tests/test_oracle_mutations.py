@@ -57,7 +57,7 @@ MUTANTS = {
     "expert count per token": (
         "num_tokens_per_expert[(int64_t)s * E + e] += 1;", "num_tokens_per_expert[(int64_t)s * E + e] = 1;"),
     "fp8 scale uses the wrong range": (
-        "amax > 0.0f ? amax / 448.0f : 1.0f", "amax > 0.0f ? amax / 240.0f : 1.0f"),
+        "amax > 0.0f ? 448.0f / amax : 0.0f", "amax > 0.0f ? 240.0f / amax : 0.0f"),
     "fp8 rounding truncates": (
         "double r = std::ldexp(std::nearbyint(std::ldexp(a, -qexp)), qexp);",
         "double r = std::ldexp(std::trunc(std::ldexp(a, -qexp)), qexp);"),

@@ -558,7 +558,8 @@ def test_block_quantisation_error_bound():
     q = np.abs(xf) / np.repeat(scales.astype(np.float64), 128, axis=1)
     e = np.floor(np.log2(np.maximum(q, 2.0 ** -6)))
     half_step = 2.0 ** (e - 3) / 2 * np.repeat(scales.astype(np.float64), 128, axis=1)
-    assert (np.abs(deq - xf) <= half_step * (1 + 1e-6) + 1e-30).all()
+    # half an E4M3 step, plus the fp32 roundings of 448/amax, amax/448 and the product
+    assert (np.abs(deq - xf) <= half_step + 2.0 ** -21 * np.abs(xf) + 1e-30).all()
     # the largest element of each block is encoded as +-448
     blocks = np.abs(xf).reshape(64, 4, 128)
     arg = blocks.argmax(-1)
