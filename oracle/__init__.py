@@ -42,9 +42,9 @@ def load_library(path: str):
     L.oracle_combine.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _ptr, _c_i64, _ptr, _ptr,
                                      _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _c_i64]
     L.oracle_ll_dispatch.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
-                                         _ptr, _ptr, _ptr, _ptr, _ptr, _ptr]
+                                         _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr]
     L.oracle_ll_combine.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
-                                        _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _c_i64]
+                                        _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _c_i64, _ptr]
     L.oracle_fp8_e4m3_encode.argtypes = [_ptr, _ptr, _c_i64]
     L.oracle_fp8_e4m3_encode.restype = None
     L.oracle_quantize_e4m3_blocks.argtypes = [_ptr, _c_i64, _c_i32, _c_i32, _ptr, _ptr]
@@ -178,7 +178,16 @@ def combine(y: np.ndarray, handle: dict, recv_topk_weights=None, bias0=None, bia
     return out, out_w
 
 
-def ll_dispatch(x, topk_idx, num_experts: int, max_tokens_per_rank: int, with_rows: bool = True):
+def _mask(rank_mask, R):
+    if rank_mask is None:
+        return None
+    m = np.ascontiguousarray(rank_mask, dtype=np.int32)
+    assert m.shape == (R,)
+    return m
+
+
+def ll_dispatch(x, topk_idx, num_experts: int, max_tokens_per_rank: int, with_rows: bool = True,
+                rank_mask=None):
     """Returns dict with packed_recv_x [R,L,R*Tmax,H] (if with_rows), packed_recv_count [R,L],
     src_info [R,L,R*Tmax], layout_range [R,L,R,2]."""
     topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int64)
@@ -191,15 +200,16 @@ def ll_dispatch(x, topk_idx, num_experts: int, max_tokens_per_rank: int, with_ro
     count = np.empty((R, L), np.int32)
     src_info = np.full((R, L, cap), -1, np.int32)
     layout_range = np.empty((R, L, R, 2), np.int32)
+    m = _mask(rank_mask, R)
     _check(lib().oracle_ll_dispatch(
         R, num_experts, T, K, H, max_tokens_per_rank, _p(x), _p(topk_idx), _p(packed),
-        _p(count), _p(src_info), _p(layout_range)), "oracle_ll_dispatch")
+        _p(count), _p(src_info), _p(layout_range), _p(m)), "oracle_ll_dispatch")
     return {"packed_recv_x": packed, "packed_recv_count": count, "src_info": src_info,
             "layout_range": layout_range}
 
 
 def ll_combine(y, topk_idx, topk_weights, src_info, layout_range, num_experts: int,
-               max_tokens_per_rank: int, tokens=None):
+               max_tokens_per_rank: int, tokens=None, rank_mask=None):
     y = np.ascontiguousarray(y, dtype=np.uint16)
     topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int64)
     w = np.ascontiguousarray(topk_weights, dtype=np.float32)
@@ -212,7 +222,7 @@ def ll_combine(y, topk_idx, topk_weights, src_info, layout_range, num_experts: i
         R, num_experts, T, K, H, max_tokens_per_rank, _p(y), _p(topk_idx), _p(w),
         _p(np.ascontiguousarray(src_info, dtype=np.int32)),
         _p(np.ascontiguousarray(layout_range, dtype=np.int32)), _p(out), _p(tok),
-        0 if tok is None else tok.size), "oracle_ll_combine")
+        0 if tok is None else tok.size, _p(_mask(rank_mask, R))), "oracle_ll_combine")
     return out.reshape(R, T, H) if tok is None else out
 
 

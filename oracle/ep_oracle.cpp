@@ -335,9 +335,14 @@ int oracle_combine(int32_t R, int32_t T, int32_t K, int32_t H,
 //   * packed_recv_count[d][j] = list length.
 // Slots at or past the count are not written.  packed_recv_x may be null
 // (handle only).
+// [API] "Dynamic Rank Masking": masked ranks are left out of the exchange
+// without tearing it down.  Reading: rank_mask[r] != 0 (nullable) removes rank
+// r both as a source (its tokens are not sent) and as a destination (its
+// experts receive nothing).
 int oracle_ll_dispatch(int32_t R, int32_t E, int32_t T, int32_t K, int32_t H, int32_t Tmax,
                        const uint16_t* x, const int64_t* topk_idx, uint16_t* packed_recv_x,
-                       int32_t* packed_recv_count, int32_t* src_info, int32_t* layout_range) {
+                       int32_t* packed_recv_count, int32_t* src_info, int32_t* layout_range,
+                       const int32_t* rank_mask) {
     if (!shape_ok(R, E, T, K) || H < 1 || Tmax < T) return ORACLE_BAD_ARG;
     const int32_t L = E / R;
     const int64_t cap = (int64_t)R * Tmax;
@@ -353,7 +358,8 @@ int oracle_ll_dispatch(int32_t R, int32_t E, int32_t T, int32_t K, int32_t H, in
                 const int64_t g = (int64_t)s * T + t;
                 bool member = false;
                 for (int32_t k = 0; k < K; ++k) member = member || topk_idx[g * K + k] == e;
-                if (!member) continue;
+                const bool masked = rank_mask != nullptr && (rank_mask[s] != 0 || rank_mask[d] != 0);
+                if (!member || masked) continue;
                 if (slot >= cap) return ORACLE_CAPACITY;
                 src_info[list * cap + slot] = t;
                 if (packed_recv_x != nullptr)
@@ -376,11 +382,13 @@ int oracle_ll_dispatch(int32_t R, int32_t E, int32_t T, int32_t K, int32_t H, in
 //   out[s][t][i] = bf16( sum_k w[s][t][k] * y[d][j][slot(s, t, e)][i] )   (fp64)
 // where e = topk_idx[s][t][k] = d*L + j and slot(s, t, e) is the position of t
 // inside layout_range[d][j][s] (found through src_info).  `tokens` as in
-// oracle_combine.
+// oracle_combine.  With a rank mask (see oracle_ll_dispatch), slots whose
+// expert lives on a masked rank contribute nothing, and the tokens of a masked
+// source rank get +0 (the rank took no part).
 int oracle_ll_combine(int32_t R, int32_t E, int32_t T, int32_t K, int32_t H, int32_t Tmax,
                       const uint16_t* y, const int64_t* topk_idx, const float* topk_weights,
                       const int32_t* src_info, const int32_t* layout_range, uint16_t* out,
-                      const int64_t* tokens, int64_t n_tokens) {
+                      const int64_t* tokens, int64_t n_tokens, const int32_t* rank_mask) {
     if (!shape_ok(R, E, T, K) || H < 1 || Tmax < T) return ORACLE_BAD_ARG;
     const int32_t L = E / R;
     const int64_t cap = (int64_t)R * Tmax;
@@ -397,6 +405,7 @@ int oracle_ll_combine(int32_t R, int32_t E, int32_t T, int32_t K, int32_t H, int
             const int64_t e = topk_idx[g * K + k];
             if (e == -1) continue;
             if (e < -1 || e >= E) return ORACLE_BAD_TOPK;
+            if (rank_mask != nullptr && (rank_mask[s] != 0 || rank_mask[e / L] != 0)) continue;
             order.emplace_back(e, k);
         }
         std::sort(order.begin(), order.end());
@@ -415,7 +424,6 @@ int oracle_ll_combine(int32_t R, int32_t E, int32_t T, int32_t K, int32_t H, int
             const uint16_t* row = y + (list * cap + slot) * H;
             for (int32_t c = 0; c < H; ++c) acc[c] += w * bf16_bits_to_double(row[c]);
         }
-        (void)L;
         for (int32_t c = 0; c < H; ++c) out[i * H + c] = double_to_bf16_bits(acc[c]);
     }
     return ORACLE_OK;

@@ -61,6 +61,8 @@ MUTANTS = {
     "fp8 rounding truncates": (
         "double r = std::ldexp(std::nearbyint(std::ldexp(a, -qexp)), qexp);",
         "double r = std::ldexp(std::trunc(std::ldexp(a, -qexp)), qexp);"),
+    "ll mask ignores the destination": (
+        "(rank_mask[s] != 0 || rank_mask[d] != 0)", "(rank_mask[s] != 0)"),
     "weights leak to other ranks": (
         "here ? topk_weights[g * K + k] : 0.0f;", "topk_weights[g * K + k];"),
 }

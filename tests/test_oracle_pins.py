@@ -566,3 +566,39 @@ def test_block_quantisation_error_bound():
     c = codes.reshape(64, 4, 128)
     picked = np.take_along_axis(c, arg[..., None], -1)[..., 0]
     assert np.isin(picked, [0x7E, 0xFE]).all()
+
+
+# ----------------------------------------------------------------------------
+# dynamic rank masking (low-latency path)
+
+@pytest.mark.parametrize("masked", [[1], [0, 3], [2, 3]])
+def test_ll_rank_mask_equals_dropping_the_slots(masked):
+    """Masking rank r is the same as dropping every slot that leaves from or goes to r;
+    the tokens of a masked source rank combine to +0."""
+    rng = np.random.default_rng(sum(masked) + 17)
+    R, E, T, K, H = 4, 16, 9, 3, 8
+    L = E // R
+    topk = random_topk(rng, R, E, T, K, mask_p=0.1)
+    x = f32_to_bf16_torch(rng.integers(-5, 6, (R, T, H)).astype(np.float32))
+    wts = (2.0 ** rng.integers(-2, 2, topk.shape)).astype(np.float32)
+    mask = np.zeros(R, np.int32)
+    mask[masked] = 1
+    dropped = topk.copy()
+    for s in range(R):
+        for t in range(T):
+            for k in range(K):
+                e = dropped[s, t, k]
+                if e != -1 and (mask[s] or mask[e // L]):
+                    dropped[s, t, k] = -1
+    a = oracle.ll_dispatch(x, topk, E, T, rank_mask=mask)
+    b = oracle.ll_dispatch(x, dropped, E, T)
+    for key in ("packed_recv_count", "layout_range", "src_info", "packed_recv_x"):
+        np.testing.assert_array_equal(a[key], b[key], err_msg=key)
+    yv = rng.integers(-4, 5, a["packed_recv_x"].shape).astype(np.float32)
+    y = f32_to_bf16_torch(yv)
+    out_a = oracle.ll_combine(y, topk, wts, a["src_info"], a["layout_range"], E, T, rank_mask=mask)
+    out_b = oracle.ll_combine(y, dropped, wts, b["src_info"], b["layout_range"], E, T)
+    np.testing.assert_array_equal(out_a, out_b)
+    assert (out_a[mask.astype(bool)] == 0).all()
+    # no expert on a masked rank receives anything
+    assert (a["packed_recv_count"][mask.astype(bool)] == 0).all()
