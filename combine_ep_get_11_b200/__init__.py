@@ -77,6 +77,9 @@ _SIGNATURES = {
     "ep_ll_dispatch": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "ep_ll_dispatch_fp8": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "ep_ll_combine": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "ep_ll_update_mask": (ctypes.c_int, [_vp, _i32, _i32, _vp]),
+    "ep_ll_query_mask": (ctypes.c_int, [_vp, _vp, _vp]),
+    "ep_ll_clean_mask": (ctypes.c_int, [_vp, _vp]),
     "ep_profile_enable": (ctypes.c_int, [_vp, ctypes.c_int]),
     "ep_profile_read": (ctypes.c_int, [_vp, ctypes.POINTER(_i64), ctypes.POINTER(ctypes.c_double)]),
 }
@@ -238,6 +241,22 @@ def ep_ll_combine(ctx, y, topk_idx, topk_weights, src_info, layout_range, out_x,
                                 _event(wait_event)), "ep_ll_combine", ctx)
 
 
+def ep_ll_update_mask(ctx, rank: int, masked: bool, stream=None):
+    _check(load().ep_ll_update_mask(ctx, rank, int(bool(masked)), _stream(stream)), "ep_ll_update_mask", ctx)
+
+
+def ep_ll_query_mask(ctx, out, stream=None):
+    """out: CPU int32 tensor [R]; filled with 0 (active) / 1 (masked)."""
+    assert out.device.type == "cpu" and out.dtype == torch.int32 and out.is_contiguous()
+    _check(load().ep_ll_query_mask(ctx, ctypes.c_void_p(out.data_ptr()), _stream(stream)),
+           "ep_ll_query_mask", ctx)
+    return out
+
+
+def ep_ll_clean_mask(ctx, stream=None):
+    _check(load().ep_ll_clean_mask(ctx, _stream(stream)), "ep_ll_clean_mask", ctx)
+
+
 def ep_profile_enable(ctx, enable: bool = True):
     _check(load().ep_profile_enable(ctx, int(enable)), "ep_profile_enable", ctx)
 
@@ -349,6 +368,16 @@ class Buffer:
         packed = torch.empty((self.R, self.L, cap, self.H), dtype=torch.bfloat16, device=self.device)
         ep_ll_dispatch(self.ctx, x, topk_idx, packed, count, src_info, layout_range, stream)
         return packed, count, (src_info, layout_range)
+
+    def low_latency_update_mask_buffer(self, rank_to_mask: int, mask: bool = True, stream=None):
+        ep_ll_update_mask(self.ctx, rank_to_mask, mask, stream)
+
+    def low_latency_query_mask_buffer(self, out=None, stream=None):
+        out = torch.empty(self.R, dtype=torch.int32) if out is None else out
+        return ep_ll_query_mask(self.ctx, out, stream)
+
+    def low_latency_clean_mask_buffer(self, stream=None):
+        ep_ll_clean_mask(self.ctx, stream)
 
     def low_latency_combine(self, y, topk_idx, topk_weights, ll_handle, stream=None):
         out = torch.empty((self.R, self.T, self.H), dtype=torch.bfloat16, device=self.device)

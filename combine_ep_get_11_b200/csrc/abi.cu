@@ -53,6 +53,7 @@ struct ep_ctx {
     int* ll_done;
     int ll_tiles;
     int* ll_boundary;           // [R+1][E]
+    int* rank_mask;             // [R] low-latency rank mask (0 active, 1 masked)
     char last_error[256];
     bool prof;
     std::vector<ep_prof_rec> pending;
@@ -131,7 +132,7 @@ template <class F>
 int launch(ep_ctx* c, int kind, bool has_work, cudaStream_t s, F&& f) {
     if (!has_work) return EP_OK;
     cudaEvent_t a = nullptr, b = nullptr;
-    if (c->prof) {
+    if (c->prof && kind >= 0) {
         if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess)
             return fail(c, EP_ERR_CUDA, "cudaEventCreate failed");
         record_event(a, s);
@@ -143,7 +144,7 @@ int launch(ep_ctx* c, int kind, bool has_work, cudaStream_t s, F&& f) {
         return fail(c, EP_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
     }
     g_launches.fetch_add(1, std::memory_order_relaxed);
-    if (c->prof) {
+    if (c->prof && kind >= 0) {
         record_event(b, s);
         c->pending.push_back({kind, a, b});
     }
@@ -243,6 +244,7 @@ int ep_create(const ep_config* cfg, ep_ctx** out) {
     c->ll_reset_bytes = ll_status_bytes + 2 * sizeof(int);
     const size_t off_ll = off;             off += align256(c->ll_reset_bytes);
     const size_t off_llb = off;            off += align256((size_t)(c->R + 1) * c->E * sizeof(int));
+    const size_t off_mask = off;           off += align256((size_t)c->R * sizeof(int));
     c->ws_bytes = off;
     if (cudaMalloc(&c->ws, c->ws_bytes) != cudaSuccess) {
         delete c;
@@ -262,6 +264,7 @@ int ep_create(const ep_config* cfg, ep_ctx** out) {
     c->ll_ticket = reinterpret_cast<int*>(c->ws + off_ll + ll_status_bytes);
     c->ll_done = c->ll_ticket + 1;
     c->ll_boundary = reinterpret_cast<int*>(c->ws + off_llb);
+    c->rank_mask = reinterpret_cast<int*>(c->ws + off_mask);   // zeroed below: every rank active
     if (cudaMemset(c->ws, 0, c->ws_bytes) != cudaSuccess) rc = EP_ERR_CUDA;
     if (rc == EP_OK && ep::ll_prepare(c->E) != cudaSuccess) rc = EP_ERR_CUDA;
     if (rc != EP_OK) {
@@ -556,7 +559,7 @@ int ll_dispatch_impl(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint
     rc = cuda_check(c, cudaMemsetAsync(c->ll_reset, 0, c->ll_reset_bytes, s), "memset low-latency scan state");
     if (rc != EP_OK) return rc;
     ep::LLCountParams cp{topk_idx, c->slot_map, packed_recv_count, src_info, layout_range,
-                         c->ll_status, c->ll_ticket, c->ll_done, c->ll_boundary, c->err,
+                         c->ll_status, c->ll_ticket, c->ll_done, c->ll_boundary, c->rank_mask, c->err,
                          c->G, c->R, c->E, c->T, c->K, c->ll_cap, c->ll_tiles};
     rc = launch(c, kLLCount, true, s, [&] { return ep::launch_ll_count(cp, s); });
     if (rc != EP_OK) return rc;
@@ -564,6 +567,7 @@ int ll_dispatch_impl(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint
     dp.x = x;
     dp.topk_idx = topk_idx;
     dp.slot_map = c->slot_map;
+    dp.rank_mask = c->rank_mask;
     dp.ll_capacity = c->ll_cap;
     dp.recv_x = packed_recv_x;
     dp.recv_fp8 = packed_fp8;
@@ -611,10 +615,35 @@ int ep_ll_combine(ep_ctx* c, const uint16_t* y, const int64_t* topk_idx, const f
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     int rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
     if (rc != EP_OK) return rc;
-    ep::LLCombineParams p{y, topk_idx, topk_weights, src_info, layout_range, out_x, c->err,
+    ep::LLCombineParams p{y, topk_idx, topk_weights, src_info, layout_range, c->rank_mask, out_x, c->err,
                           c->G, c->R, c->E, c->T, c->K, c->H, c->ll_cap,
                           ep::combine_splits(c->H)};
     return launch(c, kLLCombine, c->G > 0, s, [&] { return ep::launch_ll_combine(p, c->num_sms, s); });
+}
+
+int ep_ll_update_mask(ep_ctx* c, int32_t rank, int32_t masked, ep_stream_t stream) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (rank < 0 || rank >= c->R) return fail(c, EP_ERR_INVALID_ARG, "rank %d out of range", rank);
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return launch(c, -1, true, s, [&] { return ep::launch_set_mask(c->rank_mask, rank, masked ? 1 : 0, s); });
+}
+
+int ep_ll_query_mask(ep_ctx* c, int32_t* host_out, ep_stream_t stream) {
+    if (c == nullptr || host_out == nullptr) return EP_ERR_INVALID_ARG;
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int rc = cuda_check(c, cudaMemcpyAsync(host_out, c->rank_mask, sizeof(int32_t) * c->R, cudaMemcpyDeviceToHost, s),
+                        "read rank mask");
+    if (rc == EP_OK) rc = cuda_check(c, cudaStreamSynchronize(s), "cudaStreamSynchronize");
+    return rc;
+}
+
+int ep_ll_clean_mask(ep_ctx* c, ep_stream_t stream) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    DeviceGuard guard(c->device);
+    return cuda_check(c, cudaMemsetAsync(c->rank_mask, 0, sizeof(int) * c->R, reinterpret_cast<cudaStream_t>(stream)),
+                      "clear rank mask");
 }
 
 int ep_profile_enable(ep_ctx* c, int enable) {

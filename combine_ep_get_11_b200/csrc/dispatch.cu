@@ -59,7 +59,9 @@ dispatch_kernel(const DispatchParams p) {
     if (kPacked) {
         long long e = -1;
         if (lane < p.K) e = p.topk_idx[g * p.K + lane];
-        bool valid = e >= 0 && e < p.E;
+        // slots from or to a masked rank are not sent
+        bool valid = e >= 0 && e < p.E && p.rank_mask[g / p.T] == 0 &&
+                     p.rank_mask[(int)e / (p.E / p.R)] == 0;
         for (int k = 0; k < p.K; ++k) {   // a repeated expert is sent once
             const long long ek = __shfl_sync(kFullMask, e, k);
             if (k < lane && ek == e) valid = false;

@@ -70,6 +70,7 @@ struct DispatchParams {
     int* recv_src_idx;                 // [cap] or null
     // low latency
     const int* slot_map;               // [G][K]
+    const int* rank_mask;              // [R], 0 active / 1 masked
     int64_t ll_capacity;               // R * Tmax slots per expert
     uint16_t* recv_x;                  // normal/cached: [cap][H]; LL: [E][ll_cap][H]
     // low latency, FP8 form (recv_x unused)
@@ -113,6 +114,7 @@ struct LLCountParams {
     int* ticket;               // zeroed before launch
     int* done;                 // zeroed before launch
     int* boundary;             // [R+1][E] workspace
+    const int* rank_mask;      // [R], 0 active / 1 masked
     int* err;
     long long G;
     int R, E, T, K;
@@ -129,6 +131,7 @@ struct LLCombineParams {
     const float* topk_weights;  // [G][K]
     const int* src_info;        // [E][ll_cap]
     const int* layout_range;    // [E][R][2]
+    const int* rank_mask;       // [R], 0 active / 1 masked
     uint16_t* out_x;            // [G][H]
     int* err;
     long long G;
@@ -137,5 +140,6 @@ struct LLCombineParams {
     int splits;                 // warps per token (column slices of the row)
 };
 cudaError_t launch_ll_combine(const LLCombineParams& p, int num_sms, cudaStream_t stream);
+cudaError_t launch_set_mask(int* rank_mask, int rank, int value, cudaStream_t stream);
 
 }  // namespace ep

@@ -67,12 +67,16 @@ ll_scan_kernel(const LLCountParams p) {
     int64_t ids[kMaxK];
 #pragma unroll
     for (int k = 0; k < kMaxK; ++k) ids[k] = (g < p.G && k < p.K) ? __ldg(p.topk_idx + g * p.K + k) : -1;
+    // a slot from or to a masked rank is not part of the exchange
+    const int L = E / p.R;
+    const bool src_masked = g < p.G && p.rank_mask[g / p.T] != 0;
     bool bad = false;
 #pragma unroll
     for (int k = 0; k < kMaxK; ++k) {
         const int64_t e = ids[k];
         if (e < -1 || e >= E) { bad = true; ids[k] = -1; continue; }
-        if (e >= 0) atomicOr(&bits[e * kLLStride + w], 1u << b);
+        if (e >= 0 && (src_masked || p.rank_mask[e / L] != 0)) ids[k] = -1;
+        if (ids[k] >= 0) atomicOr(&bits[e * kLLStride + w], 1u << b);
     }
     if (bad) record_error(p.err, EP_ERR_BAD_TOPK);
     __syncthreads();
@@ -208,13 +212,14 @@ ll_combine_kernel(const LLCombineParams p) {
     if (g >= p.G) return;   // whole warp
     {
         const int s = (int)(g / p.T), t = (int)(g % p.T);
+        const bool src_masked = p.rank_mask[s] != 0;   // warp-uniform: the token took no part
         long long e = -1;
         float w = 0.f;
-        if (lane < p.K) {
+        if (lane < p.K && !src_masked) {
             e = p.topk_idx[g * p.K + lane];
             w = p.topk_weights[g * p.K + lane];
         }
-        bool valid = e >= 0 && e < p.E;
+        bool valid = e >= 0 && e < p.E && p.rank_mask[(int)e / (p.E / p.R)] == 0;
         long long row = -1;
         if (valid) {
             const int* range = p.layout_range + ((long long)e * p.R + s) * 2;
@@ -296,6 +301,13 @@ ll_combine_kernel(const LLCombineParams p) {
 }
 
 }  // namespace
+
+__global__ void set_mask_kernel(int* rank_mask, int rank, int value) { rank_mask[rank] = value; }
+
+cudaError_t launch_set_mask(int* rank_mask, int rank, int value, cudaStream_t stream) {
+    set_mask_kernel<<<1, 1, 0, stream>>>(rank_mask, rank, value);
+    return cudaGetLastError();
+}
 
 cudaError_t ll_prepare(int E) {
     // opt in to large dynamic shared memory when E needs it

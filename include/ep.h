@@ -312,6 +312,19 @@ EP_API int ep_dispatch_handle_static(int32_t num_ranks, int32_t num_experts, int
                                      const int32_t* num_tokens_per_expert, const ep_handle* handle,
                                      int32_t* error_word, ep_stream_t stream);
 
+/* Dynamic rank masking for the low-latency calls ([API] "Dynamic Rank
+ * Masking": leave ranks, e.g. failed nodes, out of the exchange without
+ * tearing it down; query reports 0 = active, 1 = masked; clean resets all).
+ * A masked rank neither sends nor receives in ep_ll_dispatch[_fp8]: its tokens
+ * are not packed and its experts receive nothing; in ep_ll_combine slots on a
+ * masked rank contribute nothing and the masked rank's own tokens get +0.
+ * Every rank starts active.  Updates and clean are stream-ordered (they apply
+ * to low-latency calls issued after them on the stream); query synchronizes
+ * the stream and writes R int32 values to host memory. */
+EP_API int ep_ll_update_mask(ep_ctx* ctx, int32_t rank, int32_t masked, ep_stream_t stream);
+EP_API int ep_ll_query_mask(ep_ctx* ctx, int32_t* host_out, ep_stream_t stream);
+EP_API int ep_ll_clean_mask(ep_ctx* ctx, ep_stream_t stream);
+
 /* Optional per-kernel timing (CUDA events around each launch on the call's
  * stream; inside a stream capture they become event-record nodes, recorded
  * each time the graph runs).  ep_profile_read synchronizes the recorded events and returns,

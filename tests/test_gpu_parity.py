@@ -294,3 +294,68 @@ def test_low_latency_fp8_rejects_unaligned_hidden(ep):
         buf.low_latency_dispatch(inp.x_d, inp.topk_d, use_fp8=True)
     assert e.value.status == 1
     buf.destroy()
+
+
+@pytest.mark.parametrize("masked", [[3], [0, 15]], ids=["mask-3", "mask-0-15"])
+def test_low_latency_rank_mask(ep, masked):
+    """A rank marked failed on the host leaves the low-latency exchange; the other ranks'
+    results equal the oracle's with that rank masked; unmask / clean restores it."""
+    w = W["ll"].scaled(num_tokens=40, hidden=1024)
+    R, E = w.num_ranks, w.num_experts
+    inp = Inputs(w)
+    buf = make_buffer(ep, w)
+    for r in masked:
+        buf.low_latency_update_mask_buffer(r, True)
+    mask = buf.low_latency_query_mask_buffer().numpy()
+    assert mask.tolist() == [int(r in masked) for r in range(R)]
+
+    packed, count, (src_info, layout_range) = buf.low_latency_dispatch(inp.x_d, inp.topk_d)
+    assert buf.sync_status() == 0
+    ll = oracle.ll_dispatch(inp.x_u16, inp.topk, E, w.tmax, rank_mask=mask)
+    np.testing.assert_array_equal(count.cpu().numpy(), ll["packed_recv_count"])
+    np.testing.assert_array_equal(layout_range.cpu().numpy(), ll["layout_range"])
+    p, si = u16(packed), src_info.cpu().numpy()
+    for d in range(R):
+        for j in range(w.local_experts):
+            n = int(ll["packed_recv_count"][d, j])
+            np.testing.assert_array_equal(si[d, j, :n], ll["src_info"][d, j, :n])
+            np.testing.assert_array_equal(p[d, j, :n], ll["packed_recv_x"][d, j, :n])
+    y_u16 = u16(synth.expert_rows(w.seed + 3, p.reshape(-1, w.hidden).shape[0], w.hidden)).reshape(p.shape)
+    out = buf.low_latency_combine(to_bf16_tensor(y_u16).cuda(), inp.topk_d, inp.weights_d,
+                                  (src_info, layout_range))
+    ref = oracle.ll_combine(y_u16, inp.topk, inp.weights, ll["src_info"], ll["layout_range"], E,
+                            w.tmax, rank_mask=mask)
+    abs_ref = oracle.ll_combine(bf16_abs(y_u16), inp.topk, np.abs(inp.weights), ll["src_info"],
+                                ll["layout_range"], E, w.tmax, rank_mask=mask)
+    got = u16(out)
+    assert_combine_close(got, ref, abs_ref, w.topk, "masked ll combine")
+    assert (got[mask.astype(bool)] == 0).all()
+
+    (codes, scales), count8, _ = buf.low_latency_dispatch(inp.x_d, inp.topk_d, use_fp8=True)
+    np.testing.assert_array_equal(count8.cpu().numpy(), ll["packed_recv_count"])
+    c = codes.cpu().numpy()
+    for d in range(R):
+        for j in range(w.local_experts):
+            n = int(ll["packed_recv_count"][d, j])
+            if n:
+                e_codes, _ = oracle.quantize_e4m3_blocks(ll["packed_recv_x"][d, j, :n], 128)
+                np.testing.assert_array_equal(c[d, j, :n], e_codes)
+
+    # recovery: unmask one rank, then clean all
+    buf.low_latency_update_mask_buffer(masked[0], False)
+    assert buf.low_latency_query_mask_buffer().numpy()[masked[0]] == 0
+    buf.low_latency_clean_mask_buffer()
+    assert not buf.low_latency_query_mask_buffer().numpy().any()
+    _, count2, _ = buf.low_latency_dispatch(inp.x_d, inp.topk_d)
+    np.testing.assert_array_equal(count2.cpu().numpy(),
+                                  oracle.ll_dispatch(None, inp.topk, E, w.tmax, with_rows=False)["packed_recv_count"])
+    assert buf.sync_status() == 0
+    buf.destroy()
+
+
+def test_low_latency_mask_rejects_bad_rank(ep):
+    w = W["tiny"]
+    buf = make_buffer(ep, w)
+    with pytest.raises(ep.EpError):
+        buf.low_latency_update_mask_buffer(w.num_ranks, True)
+    buf.destroy()
