@@ -48,9 +48,12 @@ def load_library(path: str):
     L.oracle_fp8_e4m3_encode.argtypes = [_ptr, _ptr, _c_i64]
     L.oracle_fp8_e4m3_encode.restype = None
     L.oracle_quantize_e4m3_blocks.argtypes = [_ptr, _c_i64, _c_i32, _c_i32, _ptr, _ptr]
+    L.oracle_lb_prefetch_weights.argtypes = [_ptr, _c_i32, _c_i64, _ptr, _c_i32, _ptr]
+    L.oracle_lb_reduce_grads.argtypes = [_ptr, _ptr, _c_i32, _ptr, _c_i32, _c_i64]
     for name in ("oracle_layout", "oracle_dispatch_handle", "oracle_dispatch_rows",
                  "oracle_combine", "oracle_ll_dispatch", "oracle_ll_combine",
-                 "oracle_quantize_e4m3_blocks"):
+                 "oracle_quantize_e4m3_blocks", "oracle_lb_prefetch_weights",
+                 "oracle_lb_reduce_grads"):
         getattr(L, name).restype = ctypes.c_int
     return L
 
@@ -243,3 +246,25 @@ def quantize_e4m3_blocks(rows: np.ndarray, block: int = 128):
     _check(lib().oracle_quantize_e4m3_blocks(_p(r), n, H, block, _p(codes), _p(scales)),
            "oracle_quantize_e4m3_blocks")
     return codes, scales
+
+
+def lb_prefetch_weights(expert_weights, mapping, redundant_weights):
+    """expert_weights [E, W] u16, mapping [N] i32 -> redundant_weights [N, W] u16 (updated copy)."""
+    ew = np.ascontiguousarray(expert_weights, dtype=np.uint16)
+    m = np.ascontiguousarray(mapping, dtype=np.int32)
+    out = np.array(redundant_weights, dtype=np.uint16, copy=True, order="C")
+    E, W = ew.shape
+    _check(lib().oracle_lb_prefetch_weights(_p(ew), E, W, _p(m), m.size, _p(out)),
+           "oracle_lb_prefetch_weights")
+    return out
+
+
+def lb_reduce_grads(redundant_grads, mapping, expert_grads):
+    """redundant_grads [N, W] u16, mapping [N] i32, expert_grads [E, W] u16 -> new expert_grads."""
+    rg = np.ascontiguousarray(redundant_grads, dtype=np.uint16)
+    m = np.ascontiguousarray(mapping, dtype=np.int32)
+    out = np.array(expert_grads, dtype=np.uint16, copy=True, order="C")
+    E, W = out.shape
+    _check(lib().oracle_lb_reduce_grads(_p(rg), _p(m), m.size, _p(out), E, W),
+           "oracle_lb_reduce_grads")
+    return out

@@ -495,4 +495,47 @@ int oracle_quantize_e4m3_blocks(const uint16_t* rows, int64_t n, int32_t H, int3
     return ORACLE_OK;
 }
 
+// ------------------------------------------------- load balance (redundant experts)
+//
+// [V2] "10.2 与 EP 的关联能力": lb_prefetch_weights moves the weights of
+// redundant expert replicas in before the expert compute, and lb_reduce_grads
+// folds the replicas' gradients back into the original experts in the backward
+// pass, both keyed by redundancy_mapping.  The page gives no shapes; readings:
+//   * every expert's weights (or gradients) are one block of W bf16 values:
+//     expert_weights [E][W], redundant weights/grads [N][W];
+//   * redundancy_mapping[i] is the original expert of replica i, -1 = unused;
+//   * prefetch: redundant[i] = expert_weights[mapping[i]] (bit copy);
+//   * reduce:   expert_grads[e] = bf16( expert_grads[e] + sum over replicas i
+//               of e, ascending i, of redundant_grads[i] )  (fp64 here).
+int oracle_lb_prefetch_weights(const uint16_t* expert_weights, int32_t E, int64_t W,
+                               const int32_t* mapping, int32_t N, uint16_t* redundant_weights) {
+    if (E < 1 || W < 1 || N < 0) return ORACLE_BAD_ARG;
+    for (int32_t i = 0; i < N; ++i) {
+        const int32_t e = mapping[i];
+        if (e == -1) continue;
+        if (e < -1 || e >= E) return ORACLE_BAD_TOPK;
+        for (int64_t c = 0; c < W; ++c) redundant_weights[(int64_t)i * W + c] = expert_weights[(int64_t)e * W + c];
+    }
+    return ORACLE_OK;
+}
+
+int oracle_lb_reduce_grads(const uint16_t* redundant_grads, const int32_t* mapping, int32_t N,
+                           uint16_t* expert_grads, int32_t E, int64_t W) {
+    if (E < 1 || W < 1 || N < 0) return ORACLE_BAD_ARG;
+    for (int32_t i = 0; i < N; ++i)
+        if (mapping[i] < -1 || mapping[i] >= E) return ORACLE_BAD_TOPK;
+    for (int32_t e = 0; e < E; ++e) {
+        bool any = false;
+        for (int32_t i = 0; i < N; ++i) any = any || mapping[i] == e;
+        if (!any) continue;   // untouched
+        for (int64_t c = 0; c < W; ++c) {
+            double acc = bf16_bits_to_double(expert_grads[(int64_t)e * W + c]);
+            for (int32_t i = 0; i < N; ++i)
+                if (mapping[i] == e) acc += bf16_bits_to_double(redundant_grads[(int64_t)i * W + c]);
+            expert_grads[(int64_t)e * W + c] = double_to_bf16_bits(acc);
+        }
+    }
+    return ORACLE_OK;
+}
+
 }  // extern "C"

@@ -63,6 +63,8 @@ MUTANTS = {
         "double r = std::ldexp(std::trunc(std::ldexp(a, -qexp)), qexp);"),
     "ll mask ignores the destination": (
         "(rank_mask[s] != 0 || rank_mask[d] != 0)", "(rank_mask[s] != 0)"),
+    "lb reduce drops the original gradient": (
+        "double acc = bf16_bits_to_double(expert_grads[(int64_t)e * W + c]);", "double acc = 0.0;"),
     "weights leak to other ranks": (
         "here ? topk_weights[g * K + k] : 0.0f;", "topk_weights[g * K + k];"),
 }

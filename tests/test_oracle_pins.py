@@ -602,3 +602,45 @@ def test_ll_rank_mask_equals_dropping_the_slots(masked):
     assert (out_a[mask.astype(bool)] == 0).all()
     # no expert on a masked rank receives anything
     assert (a["packed_recv_count"][mask.astype(bool)] == 0).all()
+
+
+# ----------------------------------------------------------------------------
+# load balance: redundant-expert weight prefetch and gradient reduction
+
+def test_lb_prefetch_is_a_gather():
+    rng = np.random.default_rng(31)
+    E, W, N = 6, 40, 9
+    ew = rng.integers(0, 1 << 16, (E, W)).astype(np.uint16)
+    mapping = rng.integers(-1, E, N).astype(np.int32)
+    before = rng.integers(0, 1 << 16, (N, W)).astype(np.uint16)
+    out = oracle.lb_prefetch_weights(ew, mapping, before)
+    for i in range(N):
+        np.testing.assert_array_equal(out[i], ew[mapping[i]] if mapping[i] >= 0 else before[i])
+
+
+def test_lb_reduce_integer_rows_exact():
+    rng = np.random.default_rng(32)
+    E, W, N = 5, 24, 11
+    mapping = rng.integers(-1, E, N).astype(np.int32)
+    g = rng.integers(-20, 21, (E, W)).astype(np.float32)
+    r = rng.integers(-20, 21, (N, W)).astype(np.float32)
+    out = oracle.lb_reduce_grads(f32_to_bf16_torch(r), mapping, f32_to_bf16_torch(g))
+    exp = g.astype(np.float64).copy()
+    for i in range(N):
+        if mapping[i] >= 0:
+            exp[mapping[i]] += r[i]
+    np.testing.assert_array_equal(bf16_to_f64(out), exp)
+    untouched = [e for e in range(E) if e not in set(mapping.tolist())]
+    for e in untouched:
+        np.testing.assert_array_equal(out[e], f32_to_bf16_torch(g[e]))
+
+
+def test_lb_reduce_rounds_once():
+    # 1 + 3 * 2^-8 is a tie between 1 + 2^-7 and 1 + 2^-6 and rounds to the even one, 1 + 2^-6;
+    # rounding after every addition would give 1 (each 1 + 2^-8 ties back down to 1)
+    g = f32_to_bf16_torch(np.array([[1.0]], np.float32))
+    r = f32_to_bf16_torch(np.full((3, 1), 2.0 ** -8, np.float32))
+    out = oracle.lb_reduce_grads(r, np.zeros(3, np.int32), g)
+    assert bf16_to_f64(out)[0, 0] == 1.0 + 2.0 ** -6
+    with pytest.raises(oracle.OracleError):
+        oracle.lb_reduce_grads(r, np.array([0, 9, 0], np.int32), g)
