@@ -41,6 +41,9 @@ WORKLOAD = "dsv3"
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 CPU_SAMPLE_TOKENS = 2048       # oracle baseline: first 2048 tokens of every rank
+LB_EXPERTS = 32                # load-balance workload: 32 local experts ...
+LB_EXPERT_ELEMS = 3 * 7168 * 2048   # ... of DeepSeek-V3 size (gate/up/down), bf16
+LB_REPLICAS = 8                # ... and 8 redundant replicas
 
 
 # ------------------------------------------------------------------ bytes
@@ -311,6 +314,29 @@ class Path:
                 ep.ep_ll_combine(ctx, self.packed, td, wd, self.src_info, self.layout_range, self.out)
             self.step = step
             return
+        if w.name == "lb":
+            # redundant-expert load balance: weight prefetch + gradient reduction of
+            # DeepSeek-V3-sized experts (3 x 7168 x 2048 bf16 per expert)
+            E_l, W = LB_EXPERTS, LB_EXPERT_ELEMS
+            self.mapping = torch.from_numpy(synth.redundancy_mapping(E_l, LB_REPLICAS, seed=w.seed)).to(dev)
+            m = self.mapping.cpu().numpy()
+            self.ew = synth.expert_rows_device(w.seed + 1, E_l, W, dev)
+            self.red = torch.empty((LB_REPLICAS, W), dtype=torch.bfloat16, device=dev)
+            self.grads = synth.expert_rows_device(w.seed + 2, E_l, W, dev)
+            self.rgrads = synth.expert_rows_device(w.seed + 3, LB_REPLICAS, W, dev)
+            nv = int((m >= 0).sum())
+            touched = len(set(m[m >= 0].tolist()))
+            self.N = nv
+            self.bytes = {"lb_prefetch": 2 * nv * W * 2, "lb_reduce": (2 * touched + nv) * W * 2}
+            self.dominant = ("lb_prefetch", "lb_reduce")
+            self.inputs = ("x",)
+            self.lb_units = E_l
+
+            def step(xd, td, wd):
+                ep.ep_lb_prefetch_weights(ctx, self.ew, self.mapping, self.red)
+                ep.ep_lb_reduce_grads(ctx, self.rgrads, self.mapping, self.grads)
+            self.step = step
+            return
         ntr = torch.empty((R, R), dtype=torch.int32, device=dev)
         nte = torch.empty((R, E), dtype=torch.int32, device=dev)
         tin = torch.empty((R, T, R), dtype=torch.uint8, device=dev)
@@ -376,7 +402,7 @@ def run_ours(args):
 
     # inputs smaller than L2 are re-read from L2 across steps: flush between steps then
     input_bytes = R * T * H * 2
-    flush = input_bytes < 2 * L2_BYTES
+    flush = input_bytes < 2 * L2_BYTES and w.name != "lb"    # lb moves GB-sized expert blocks
     # flush by reading (a written scrub leaves ~L2 of dirty lines whose write-back
     # would overlap the next timed kernel)
     scrub = torch.ones(L2_BYTES, dtype=torch.float16, device=dev) if flush else None
@@ -437,7 +463,8 @@ def run_ours(args):
     if rc != 0:
         raise RuntimeError(f"device status {rc} after the timed region")
 
-    ms, gbs, tokens_per_s = aggregate(ms_local, step_total, R * T, args.steps, world, dev)
+    units = getattr(path, "lb_units", R * T)          # tokens (experts for the lb workload)
+    ms, gbs, tokens_per_s = aggregate(ms_local, step_total, units, args.steps, world, dev)
 
     # ---- per-kernel times (events around each launch on the call's stream)
     stage_ms = {k: (v[1] / v[0]) for k, v in prof.items() if v[0]}

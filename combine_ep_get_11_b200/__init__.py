@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "EP_OK", 1: "EP_ERR_INVALID_ARG", 2: "EP_ERR_ALIGNMENT", 3: "
                 4: "EP_ERR_BAD_TOPK", 5: "EP_ERR_HANDLE_MISMATCH", 6: "EP_ERR_TIMEOUT",
                 7: "EP_ERR_CUDA", 8: "EP_ERR_UNIMPLEMENTED"}
 PROFILE_KINDS = ["layout", "scan", "dispatch", "dispatch_cached", "combine", "ll_count",
-                 "ll_copy", "ll_combine", "ll_copy_fp8"]
+                 "ll_copy", "ll_combine", "ll_copy_fp8", "lb_prefetch", "lb_reduce"]
 
 _vp = ctypes.c_void_p
 _i32 = ctypes.c_int32
@@ -77,6 +77,8 @@ _SIGNATURES = {
     "ep_ll_dispatch": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "ep_ll_dispatch_fp8": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "ep_ll_combine": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "ep_lb_prefetch_weights": (ctypes.c_int, [_vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp]),
+    "ep_lb_reduce_grads": (ctypes.c_int, [_vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp]),
     "ep_ll_update_mask": (ctypes.c_int, [_vp, _i32, _i32, _vp]),
     "ep_ll_query_mask": (ctypes.c_int, [_vp, _vp, _vp]),
     "ep_ll_clean_mask": (ctypes.c_int, [_vp, _vp]),
@@ -241,6 +243,23 @@ def ep_ll_combine(ctx, y, topk_idx, topk_weights, src_info, layout_range, out_x,
                                 _event(wait_event)), "ep_ll_combine", ctx)
 
 
+def ep_lb_prefetch_weights(ctx, expert_weights, redundancy_mapping, redundant_weights, stream=None,
+                           wait_event=None):
+    """expert_weights [E, ...] bf16, redundancy_mapping [N] int32, redundant_weights [N, ...] bf16."""
+    w = expert_weights[0].numel() if expert_weights.dim() > 1 else 1
+    _check(load().ep_lb_prefetch_weights(ctx, _ptr(expert_weights), w, _ptr(redundancy_mapping),
+                                         redundancy_mapping.numel(), _ptr(redundant_weights),
+                                         _stream(stream), _event(wait_event)), "ep_lb_prefetch_weights", ctx)
+
+
+def ep_lb_reduce_grads(ctx, redundant_grads, redundancy_mapping, expert_grads, stream=None, wait_event=None):
+    """redundant_grads [N, ...] bf16, redundancy_mapping [N] int32, expert_grads [E, ...] bf16 (in/out)."""
+    w = expert_grads[0].numel() if expert_grads.dim() > 1 else 1
+    _check(load().ep_lb_reduce_grads(ctx, _ptr(redundant_grads), w, _ptr(redundancy_mapping),
+                                     redundancy_mapping.numel(), _ptr(expert_grads), _stream(stream),
+                                     _event(wait_event)), "ep_lb_reduce_grads", ctx)
+
+
 def ep_ll_update_mask(ctx, rank: int, masked: bool, stream=None):
     _check(load().ep_ll_update_mask(ctx, rank, int(bool(masked)), _stream(stream)), "ep_ll_update_mask", ctx)
 
@@ -368,6 +387,12 @@ class Buffer:
         packed = torch.empty((self.R, self.L, cap, self.H), dtype=torch.bfloat16, device=self.device)
         ep_ll_dispatch(self.ctx, x, topk_idx, packed, count, src_info, layout_range, stream)
         return packed, count, (src_info, layout_range)
+
+    def lb_prefetch_weights(self, redundant_expert_weights, expert_weights, redundancy_mapping, stream=None):
+        ep_lb_prefetch_weights(self.ctx, expert_weights, redundancy_mapping, redundant_expert_weights, stream)
+
+    def lb_reduce_grads(self, redundant_expert_grads, expert_grads, redundancy_mapping, stream=None):
+        ep_lb_reduce_grads(self.ctx, redundant_expert_grads, redundancy_mapping, expert_grads, stream)
 
     def low_latency_update_mask_buffer(self, rank_to_mask: int, mask: bool = True, stream=None):
         ep_ll_update_mask(self.ctx, rank_to_mask, mask, stream)

@@ -10,6 +10,7 @@
 //   ep_combine             : combine_kernel
 //   ep_ll_dispatch[_fp8]   : memset(LL scan state) + ll_scan_kernel + dispatch_kernel<packed[, FP8]>
 //   ep_ll_combine          : ll_combine_kernel
+//   ep_lb_prefetch_weights : lb_prefetch_kernel;  ep_lb_reduce_grads : lb_reduce_kernel
 
 #include <atomic>
 #include <cstdarg>
@@ -66,7 +67,7 @@ namespace {
 std::atomic<uint64_t> g_launches{0};
 
 enum Kind { kLayout = 0, kScan = 1, kDispatch = 2, kCached = 3, kCombine = 4,
-            kLLCount = 5, kLLCopy = 6, kLLCombine = 7, kLLCopyFp8 = 8 };
+            kLLCount = 5, kLLCopy = 6, kLLCombine = 7, kLLCopyFp8 = 8, kLBPrefetch = 9, kLBReduce = 10 };
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
@@ -619,6 +620,50 @@ int ep_ll_combine(ep_ctx* c, const uint16_t* y, const int64_t* topk_idx, const f
                           c->G, c->R, c->E, c->T, c->K, c->H, c->ll_cap,
                           ep::combine_splits(c->H)};
     return launch(c, kLLCombine, c->G > 0, s, [&] { return ep::launch_ll_combine(p, c->num_sms, s); });
+}
+
+int ep_lb_prefetch_weights(ep_ctx* c, const uint16_t* expert_weights, int64_t elems_per_expert,
+                           const int32_t* redundancy_mapping, int32_t num_redundant,
+                           uint16_t* redundant_weights, ep_stream_t stream, ep_event_t wait_event) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (elems_per_expert < 0 || num_redundant < 0 || num_redundant > 65535)
+        return fail(c, EP_ERR_INVALID_ARG, "bad sizes");
+    if (elems_per_expert % 8 != 0) return fail(c, EP_ERR_ALIGNMENT, "elems_per_expert must be a multiple of 8");
+    if (num_redundant > 0 && elems_per_expert > 0 &&
+        (expert_weights == nullptr || redundancy_mapping == nullptr || redundant_weights == nullptr))
+        return fail(c, EP_ERR_INVALID_ARG, "argument missing");
+    if (!aligned16(expert_weights) || !aligned16(redundant_weights) || !aligned(redundancy_mapping, 4))
+        return fail(c, EP_ERR_ALIGNMENT, "buffers misaligned");
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
+    if (rc != EP_OK) return rc;
+    ep::LBParams p{const_cast<uint16_t*>(expert_weights), redundant_weights, redundancy_mapping, c->err,
+                   elems_per_expert / 8, c->E, num_redundant};
+    return launch(c, kLBPrefetch, num_redundant > 0 && elems_per_expert > 0, s,
+                  [&] { return ep::launch_lb_prefetch(p, s); });
+}
+
+int ep_lb_reduce_grads(ep_ctx* c, const uint16_t* redundant_grads, int64_t elems_per_expert,
+                       const int32_t* redundancy_mapping, int32_t num_redundant,
+                       uint16_t* expert_grads, ep_stream_t stream, ep_event_t wait_event) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (elems_per_expert < 0 || num_redundant < 0 || num_redundant > 65535)
+        return fail(c, EP_ERR_INVALID_ARG, "bad sizes");
+    if (elems_per_expert % 8 != 0) return fail(c, EP_ERR_ALIGNMENT, "elems_per_expert must be a multiple of 8");
+    if (num_redundant > 0 && elems_per_expert > 0 &&
+        (redundant_grads == nullptr || redundancy_mapping == nullptr || expert_grads == nullptr))
+        return fail(c, EP_ERR_INVALID_ARG, "argument missing");
+    if (!aligned16(redundant_grads) || !aligned16(expert_grads) || !aligned(redundancy_mapping, 4))
+        return fail(c, EP_ERR_ALIGNMENT, "buffers misaligned");
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
+    if (rc != EP_OK) return rc;
+    ep::LBParams p{expert_grads, const_cast<uint16_t*>(redundant_grads), redundancy_mapping, c->err,
+                   elems_per_expert / 8, c->E, num_redundant};
+    return launch(c, kLBReduce, num_redundant > 0 && elems_per_expert > 0, s,
+                  [&] { return ep::launch_lb_reduce(p, s); });
 }
 
 int ep_ll_update_mask(ep_ctx* c, int32_t rank, int32_t masked, ep_stream_t stream) {

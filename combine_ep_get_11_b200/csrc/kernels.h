@@ -142,4 +142,16 @@ struct LLCombineParams {
 cudaError_t launch_ll_combine(const LLCombineParams& p, int num_sms, cudaStream_t stream);
 cudaError_t launch_set_mask(int* rank_mask, int rank, int value, cudaStream_t stream);
 
+// ------------------------------------------------------------ load balance
+struct LBParams {
+    uint16_t* expert;           // prefetch: expert weights [E][W] (read); reduce: expert grads (in/out)
+    uint16_t* redundant;        // prefetch: replica weights [N][W] (written); reduce: replica grads (read)
+    const int* mapping;         // [N] replica -> original expert, -1 unused
+    int* err;
+    long long Wv;               // 16-byte vectors per expert block (W / 8)
+    int E, N;
+};
+cudaError_t launch_lb_prefetch(const LBParams& p, cudaStream_t stream);
+cudaError_t launch_lb_reduce(const LBParams& p, cudaStream_t stream);
+
 }  // namespace ep

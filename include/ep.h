@@ -277,6 +277,28 @@ EP_API int ep_ll_combine(ep_ctx* ctx, const uint16_t* y, const int64_t* topk_idx
                   const int32_t* layout_range, uint16_t* out_x,
                   ep_stream_t stream, ep_event_t wait_event);
 
+/* Load balance for redundant experts ("第 10 章 V2：EP 之外的 Buffer 与扩展能力",
+ * section 10.2: replica weights are fetched before the expert compute and the
+ * replicas' gradients are folded back into the original experts in the
+ * backward pass, keyed by redundancy_mapping).  Every expert's weights (or
+ * gradients) are one block of W bf16 values, W % 8 == 0 (EP_ERR_ALIGNMENT):
+ *   redundancy_mapping  i32 [N]: original expert (in [0, E)) of replica i, -1 = unused
+ *   ep_lb_prefetch_weights: redundant_weights[i] = expert_weights[mapping[i]]
+ *     (expert_weights bf16 [E][W], redundant_weights bf16 [N][W]; rows of unused
+ *     replicas are left untouched)
+ *   ep_lb_reduce_grads: expert_grads[e] = bf16( expert_grads[e] + sum over
+ *     replicas i of e, ascending i, of redundant_grads[i] ), fp32 accumulation
+ *     in that order, one rounding; experts without replicas are untouched
+ *     (expert_grads bf16 [E][W] in/out, redundant_grads bf16 [N][W])
+ * E is the context's num_experts; N <= 65535, at most 1024 replicas per expert.
+ * Mapping entries outside [-1, E) record EP_ERR_BAD_TOPK for ep_sync_status. */
+EP_API int ep_lb_prefetch_weights(ep_ctx* ctx, const uint16_t* expert_weights, int64_t elems_per_expert,
+                                  const int32_t* redundancy_mapping, int32_t num_redundant,
+                                  uint16_t* redundant_weights, ep_stream_t stream, ep_event_t wait_event);
+EP_API int ep_lb_reduce_grads(ep_ctx* ctx, const uint16_t* redundant_grads, int64_t elems_per_expert,
+                              const int32_t* redundancy_mapping, int32_t num_redundant,
+                              uint16_t* expert_grads, ep_stream_t stream, ep_event_t wait_event);
+
 /* Size of the library's static device scratch array (512 KiB on every GPU that
  * loads the library, held until the process exits). */
 #define EP_STATIC_SCRATCH_BYTES (512u * 1024u)
@@ -330,8 +352,9 @@ EP_API int ep_ll_clean_mask(ep_ctx* ctx, ep_stream_t stream);
  * each time the graph runs).  ep_profile_read synchronizes the recorded events and returns,
  * per kernel kind, the number of launches and total milliseconds since the
  * last read; kinds: 0 layout, 1 scan (handle), 2 dispatch, 3 cached dispatch,
- * 4 combine, 5 ll slots, 6 ll copy, 7 ll combine, 8 ll copy (FP8). */
-#define EP_PROFILE_KINDS 9
+ * 4 combine, 5 ll slots, 6 ll copy, 7 ll combine, 8 ll copy (FP8),
+ * 9 lb prefetch, 10 lb reduce. */
+#define EP_PROFILE_KINDS 11
 EP_API int ep_profile_enable(ep_ctx* ctx, int enable);
 EP_API int ep_profile_read(ep_ctx* ctx, int64_t* launches, double* total_ms);
 

@@ -42,6 +42,7 @@ _KIND_X = 4
 _KIND_Y = 5
 _KIND_BIAS = 6
 _KIND_PERM = 7
+_KIND_REDUNDANCY = 8
 
 
 @dataclasses.dataclass(frozen=True)
@@ -86,6 +87,9 @@ WORKLOADS = {
                    max_tokens_per_rank=128),
     "zipf": Workload("zipf", 32, 256, 8192, 7168, 8, "zipf", SEED_BASE + 3),
     "reuse": Workload("reuse", 8, 256, 4096, 4096, 8, "group_limited", SEED_BASE + 4),
+    # redundant-expert load balance (weights, not tokens: the token fields size the
+    # context only)
+    "lb": Workload("lb", 8, 256, 16, 128, 8, "uniform", SEED_BASE + 5),
 }
 
 
@@ -206,3 +210,13 @@ def expert_rows_device(seed: int, num_rows: int, hidden: int, device="cuda", chu
         hi = min(num_rows, lo + chunk_rows)
         y[lo:hi] = torch.randn((hi - lo, hidden), generator=gen, device=device, dtype=torch.float32)
     return y
+
+
+def redundancy_mapping(num_experts: int, num_redundant: int, seed: int, unused_prob: float = 0.0):
+    """[N] int32: the original expert of each redundant replica (seeded; an expert may have
+    several replicas; -1 marks an unused replica slot with probability unused_prob)."""
+    rng = _rng(seed, 0, _KIND_REDUNDANCY)
+    m = rng.integers(0, num_experts, num_redundant).astype(np.int32)
+    if unused_prob > 0:
+        m[rng.random(num_redundant) < unused_prob] = -1
+    return m

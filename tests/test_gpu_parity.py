@@ -250,8 +250,13 @@ def test_profile_counts_every_kernel(ep):
     packed, _, llh = buf.low_latency_dispatch(inp.x_d, inp.topk_d)
     buf.low_latency_combine(packed, inp.topk_d, inp.weights_d, llh)
     buf.low_latency_dispatch(inp.x_d, inp.topk_d, use_fp8=True)
+    mapping = torch.tensor([1, -1, 1, 3], dtype=torch.int32, device="cuda")
+    ew = torch.ones((w.num_experts, 64), dtype=torch.bfloat16, device="cuda")
+    red = torch.zeros((4, 64), dtype=torch.bfloat16, device="cuda")
+    buf.lb_prefetch_weights(red, ew, mapping)
+    buf.lb_reduce_grads(red, ew, mapping)
     prof = ep.ep_profile_read(buf.ctx)
-    assert ep.kernel_launch_count() - before == 10
+    assert ep.kernel_launch_count() - before == 12
     for kind in ep.PROFILE_KINDS:
         n, ms = prof[kind]
         assert n == (2 if kind == "ll_count" else 1) and ms > 0, kind
@@ -358,4 +363,47 @@ def test_low_latency_mask_rejects_bad_rank(ep):
     buf = make_buffer(ep, w)
     with pytest.raises(ep.EpError):
         buf.low_latency_update_mask_buffer(w.num_ranks, True)
+    buf.destroy()
+
+
+@pytest.mark.parametrize("E,W,N", [(32, 7168 * 8, 12), (8, 24, 5), (4, 4096, 9)])
+def test_load_balance_prefetch_and_reduce(ep, E, W, N):
+    w = synth.Workload("lb", 4, E, 16, 64, 2, "uniform", 90)
+    buf = make_buffer(ep, w)
+    mapping = synth.redundancy_mapping(E, N, seed=E * 1000 + N, unused_prob=0.2)
+    mapping[0] = mapping[1] = 2                    # an expert with several replicas
+    ew = synth.expert_rows(91, E, W)
+    before = synth.expert_rows(92, N, W)
+    red = before.clone().cuda()
+    buf.lb_prefetch_weights(red, ew.cuda(), torch.from_numpy(mapping).cuda())
+    assert buf.sync_status() == 0
+    np.testing.assert_array_equal(u16(red), oracle.lb_prefetch_weights(u16(ew), mapping, u16(before)))
+
+    grads = synth.expert_rows(93, E, W)
+    rg = synth.expert_rows(94, N, W)
+    g_d = grads.clone().cuda()
+    buf.lb_reduce_grads(rg.cuda(), g_d, torch.from_numpy(mapping).cuda())
+    assert buf.sync_status() == 0
+    ref = oracle.lb_reduce_grads(u16(rg), mapping, u16(grads))
+    abs_ref = oracle.lb_reduce_grads(bf16_abs(u16(rg)), mapping, bf16_abs(u16(grads)))
+    got = u16(g_d)
+    n_terms = 1 + int(np.bincount(mapping[mapping >= 0], minlength=E).max())
+    assert_combine_close(got, ref, abs_ref, n_terms, "lb reduce")
+    untouched = np.setdiff1d(np.arange(E), mapping)
+    np.testing.assert_array_equal(got[untouched], u16(grads)[untouched])
+    buf.destroy()
+
+
+def test_load_balance_bad_mapping_is_reported(ep):
+    w = synth.Workload("lb", 4, 8, 16, 64, 2, "uniform", 90)
+    buf = make_buffer(ep, w)
+    ew = torch.zeros((8, 64), dtype=torch.bfloat16, device="cuda")
+    red = torch.zeros((2, 64), dtype=torch.bfloat16, device="cuda")
+    buf.lb_prefetch_weights(red, ew, torch.tensor([1, 8], dtype=torch.int32, device="cuda"))
+    assert buf.sync_status() == 4
+    with pytest.raises(ep.EpError) as e:               # 60 values per expert: not whole 16-byte vectors
+        buf.lb_prefetch_weights(torch.zeros((2, 60), dtype=torch.bfloat16, device="cuda"),
+                                torch.zeros((8, 60), dtype=torch.bfloat16, device="cuda"),
+                                torch.tensor([1, 2], dtype=torch.int32, device="cuda"))
+    assert e.value.status == 2
     buf.destroy()
