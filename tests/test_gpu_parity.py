@@ -26,6 +26,12 @@ CASES = [
     synth.Workload("top1", 4, 8, 33, 64, 1, "uniform_masked", 98, num_channels=3, mask_prob=0.3),
     synth.Workload("one-rank", 1, 6, 40, 16, 2, "uniform_masked", 97, num_channels=4, mask_prob=0.3),
     synth.Workload("chan>T", 2, 4, 5, 8, 2, "uniform", 96, num_channels=12),
+    # limits: 32 ranks with top-32 (fan-out up to 32), the widest row, the narrowest row,
+    # the most experts
+    synth.Workload("R32-K32", 32, 64, 40, 64, 32, "uniform", 89, num_channels=5),
+    synth.Workload("H32768", 2, 4, 20, 32768, 2, "uniform", 88, num_channels=3),
+    synth.Workload("H8", 2, 4, 33, 8, 2, "uniform_masked", 87, num_channels=2, mask_prob=0.2),
+    synth.Workload("E4096", 8, 4096, 50, 16, 8, "uniform", 86, num_channels=4),
 ]
 
 
@@ -127,6 +133,7 @@ LL_CASES = [
     # more than 4096 tokens, and more than 16 slots: the tiled lookback slot scan
     synth.Workload("ll-big", 32, 256, 160, 64, 8, "uniform", 94),
     synth.Workload("ll-k20", 4, 64, 50, 32, 20, "uniform_masked", 93, mask_prob=0.1),
+    synth.Workload("ll-E4096", 8, 4096, 40, 128, 8, "uniform", 92),
 ]
 
 
