@@ -289,6 +289,16 @@ def ep_profile_read(ctx) -> dict:
 
 # ---------------------------------------------------------- convenience API
 
+_deferred: list = []     # contexts whose release waits for the end of a graph capture
+
+
+def _release_deferred():
+    if not _deferred or (torch.cuda.is_available() and torch.cuda.is_current_stream_capturing()):
+        return
+    while _deferred:
+        ep_destroy(_deferred.pop())
+
+
 class Buffer:
     """Dispatch/combine on R virtual ranks of one GPU, shaped like DeepEP's Buffer.
 
@@ -300,6 +310,7 @@ class Buffer:
                  ll_max_tokens_per_rank=0, device=None):
         self.device = (torch.device("cuda", torch.cuda.current_device()) if device is None
                        else torch.device(device))
+        _release_deferred()
         with torch.cuda.device(self.device):
             self.ctx = ep_create(num_ranks, num_experts, num_tokens, hidden, topk, num_channels,
                                  ll_max_tokens_per_rank)
@@ -309,13 +320,23 @@ class Buffer:
         self.Tmax = ll_max_tokens_per_rank or num_tokens
 
     def destroy(self):
+        _release_deferred()
         if self.ctx is not None:
             ep_destroy(self.ctx)
             self.ctx = None
 
     def __del__(self):
+        # The garbage collector may run this in the middle of a CUDA graph capture,
+        # where freeing device memory would invalidate the capture: the context is
+        # then released by the next Buffer created or destroyed outside a capture.
         try:
-            self.destroy()
+            if self.ctx is None:
+                return
+            if torch.cuda.is_available() and torch.cuda.is_current_stream_capturing():
+                _deferred.append(self.ctx)
+                self.ctx = None
+            else:
+                self.destroy()
         except Exception:
             pass
 
