@@ -4,11 +4,11 @@
 //
 // Entry point -> kernels (all on the caller's stream):
 //   ep_get_dispatch_layout : memset(histograms) + layout_kernel
-//   ep_dispatch            : [layout_kernel] + memset(scan state) + scan_kernel
+//   ep_dispatch            : [layout_kernel] + scan_kernel (call-tagged scan state, nothing to clear)
 //                            [+ one host read of N] + dispatch_kernel<normal>
 //   ep_dispatch_cached     : dispatch_kernel<cached>
 //   ep_combine             : combine_kernel
-//   ep_ll_dispatch[_fp8]   : memset(LL scan state) + ll_scan_kernel + dispatch_kernel<packed[, FP8]>
+//   ep_ll_dispatch[_fp8]   : ll_slot_kernel (call-tagged scan state, nothing to clear) + dispatch_kernel<packed[, FP8]>
 //   ep_ll_combine          : ll_combine_kernel
 //   ep_lb_prefetch_weights : lb_prefetch_kernel;  ep_lb_reduce_grads : lb_reduce_kernel
 
@@ -37,23 +37,18 @@ struct ep_ctx {
     char* ws;
     size_t ws_bytes;
     int* err;
-    char* scan_reset;           // status | ticket | done, zeroed before every scan
-    size_t scan_reset_bytes;
-    unsigned long long* scan_status;
-    int* scan_ticket;
-    int* scan_done;
+    unsigned long long* scan_status;   // [scan_tiles][R] call-tagged tile status (never cleared)
+    unsigned long long* scan_ticket;   // block ticket (only incremented)
     int scan_tiles;
-    int* boundary;              // [R][C+1][R]
+    unsigned long long* rank_start;    // [R][R] call-tagged P(s*T)[d] of the handle scan
     int* ntr_ws;                // [R][R]   (layout computed inside ep_dispatch)
     int* nte_ws;                // [R][E]
     int* slot_map;              // [G][K]   (low-latency slots)
-    char* ll_reset;             // LL scan: status | ticket | done, zeroed before every LL scan
-    size_t ll_reset_bytes;
-    unsigned long long* ll_status;
-    int* ll_ticket;
-    int* ll_done;
+    unsigned long long* ll_status;  // [ll_tiles][E] call-tagged tile status of the LL slot scan
+    unsigned long long* ll_src_begin;  // [R][E] call-tagged first slot per source
+    unsigned long long* ll_ticket;  // LL slot scan block ticket (only ever incremented)
+    int ll_tiles_per_src;
     int ll_tiles;
-    int* ll_boundary;           // [R+1][E]
     int* rank_mask;             // [R] low-latency rank mask (0 active, 1 masked)
     char last_error[256];
     bool prof;
@@ -234,17 +229,16 @@ int ep_create(const ep_config* cfg, ep_ctx** out) {
     const size_t off_err = off;            off += align256(sizeof(int));
     const size_t off_scan = off;
     const size_t status_bytes = (size_t)c->scan_tiles * c->R * sizeof(unsigned long long);
-    c->scan_reset_bytes = status_bytes + 2 * sizeof(int);
-    off += align256(c->scan_reset_bytes);
-    const size_t off_bnd = off;            off += align256((size_t)c->R * (c->C + 1) * c->R * sizeof(int));
+    off += align256(status_bytes + sizeof(unsigned long long));
+    const size_t off_rs = off;             off += align256((size_t)c->R * c->R * sizeof(unsigned long long));
     const size_t off_ntr = off;            off += align256((size_t)c->R * c->R * sizeof(int));
     const size_t off_nte = off;            off += align256((size_t)c->R * c->E * sizeof(int));
     const size_t off_slot = off;           off += align256((size_t)c->G * c->K * sizeof(int));
-    c->ll_tiles = (int)((c->G + ep::kLLTile - 1) / ep::kLLTile);
-    const size_t ll_status_bytes = (size_t)c->ll_tiles * c->E * sizeof(unsigned long long);
-    c->ll_reset_bytes = ll_status_bytes + 2 * sizeof(int);
-    const size_t off_ll = off;             off += align256(c->ll_reset_bytes);
-    const size_t off_llb = off;            off += align256((size_t)(c->R + 1) * c->E * sizeof(int));
+    c->ll_tiles_per_src = (c->T + ep::kLLTile - 1) / ep::kLLTile;
+    c->ll_tiles = c->R * c->ll_tiles_per_src;
+    const size_t off_lls = off;            off += align256((size_t)c->ll_tiles * c->E * sizeof(unsigned long long));
+    const size_t off_llb = off;            off += align256((size_t)c->R * c->E * sizeof(unsigned long long));
+    const size_t off_llc = off;            off += align256(sizeof(unsigned long long));
     const size_t off_mask = off;           off += align256((size_t)c->R * sizeof(int));
     c->ws_bytes = off;
     if (cudaMalloc(&c->ws, c->ws_bytes) != cudaSuccess) {
@@ -252,19 +246,15 @@ int ep_create(const ep_config* cfg, ep_ctx** out) {
         return EP_ERR_CUDA;
     }
     c->err = reinterpret_cast<int*>(c->ws + off_err);
-    c->scan_reset = c->ws + off_scan;
     c->scan_status = reinterpret_cast<unsigned long long*>(c->ws + off_scan);
-    c->scan_ticket = reinterpret_cast<int*>(c->ws + off_scan + status_bytes);
-    c->scan_done = c->scan_ticket + 1;
-    c->boundary = reinterpret_cast<int*>(c->ws + off_bnd);
+    c->scan_ticket = reinterpret_cast<unsigned long long*>(c->ws + off_scan + status_bytes);
+    c->rank_start = reinterpret_cast<unsigned long long*>(c->ws + off_rs);
     c->ntr_ws = reinterpret_cast<int*>(c->ws + off_ntr);
     c->nte_ws = reinterpret_cast<int*>(c->ws + off_nte);
     c->slot_map = reinterpret_cast<int*>(c->ws + off_slot);
-    c->ll_reset = c->ws + off_ll;
-    c->ll_status = reinterpret_cast<unsigned long long*>(c->ws + off_ll);
-    c->ll_ticket = reinterpret_cast<int*>(c->ws + off_ll + ll_status_bytes);
-    c->ll_done = c->ll_ticket + 1;
-    c->ll_boundary = reinterpret_cast<int*>(c->ws + off_llb);
+    c->ll_status = reinterpret_cast<unsigned long long*>(c->ws + off_lls);
+    c->ll_src_begin = reinterpret_cast<unsigned long long*>(c->ws + off_llb);
+    c->ll_ticket = reinterpret_cast<unsigned long long*>(c->ws + off_llc);
     c->rank_mask = reinterpret_cast<int*>(c->ws + off_mask);   // zeroed below: every rank active
     if (cudaMemset(c->ws, 0, c->ws_bytes) != cudaSuccess) rc = EP_ERR_CUDA;
     if (rc == EP_OK && ep::ll_prepare(c->E) != cudaSuccess) rc = EP_ERR_CUDA;
@@ -414,15 +404,12 @@ int ep_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, const flo
     }
 
     // 2. handle (prefix scan)
-    rc = cuda_check(c, cudaMemsetAsync(c->scan_reset, 0, c->scan_reset_bytes, s), "memset scan state");
-    if (rc != EP_OK) return rc;
     ep::ScanParams sp{};
     sp.is_token_in_rank = h->is_token_in_rank;
     sp.num_tokens_per_expert = nte;
     sp.status = c->scan_status;
     sp.ticket = c->scan_ticket;
-    sp.done = c->scan_done;
-    sp.boundary = c->boundary;
+    sp.rank_start = c->rank_start;
     sp.send_head = h->send_head;
     sp.rank_prefix_matrix = h->rank_prefix_matrix;
     sp.channel_prefix_matrix = h->channel_prefix_matrix;
@@ -557,11 +544,10 @@ int ll_dispatch_impl(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint
         if (e == cudaSuccess) e = cudaMemsetAsync(layout_range, 0, sizeof(int) * 2 * (size_t)c->E * c->R, s);
         return cuda_check(c, e, "zero low-latency counts");
     }
-    rc = cuda_check(c, cudaMemsetAsync(c->ll_reset, 0, c->ll_reset_bytes, s), "memset low-latency scan state");
-    if (rc != EP_OK) return rc;
     ep::LLCountParams cp{topk_idx, c->slot_map, packed_recv_count, src_info, layout_range,
-                         c->ll_status, c->ll_ticket, c->ll_done, c->ll_boundary, c->rank_mask, c->err,
-                         c->G, c->R, c->E, c->T, c->K, c->ll_cap, c->ll_tiles};
+                         c->ll_status, c->ll_src_begin, c->ll_ticket,
+                         c->rank_mask, c->err, c->G, c->R, c->E, c->T, c->K, c->ll_cap,
+                         c->ll_tiles_per_src, c->ll_tiles};
     rc = launch(c, kLLCount, true, s, [&] { return ep::launch_ll_count(cp, s); });
     if (rc != EP_OK) return rc;
     ep::DispatchParams dp{};

@@ -35,10 +35,9 @@ cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream);
 struct ScanParams {
     const uint8_t* is_token_in_rank;   // [G][R]
     const int* num_tokens_per_expert;  // [R][E]
-    unsigned long long* status;        // [num_tiles][R], zeroed before launch
-    int* ticket;                       // zeroed before launch
-    int* done;                         // zeroed before launch
-    int* boundary;                     // [R][C+1][R] workspace
+    unsigned long long* status;        // [num_tiles][R] call-tagged words (zero words never match)
+    unsigned long long* ticket;        // block ticket: only incremented (or zeroed with status)
+    unsigned long long* rank_start;    // [R][R] call-tagged P(s*T)[d] (zeroed with the ticket if at all)
     int* send_head;                    // [G][R]
     int* rank_prefix_matrix;           // [R][R]
     int* channel_prefix_matrix;        // [R][R][C]
@@ -110,16 +109,16 @@ struct LLCountParams {
     int* packed_recv_count;    // [E]  (= [R][L])
     int* src_info;             // [E][ll_cap]
     int* layout_range;         // [E][R][2]
-    unsigned long long* status;// [num_tiles][E], zeroed before launch
-    int* ticket;               // zeroed before launch
-    int* done;                 // zeroed before launch
-    int* boundary;             // [R+1][E] workspace
+    unsigned long long* status;    // [num_tiles][E] tile status words (call-tagged, never cleared)
+    unsigned long long* src_begin; // [R][E] first slot of each source (call-tagged), sources of > 1 tile
+    unsigned long long* ticket;    // block ticket, only ever incremented
     const int* rank_mask;      // [R], 0 active / 1 masked
     int* err;
     long long G;
     int R, E, T, K;
     int64_t ll_capacity;
-    int num_tiles;
+    int tiles_per_src;         // ceil(T / kLLTile)
+    int num_tiles;             // R * tiles_per_src
 };
 constexpr int kLLTile = 256;   // tokens per tile == threads per block
 cudaError_t launch_ll_count(const LLCountParams& p, cudaStream_t stream);

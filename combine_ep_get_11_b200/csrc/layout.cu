@@ -5,7 +5,8 @@
 // receives and which ranks each token goes to; the per-expert counts are the
 // receive counts of the "Code Examples" section.
 //
-// One thread per token.  The rank-hit set of a token is a 32-bit mask (R <= 32);
+// One thread per token, all its K ids loaded at once.  The rank-hit set of a
+// token is a 32-bit mask (R <= 32);
 // per-rank counts come from warp ballots + popc, per-expert counts from shared
 // memory atomics, and each block adds its counts to the global histograms.
 // The grid is (token blocks, source rank), so a block never straddles ranks.
@@ -23,31 +24,36 @@ __device__ __forceinline__ uint32_t spread4(uint32_t m) {
     return (m & 1u) | ((m & 2u) << 7) | ((m & 4u) << 14) | ((m & 8u) << 21);
 }
 
+template <int kMaxK>
 __global__ void __launch_bounds__(kLayoutThreads)
 layout_kernel(const LayoutParams p) {
     extern __shared__ int sh[];
     int* sh_rank = sh;        // [32]
     int* sh_expert = sh + 32; // [E]
     for (int i = threadIdx.x; i < 32 + p.E; i += blockDim.x) sh[i] = 0;
-    __syncthreads();
 
     const int s = blockIdx.y;
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t g = (int64_t)s * p.T + t;
+    int64_t ids[kMaxK];   // all of the token's ids in flight at once
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k) ids[k] = (t < p.T && k < p.K) ? __ldg(p.topk_idx + g * p.K + k) : -1;
+    __syncthreads();
+
     uint32_t mask = 0;
-    if (t < p.T) {
-        const int64_t g = (int64_t)s * p.T + t;
-        const int64_t* row = p.topk_idx + g * p.K;
-        bool bad = false;
-        for (int k = 0; k < p.K; ++k) {
-            const int64_t e = __ldg(row + k);
-            if (e == -1) continue;
-            if (e < -1 || e >= p.E) {
-                bad = true;
-                continue;
-            }
-            mask |= 1u << (int)(e / p.L);
-            atomicAdd(&sh_expert[e], 1);
+    bool bad = false;
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k) {
+        const int64_t e = ids[k];
+        if (e == -1) continue;
+        if (e < -1 || e >= p.E) {
+            bad = true;
+            continue;
         }
+        mask |= 1u << ((uint32_t)e / (uint32_t)p.L);
+        atomicAdd(&sh_expert[e], 1);
+    }
+    if (t < p.T) {
         if (bad) record_error(p.err, EP_ERR_BAD_TOPK);
         uint8_t* out = p.is_token_in_rank + g * p.R;
         if ((p.R & 3) == 0) {
@@ -75,7 +81,12 @@ cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream) {
     if (p.T == 0) return cudaSuccess;
     dim3 grid((p.T + kLayoutThreads - 1) / kLayoutThreads, p.R);
     const size_t smem = (32 + (size_t)p.E) * sizeof(int);
-    layout_kernel<<<grid, kLayoutThreads, smem, stream>>>(p);
+    if (p.K <= 8)
+        layout_kernel<8><<<grid, kLayoutThreads, smem, stream>>>(p);
+    else if (p.K <= 16)
+        layout_kernel<16><<<grid, kLayoutThreads, smem, stream>>>(p);
+    else
+        layout_kernel<32><<<grid, kLayoutThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 

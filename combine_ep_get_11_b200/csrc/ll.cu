@@ -9,11 +9,12 @@
 //
 // Slot order: the tokens of expert e are packed in (source rank, token) order,
 // so slot(s, t, e) = #{(s', t') < (s, t) naming e}: an exclusive running count
-// over the G tokens, one column per expert.  ll_scan_kernel computes all E
-// columns in one decoupled-lookback pass and writes src_info (token index per
-// slot), layout_range (first slot and count per source rank), the counts and a
-// [G][K] slot map for the copy kernel (the dispatch kernel's packed mode).  No
-// atomic decides an order, so the packing is deterministic.
+// over the G tokens, one column per expert.  ll_slot_kernel computes all E
+// columns in one decoupled-lookback pass over tiles of at most 256 tokens of
+// one source rank each, and writes src_info (token index per slot),
+// layout_range (first slot and count per source rank), the counts and a [G][K]
+// slot map for the copy kernel (the dispatch kernel's packed mode).  No atomic
+// decides an order, so the packing is deterministic.
 //
 // ll_combine_kernel: one warp per token.  Lane k finds the slot of its expert
 // by binary search in src_info inside layout_range[e][s] (ascending token
@@ -32,72 +33,134 @@ constexpr int kLLCombineWarps = kLLCombineThreads / 32;
 constexpr int kLLRowsPerGroup = 8;
 constexpr int kLLWords = kLLTile / 32;
 constexpr int kLLStride = kLLWords + 1;   // odd row stride: no shared-memory bank conflicts
-constexpr unsigned long long kLLFlagAggregate = 1ull << 62;
-constexpr unsigned long long kLLFlagInclusive = 2ull << 62;
+constexpr int kLLWindow = 16;             // predecessor tiles read at once in the lookback
+// Tile status word: count in bits 0-31, flag in bits 32-33, call epoch in bits 34-63.
+constexpr unsigned long long kLLFlagAggregate = 1ull << 32;
+constexpr unsigned long long kLLFlagInclusive = 2ull << 32;
+constexpr unsigned long long kLLFlagMask = 3ull << 32;
+constexpr unsigned long long kLLTagMask = ~0ull << 34;
+constexpr int kLLEpochShift = 34;
 
-__host__ __device__ inline size_t ll_scan_smem(int E) {
-    return (size_t)E * kLLStride * sizeof(uint32_t) + (size_t)E * sizeof(int);
+__host__ __device__ inline size_t ll_slot_smem(int E) {
+    return (size_t)E * kLLStride * sizeof(uint32_t)   // membership bitmap
+           + (size_t)E * sizeof(int)                  // exclusive prefix per expert
+           + (size_t)E * kLLWords                     // members before each word (<= 224)
+           + (size_t)E;                               // expert on a masked rank
 }
 
-// One 256-token tile per block (ticket order).  Each thread owns one token:
-// its experts set one bit each in the tile's [E][8]-word membership bitmap (a
-// token naming an expert twice sets the same bit).  Thread e then publishes
-// expert e's tile count and looks back over earlier tiles for the exclusive
-// prefix (bounded wait); a member's slot is that prefix plus the members of the
-// expert earlier in the tile.  Samples of the running counts at each source
-// rank's first token go to `boundary`; the last tile to finish turns them into
-// layout_range and the per-expert counts.
+__device__ __forceinline__ bool ll_published(unsigned long long v, unsigned long long tag) {
+    return (v & kLLTagMask) == tag && (v & kLLFlagMask) != 0;
+}
+
+// Tiles: source rank s is cut into m = ceil(T/256) tiles of at most 256 of its
+// tokens, numbered s*m + j in token order.  Blocks take tickets from one 64-bit
+// counter that is never reset: ticket = call * num_tiles + tile, so a tile
+// only waits on tiles that already started, and the call number tags every
+// status word (words left by an earlier call never match; nothing is cleared
+// between calls).  Each thread owns one token: its experts set one bit each in
+// the tile's [E][8]-word membership bitmap (a token naming an expert twice
+// sets the same bit).  Thread e then publishes expert e's tile count and looks
+// back over earlier tiles, 16 status words loaded at once per round and summed
+// up to the first inclusive prefix (while a word before it is unpublished, the
+// window is re-read, with a bounded wait).  A member's slot is that prefix
+// plus the members of the expert earlier in the tile.  The first tile of a
+// source writes layout_range's start; its last tile the count (reading the
+// start from a tagged word when the source spans several tiles); the last tile
+// of all the per-expert totals.
 template <int kMaxK>
-__global__ void __launch_bounds__(kLLTile)
-ll_scan_kernel(const LLCountParams p) {
+__global__ void __launch_bounds__(kLLTile, 1)
+ll_slot_kernel(const LLCountParams p) {
     extern __shared__ uint32_t ll_smem[];
-    uint32_t* bits = ll_smem;                                       // [E][kLLStride]
-    int* s_excl = reinterpret_cast<int*>(ll_smem + (size_t)p.E * kLLStride);  // [E]
-    __shared__ int s_tile, s_last;
-    const int tid = threadIdx.x;
     const int E = p.E;
-    if (tid == 0) s_tile = atomicAdd(p.ticket, 1);
-    for (int i = tid; i < E * kLLStride; i += kLLTile) bits[i] = 0;
+    uint32_t* bits = ll_smem;                                                 // [E][kLLStride]
+    int* s_excl = reinterpret_cast<int*>(bits + (size_t)E * kLLStride);       // [E]
+    uint8_t* s_wpref = reinterpret_cast<uint8_t*>(s_excl + E);                // [E][kLLWords]
+    uint8_t* s_dead = s_wpref + (size_t)E * kLLWords;                         // [E]
+    __shared__ int s_tile;
+    __shared__ unsigned long long s_tag;
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        const unsigned long long tk = atomicAdd(p.ticket, 1ull);
+        s_tile = (int)(tk % (unsigned long long)p.num_tiles);
+        s_tag = (tk / (unsigned long long)p.num_tiles + 1) << kLLEpochShift;   // never 0
+    }
+    const int lane = tid & 31;   // masked ranks (R <= 32): one load per lane, in every warp
+    const uint32_t mbits = __ballot_sync(kFullMask, lane < p.R && p.rank_mask[lane] != 0);
+    const int L = E / p.R;
+    for (int e = tid; e < E; e += kLLTile) {
+#pragma unroll
+        for (int q = 0; q < kLLStride; ++q) bits[e * kLLStride + q] = 0;
+        s_dead[e] = (uint8_t)((mbits >> (e / L)) & 1u);
+    }
     __syncthreads();
     const int tile = s_tile;
-    const long long g0 = (long long)tile * kLLTile;
-    const long long g = g0 + tid;
+    const unsigned long long tag = s_tag;
+    const int m = p.tiles_per_src;
+    const int s = tile / m, j = tile - s * m;
+    const int t = j * kLLTile + tid;                        // token of this thread in source s
+    const int n = min(kLLTile, p.T - j * kLLTile);          // tokens in the tile
+    const long long g = (long long)s * p.T + t;
+    const bool src_live = ((mbits >> s) & 1u) == 0;        // a masked rank sends nothing
     const int w = tid >> 5, b = tid & 31;
 
-    int64_t ids[kMaxK];
-#pragma unroll
-    for (int k = 0; k < kMaxK; ++k) ids[k] = (g < p.G && k < p.K) ? __ldg(p.topk_idx + g * p.K + k) : -1;
-    // a slot from or to a masked rank is not part of the exchange
-    const int L = E / p.R;
-    const bool src_masked = g < p.G && p.rank_mask[g / p.T] != 0;
+    int ids[kMaxK];
     bool bad = false;
 #pragma unroll
     for (int k = 0; k < kMaxK; ++k) {
-        const int64_t e = ids[k];
-        if (e < -1 || e >= E) { bad = true; ids[k] = -1; continue; }
-        if (e >= 0 && (src_masked || p.rank_mask[e / L] != 0)) ids[k] = -1;
-        if (ids[k] >= 0) atomicOr(&bits[e * kLLStride + w], 1u << b);
+        const int64_t e = (tid < n && k < p.K) ? __ldg(p.topk_idx + g * p.K + k) : -1;
+        bad |= e < -1 || e >= E;
+        ids[k] = (e >= 0 && e < E && src_live && !s_dead[(int)e]) ? (int)e : -1;
     }
     if (bad) record_error(p.err, EP_ERR_BAD_TOPK);
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k)
+        if (ids[k] >= 0) atomicOr(&bits[ids[k] * kLLStride + w], 1u << b);
     __syncthreads();
 
+    const bool last_of_src = j == m - 1, last_tile = tile == p.num_tiles - 1;
     for (int e = tid; e < E; e += kLLTile) {
         int agg = 0;
 #pragma unroll
-        for (int q = 0; q < kLLWords; ++q) agg += __popc(bits[e * kLLStride + q]);
+        for (int q = 0; q < kLLWords; ++q) {
+            s_wpref[e * kLLWords + q] = (uint8_t)agg;
+            agg += __popc(bits[e * kLLStride + q]);
+        }
         unsigned long long* mine = p.status + (size_t)tile * E + e;
-        int excl = 0;
+        long long excl = 0;
         if (tile == 0) {
-            st_relaxed_u64(mine, kLLFlagInclusive | (unsigned)agg);
+            st_relaxed_u64(mine, tag | kLLFlagInclusive | (unsigned)agg);
         } else {
-            st_relaxed_u64(mine, kLLFlagAggregate | (unsigned)agg);
-            int j = tile - 1;
+            st_relaxed_u64(mine, tag | kLLFlagAggregate | (unsigned)agg);
+            int top = tile - 1;             // newest tile of the current window
+            bool found = false;
             uint64_t t0 = 0;
             uint32_t spins = 0;
-            while (j >= 0) {
-                const unsigned long long v = ld_relaxed_u64(p.status + (size_t)j * E + e);
-                const unsigned long long flag = v & (3ull << 62);
-                if (flag == 0) {
+            while (top >= 0 && !found) {
+                const int cnt = min(kLLWindow, top + 1);
+                unsigned long long v[kLLWindow];
+                bool ok = false;
+                int take = 0;
+                for (;;) {
+#pragma unroll
+                    for (int u = 0; u < kLLWindow; ++u)
+                        v[u] = u < cnt ? ld_relaxed_u64(p.status + (size_t)(top - u) * E + e) : 0ull;
+                    // words are needed only up to the first inclusive one
+                    ok = true;
+                    found = false;
+                    take = cnt;
+#pragma unroll
+                    for (int u = 0; u < kLLWindow; ++u) {
+                        if (u < take) {
+                            if (!ll_published(v[u], tag)) {
+                                ok = false;
+                                take = u;
+                            } else if ((v[u] & kLLFlagMask) == kLLFlagInclusive) {
+                                found = true;
+                                take = u + 1;
+                            }
+                        }
+                    }
+                    if (ok) break;
                     if (spins == 0) t0 = globaltimer_ns();
                     ++spins;
                     if (spins > kWaitLimitIters ||
@@ -105,28 +168,51 @@ ll_scan_kernel(const LLCountParams p) {
                         record_error(p.err, EP_ERR_TIMEOUT);
                         break;
                     }
-                    continue;
                 }
-                excl += (int)(uint32_t)v;
-                if (flag == kLLFlagInclusive) break;
-                --j;
+                if (!ok) break;
+#pragma unroll
+                for (int u = 0; u < kLLWindow; ++u)
+                    if (u < take) excl += (uint32_t)v[u];
+                top -= cnt;
             }
-            st_relaxed_u64(mine, kLLFlagInclusive | (unsigned)(excl + agg));
+            st_relaxed_u64(mine, tag | kLLFlagInclusive | (unsigned)(excl + agg));
         }
-        s_excl[e] = excl;
+        s_excl[e] = (int)excl;
+
+        // layout_range[e][s] = (first slot of source s, its count); the per-expert totals
+        int* lr = p.layout_range + ((long long)e * p.R + s) * 2;
+        long long begin = excl;
+        if (j == 0) {
+            lr[0] = (int)excl;
+            if (m > 1) st_relaxed_u64(p.src_begin + (size_t)s * E + e, tag | kLLFlagInclusive | (unsigned)excl);
+        } else if (last_of_src) {   // the source's first tile started earlier: bounded wait for its start
+            unsigned long long v = ld_relaxed_u64(p.src_begin + (size_t)s * E + e);
+            uint32_t sp = 0;
+            uint64_t ts = 0;
+            while (!ll_published(v, tag)) {
+                if (sp == 0) ts = globaltimer_ns();
+                ++sp;
+                if (sp > kWaitLimitIters || ((sp & 63u) == 0 && globaltimer_ns() - ts > kWaitLimitNs)) {
+                    record_error(p.err, EP_ERR_TIMEOUT);
+                    break;
+                }
+                v = ld_relaxed_u64(p.src_begin + (size_t)s * E + e);
+            }
+            begin = (uint32_t)v;
+        }
+        if (last_of_src) lr[1] = (int)(excl + agg - begin);
+        if (last_tile) p.packed_recv_count[e] = (int)(excl + agg);
     }
     __syncthreads();
 
-    const long long cap = p.ll_capacity;
-    if (g < p.G) {
-        const int t = (int)(g % p.T);
+    if (tid < n) {
+        const long long cap = p.ll_capacity;
+        const uint32_t below = (1u << b) - 1u;
 #pragma unroll
         for (int k = 0; k < kMaxK; ++k) {
-            const int64_t e = ids[k];
+            const int e = ids[k];
             if (e < 0) continue;
-            const uint32_t* be = bits + e * kLLStride;
-            int slot = s_excl[e] + __popc(be[w] & ((1u << b) - 1u));
-            for (int q = 0; q < w; ++q) slot += __popc(be[q]);
+            const int slot = s_excl[e] + s_wpref[e * kLLWords + w] + __popc(bits[e * kLLStride + w] & below);
             if (slot < cap) {
                 p.slot_map[g * p.K + k] = slot;
                 p.src_info[e * cap + slot] = t;
@@ -135,55 +221,6 @@ ll_scan_kernel(const LLCountParams p) {
             }
         }
     }
-
-    // running counts at source starts s*T (s = 0..R; s*T == G belongs to the last tile)
-    const bool last_tile = tile == p.num_tiles - 1;
-    const int s_lo = (int)((g0 + p.T - 1) / p.T);
-    const int s_hi = (int)min((long long)p.R, (g0 + kLLTile) / p.T);
-    for (int s = s_lo; s <= s_hi; ++s) {
-        const long long gb = (long long)s * p.T;
-        const bool mine = (gb >= g0 && gb < g0 + kLLTile && gb < p.G) || (gb == p.G && last_tile);
-        if (!mine) continue;
-        const int rel = (int)(gb - g0);    // 0..256
-        for (int e = tid; e < E; e += kLLTile) {
-            const uint32_t* be = bits + e * kLLStride;
-            int cnt = 0;
-            for (int q = 0; q < (rel >> 5); ++q) cnt += __popc(be[q]);
-            if ((rel >> 5) < kLLWords) cnt += __popc(be[rel >> 5] & ((1u << (rel & 31)) - 1u));
-            p.boundary[(long long)s * E + e] = s_excl[e] + cnt;
-        }
-    }
-
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(p.done, 1) == p.num_tiles - 1;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    // loads of each batch before its stores, so the L2 round trips overlap
-    constexpr int kBatch = 8;
-    const int nr = E * p.R;
-    for (int i0 = 0; i0 < nr; i0 += kLLTile * kBatch) {
-        int vb[kBatch], vn[kBatch];
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int i = i0 + u * kLLTile + tid;   // i = e*R + s
-            if (i < nr) {
-                const int e = i / p.R, s = i % p.R;
-                vb[u] = __ldcg(p.boundary + (long long)s * E + e);
-                vn[u] = __ldcg(p.boundary + (long long)(s + 1) * E + e);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int i = i0 + u * kLLTile + tid;
-            if (i < nr) {
-                p.layout_range[(long long)i * 2 + 0] = vb[u];
-                p.layout_range[(long long)i * 2 + 1] = vn[u] - vb[u];
-            }
-        }
-    }
-    for (int e = tid; e < E; e += kLLTile) p.packed_recv_count[e] = __ldcg(p.boundary + (long long)p.R * E + e);
 }
 
 __device__ __forceinline__ void fma_bf16x8(float* acc, float w, const uint4& v) {
@@ -311,25 +348,25 @@ cudaError_t launch_set_mask(int* rank_mask, int rank, int value, cudaStream_t st
 
 cudaError_t ll_prepare(int E) {
     // opt in to large dynamic shared memory when E needs it
-    const size_t smem = ll_scan_smem(E);
+    const size_t smem = ll_slot_smem(E);
     if (smem <= 48 * 1024) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(ll_scan_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(ll_slot_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(ll_scan_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = cudaFuncSetAttribute(ll_slot_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(ll_scan_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = cudaFuncSetAttribute(ll_slot_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     return e;
 }
 
 cudaError_t launch_ll_count(const LLCountParams& p, cudaStream_t stream) {
     if (p.G == 0 || p.E == 0) return cudaSuccess;
-    const size_t smem = ll_scan_smem(p.E);
+    const size_t smem = ll_slot_smem(p.E);
     if (p.K <= 8)
-        ll_scan_kernel<8><<<p.num_tiles, kLLTile, smem, stream>>>(p);
+        ll_slot_kernel<8><<<p.num_tiles, kLLTile, smem, stream>>>(p);
     else if (p.K <= 16)
-        ll_scan_kernel<16><<<p.num_tiles, kLLTile, smem, stream>>>(p);
+        ll_slot_kernel<16><<<p.num_tiles, kLLTile, smem, stream>>>(p);
     else
-        ll_scan_kernel<32><<<p.num_tiles, kLLTile, smem, stream>>>(p);
+        ll_slot_kernel<32><<<p.num_tiles, kLLTile, smem, stream>>>(p);
     return cudaGetLastError();
 }
 

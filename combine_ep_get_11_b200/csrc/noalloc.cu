@@ -6,8 +6,8 @@
 // fixed budget, or code that must not risk the device-wide synchronisation that
 // cudaMalloc/cudaFree can cause.  ep_create allocates a workspace, so those
 // callers cannot use the context-based calls.  This entry point needs no
-// context: the scan's scratch (tile status flags, tile ticket, finish counter
-// and the channel-boundary samples) lives in the file-scope array below, which
+// context: the scan's scratch (tile status words, the tile ticket and the
+// rank-start words) lives in the file-scope array below, which
 // every GPU that loads the library holds until the process exits.  The caller
 // still passes all inputs and outputs.
 //
@@ -27,7 +27,7 @@ namespace {
 static __device__ __align__(256) unsigned char g_static_scratch[EP_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-constexpr size_t kCounterBytes = 256;   // ticket + finish counter, padded
+constexpr size_t kCounterBytes = 256;   // the tile ticket, padded
 
 std::mutex g_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
@@ -77,8 +77,8 @@ extern "C" EP_API int ep_dispatch_handle_static(int32_t num_ranks, int32_t num_e
 
     const int tiles = (int)((G + ep::kScanTile - 1) / ep::kScanTile);
     const size_t status_bytes = (size_t)tiles * R * sizeof(unsigned long long);
-    const size_t boundary_bytes = (size_t)R * (C + 1) * R * sizeof(int);
-    if (kCounterBytes + round256(status_bytes) + boundary_bytes > EP_STATIC_SCRATCH_BYTES)
+    const size_t rank_start_bytes = (size_t)R * R * sizeof(unsigned long long);
+    if (kCounterBytes + round256(status_bytes) + rank_start_bytes > EP_STATIC_SCRATCH_BYTES)
         return EP_ERR_CAPACITY;   // the problem needs more scratch than the static array holds
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -95,17 +95,18 @@ extern "C" EP_API int ep_dispatch_handle_static(int32_t num_ranks, int32_t num_e
     void* base = nullptr;
     if (scratch_address(&base) != cudaSuccess) return EP_ERR_CUDA;
     unsigned char* scratch = static_cast<unsigned char*>(base);
-    // The array keeps the previous call's contents: the counters and flags must
-    // start at zero (the boundary samples are fully rewritten before use).
-    if (cudaMemsetAsync(scratch, 0, kCounterBytes + status_bytes, s) != cudaSuccess) return EP_ERR_CUDA;
+    // The array keeps the previous call's contents, possibly from a call of
+    // another shape: the ticket, status and rank-start words start at zero on
+    // every call (the ticket restarts at call 0; zeroed words never match its tag).
+    if (cudaMemsetAsync(scratch, 0, kCounterBytes + round256(status_bytes) + rank_start_bytes, s) != cudaSuccess)
+        return EP_ERR_CUDA;
 
     ep::ScanParams p{};
     p.is_token_in_rank = is_token_in_rank;
     p.num_tokens_per_expert = num_tokens_per_expert;
-    p.ticket = reinterpret_cast<int*>(scratch);
-    p.done = reinterpret_cast<int*>(scratch) + 1;
+    p.ticket = reinterpret_cast<unsigned long long*>(scratch);
     p.status = reinterpret_cast<unsigned long long*>(scratch + kCounterBytes);
-    p.boundary = reinterpret_cast<int*>(scratch + kCounterBytes + round256(status_bytes));
+    p.rank_start = reinterpret_cast<unsigned long long*>(scratch + kCounterBytes + round256(status_bytes));
     p.send_head = handle->send_head;
     p.rank_prefix_matrix = handle->rank_prefix_matrix;
     p.channel_prefix_matrix = handle->channel_prefix_matrix;

@@ -321,7 +321,7 @@ EP_API int ep_lb_reduce_grads(ep_ctx* ctx, const uint16_t* redundant_grads, int6
  *   error_word            nullable device int32, zeroed by the caller; a device
  *                         wait that runs out stores EP_ERR_TIMEOUT there
  * Limits as for ep_config; in addition the scratch it needs,
- *   256 + round_up(8 * R * ceil(R*T / 256), 256) + 4 * R * R * (C + 1) bytes,
+ *   256 + round_up(8 * R * ceil(R*T / 256), 256) + 8 * R * R bytes,
  * must fit in EP_STATIC_SCRATCH_BYTES, or the call returns EP_ERR_CAPACITY
  * before launching anything (R = 32, T = 8192, C = 10 needs about 300 KiB).
  * The first call on a device looks up the array's device address (once, with

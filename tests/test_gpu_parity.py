@@ -130,10 +130,12 @@ LL_CASES = [
     dataclasses.replace(W["ll"].scaled(num_tokens=50, hidden=256), max_tokens_per_rank=64,
                         name="ll-tmax64"),
     synth.Workload("ll-odd", 3, 12, 30, 40, 5, "uniform_masked", 95, mask_prob=0.2),
-    # more than 4096 tokens, and more than 16 slots: the tiled lookback slot scan
+    # more than two 2048-token chunks of the slot kernel, 32 ranks
     synth.Workload("ll-big", 32, 256, 160, 64, 8, "uniform", 94),
     synth.Workload("ll-k20", 4, 64, 50, 32, 20, "uniform_masked", 93, mask_prob=0.1),
     synth.Workload("ll-E4096", 8, 4096, 40, 128, 8, "uniform", 92),
+    # sources longer than one 256-token slot tile (3 tiles each, the last one ragged)
+    synth.Workload("ll-T600", 4, 32, 600, 64, 4, "uniform_masked", 91, mask_prob=0.1),
 ]
 
 
@@ -164,6 +166,42 @@ def test_low_latency(ep, w):
         abs_ref = oracle.ll_combine(bf16_abs(y_u16), inp.topk, np.abs(inp.weights), ll["src_info"],
                                     ll["layout_range"], w.num_experts, w.tmax)
         assert_combine_close(u16(out), ref, abs_ref, w.topk, "ll combine")
+    assert buf.sync_status() == 0
+    buf.destroy()
+
+
+# ----------------------------------------------------------------------------- repeated calls
+
+def test_repeated_calls_on_one_context(ep):
+    """The scans keep their status words between calls (tagged with the call): calls
+    with other routings on the same context must not see a previous call's words."""
+    base = W["dsv3"].scaled(num_tokens=700, hidden=64)           # 5600 tokens: 22 scan tiles
+    buf = make_buffer(ep, base)
+    for seed in (base.seed, base.seed + 1, base.seed, base.seed + 2):
+        w = dataclasses.replace(base, seed=seed)
+        inp = Inputs(w)
+        _, h, (o_recv_x, _, _) = oracle_normal(inp)
+        recv_x, _, _, handle = buf.dispatch(inp.x_d, inp.topk_d, inp.weights_d)
+        for key in HANDLE_KEYS:
+            np.testing.assert_array_equal(getattr(handle, key).cpu().numpy(), h[key], err_msg=key)
+        np.testing.assert_array_equal(u16(recv_x), o_recv_x)
+    assert buf.sync_status() == 0
+    buf.destroy()
+
+    base = synth.Workload("ll-rep", 8, 64, 300, 64, 6, "uniform_masked", 84, mask_prob=0.1)
+    buf = make_buffer(ep, base)
+    for seed in (base.seed, base.seed + 1, base.seed, base.seed + 2):
+        w = dataclasses.replace(base, seed=seed)
+        inp = Inputs(w)
+        packed, count, (src_info, layout_range) = buf.low_latency_dispatch(inp.x_d, inp.topk_d)
+        ll = oracle.ll_dispatch(inp.x_u16, inp.topk, w.num_experts, w.tmax)
+        np.testing.assert_array_equal(count.cpu().numpy(), ll["packed_recv_count"])
+        np.testing.assert_array_equal(layout_range.cpu().numpy(), ll["layout_range"])
+        si = src_info.cpu().numpy()
+        for d in range(w.num_ranks):
+            for j in range(w.local_experts):
+                n = int(ll["packed_recv_count"][d, j])
+                np.testing.assert_array_equal(si[d, j, :n], ll["src_info"][d, j, :n])
     assert buf.sync_status() == 0
     buf.destroy()
 
