@@ -82,6 +82,18 @@ _SIGNATURES = {
     "ep_ll_update_mask": (ctypes.c_int, [_vp, _i32, _i32, _vp]),
     "ep_ll_query_mask": (ctypes.c_int, [_vp, _vp, _vp]),
     "ep_ll_clean_mask": (ctypes.c_int, [_vp, _vp]),
+    "ep_create_sharded": (ctypes.c_int, [ctypes.POINTER(ep_config), ctypes.c_int, ctypes.c_int,
+                                         ctypes.POINTER(_vp)]),
+    "ep_sharded_handle": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "ep_sharded_dispatch": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.POINTER(_vp),
+                                           ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp),
+                                           _i64, _vp, _vp]),
+    "ep_sharded_combine": (ctypes.c_int, [_vp, ctypes.c_int, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _i64,
+                                          _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "ep_shared_alloc": (ctypes.c_int, [ctypes.c_size_t, ctypes.POINTER(_vp), ctypes.POINTER(ctypes.c_uint8)]),
+    "ep_shared_free": (ctypes.c_int, [_vp]),
+    "ep_ipc_open": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(_vp)]),
+    "ep_ipc_close": (ctypes.c_int, [_vp]),
     "ep_profile_enable": (ctypes.c_int, [_vp, ctypes.c_int]),
     "ep_profile_read": (ctypes.c_int, [_vp, ctypes.POINTER(_i64), ctypes.POINTER(ctypes.c_double)]),
 }

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build", "libep")
 LIB = os.path.join(PKG, "libep.so")
-SOURCES = ["abi.cu", "layout.cu", "scan.cu", "dispatch.cu", "combine.cu", "ll.cu", "lb.cu", "noalloc.cu"]
+SOURCES = ["abi.cu", "layout.cu", "scan.cu", "dispatch.cu", "combine.cu", "ll.cu", "lb.cu", "noalloc.cu", "shard.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

@@ -29,7 +29,9 @@ struct ep_prof_rec {
 struct ep_ctx {
     ep_config cfg;
     int R, E, L, T, H, K, C, Tmax;
-    long long G;
+    long long G;                // tokens of this context's source ranks: Rl * T
+    int num_shards, shard;      // sharded exchange: this GPU hosts ranks [r0, r0 + Rl)
+    int Rl, r0;                 // (one shard: Rl = R, r0 = 0)
     int64_t ll_cap;
     int device;
     int num_sms;
@@ -50,6 +52,7 @@ struct ep_ctx {
     int ll_tiles_per_src;
     int ll_tiles;
     int* rank_mask;             // [R] low-latency rank mask (0 active, 1 masked)
+    int* shard_base;            // [R] tokens of earlier shards per destination (sharded scan base)
     char last_error[256];
     bool prof;
     std::vector<ep_prof_rec> pending;
@@ -192,11 +195,18 @@ const char* ep_status_string(int status) {
 
 uint64_t ep_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
-int ep_create(const ep_config* cfg, ep_ctx** out) {
+}  // extern "C"
+
+namespace {
+
+int create_impl(const ep_config* cfg, int num_shards, int shard, ep_ctx** out) {
     if (out == nullptr) return EP_ERR_INVALID_ARG;
     *out = nullptr;
     const int v = validate_config(cfg);
     if (v != EP_OK) return v;
+    if (num_shards < 1 || num_shards > ep::kMaxShards || cfg->num_ranks % num_shards != 0 || shard < 0 ||
+        shard >= num_shards)
+        return EP_ERR_INVALID_ARG;
 
     ep_ctx* c = new ep_ctx();
     c->cfg = *cfg;
@@ -208,7 +218,11 @@ int ep_create(const ep_config* cfg, ep_ctx** out) {
     c->K = cfg->topk;
     c->C = cfg->num_channels;
     c->Tmax = cfg->ll_max_tokens_per_rank ? cfg->ll_max_tokens_per_rank : cfg->num_tokens;
-    c->G = (long long)c->R * c->T;
+    c->num_shards = num_shards;
+    c->shard = shard;
+    c->Rl = c->R / num_shards;
+    c->r0 = shard * c->Rl;
+    c->G = (long long)c->Rl * c->T;
     c->ll_cap = (int64_t)c->R * c->Tmax;
 
     int rc = EP_OK;
@@ -240,6 +254,7 @@ int ep_create(const ep_config* cfg, ep_ctx** out) {
     const size_t off_llb = off;            off += align256((size_t)c->R * c->E * sizeof(unsigned long long));
     const size_t off_llc = off;            off += align256(sizeof(unsigned long long));
     const size_t off_mask = off;           off += align256((size_t)c->R * sizeof(int));
+    const size_t off_sbase = off;          off += align256((size_t)c->R * sizeof(int));
     c->ws_bytes = off;
     if (cudaMalloc(&c->ws, c->ws_bytes) != cudaSuccess) {
         delete c;
@@ -256,6 +271,7 @@ int ep_create(const ep_config* cfg, ep_ctx** out) {
     c->ll_src_begin = reinterpret_cast<unsigned long long*>(c->ws + off_llb);
     c->ll_ticket = reinterpret_cast<unsigned long long*>(c->ws + off_llc);
     c->rank_mask = reinterpret_cast<int*>(c->ws + off_mask);   // zeroed below: every rank active
+    c->shard_base = reinterpret_cast<int*>(c->ws + off_sbase);
     if (cudaMemset(c->ws, 0, c->ws_bytes) != cudaSuccess) rc = EP_ERR_CUDA;
     if (rc == EP_OK && ep::ll_prepare(c->E) != cudaSuccess) rc = EP_ERR_CUDA;
     if (rc != EP_OK) {
@@ -265,6 +281,16 @@ int ep_create(const ep_config* cfg, ep_ctx** out) {
     }
     *out = c;
     return EP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ep_create(const ep_config* cfg, ep_ctx** out) { return create_impl(cfg, 1, 0, out); }
+
+int ep_create_sharded(const ep_config* cfg, int num_shards, int shard, ep_ctx** out) {
+    return create_impl(cfg, num_shards, shard, out);
 }
 
 int ep_destroy(ep_ctx* c) {
@@ -337,12 +363,12 @@ int ep_get_dispatch_layout(ep_ctx* c, const int64_t* topk_idx, int32_t* num_toke
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     int rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
     if (rc != EP_OK) return rc;
-    rc = cuda_check(c, cudaMemsetAsync(num_tokens_per_rank, 0, sizeof(int) * c->R * c->R, s), "memset");
+    rc = cuda_check(c, cudaMemsetAsync(num_tokens_per_rank, 0, sizeof(int) * c->Rl * c->R, s), "memset");
     if (rc == EP_OK)
-        rc = cuda_check(c, cudaMemsetAsync(num_tokens_per_expert, 0, sizeof(int) * (size_t)c->R * c->E, s), "memset");
+        rc = cuda_check(c, cudaMemsetAsync(num_tokens_per_expert, 0, sizeof(int) * (size_t)c->Rl * c->E, s), "memset");
     if (rc != EP_OK) return rc;
     ep::LayoutParams p{topk_idx, is_token_in_rank, num_tokens_per_rank, num_tokens_per_expert, c->err,
-                       c->R, c->E, c->L, c->T, c->K};
+                       c->R, c->E, c->L, c->T, c->K, c->Rl};
     return launch(c, kLayout, c->G > 0, s, [&] { return ep::launch_layout(p, s); });
 }
 
@@ -352,6 +378,7 @@ int ep_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, const flo
                 int64_t* recv_topk_idx, float* recv_topk_weights, int64_t recv_capacity_rows,
                 int64_t* num_recv_host, ep_stream_t stream, ep_event_t wait_event) {
     if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (c->num_shards > 1) return fail(c, EP_ERR_INVALID_ARG, "sharded context: use the ep_sharded_* calls");
     int rc = check_handle(c, h);
     if (rc != EP_OK) return rc;
     if (recv_capacity_rows < 0) return fail(c, EP_ERR_INVALID_ARG, "negative capacity");
@@ -393,7 +420,8 @@ int ep_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, const flo
         rc = cuda_check(c, cudaMemsetAsync(c->ntr_ws, 0, sizeof(int) * c->R * c->R, s), "memset");
         if (rc == EP_OK) rc = cuda_check(c, cudaMemsetAsync(c->nte_ws, 0, sizeof(int) * (size_t)c->R * c->E, s), "memset");
         if (rc != EP_OK) return rc;
-        ep::LayoutParams lp{topk_idx, h->is_token_in_rank, c->ntr_ws, c->nte_ws, c->err, c->R, c->E, c->L, c->T, c->K};
+        ep::LayoutParams lp{topk_idx, h->is_token_in_rank, c->ntr_ws, c->nte_ws, c->err, c->R, c->E, c->L, c->T, c->K,
+                            c->R};
         rc = launch(c, kLayout, c->G > 0, s, [&] { return ep::launch_layout(lp, s); });
         if (rc != EP_OK) return rc;
         nte = c->nte_ws;
@@ -458,6 +486,7 @@ int ep_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, const flo
 int ep_dispatch_cached(ep_ctx* c, const uint16_t* x, const ep_handle* h, uint16_t* recv_x,
                        int64_t recv_capacity_rows, ep_stream_t stream, ep_event_t wait_event) {
     if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (c->num_shards > 1) return fail(c, EP_ERR_INVALID_ARG, "sharded context: use the ep_sharded_* calls");
     int rc = check_handle(c, h);
     if (rc != EP_OK) return rc;
     if (recv_capacity_rows < 0) return fail(c, EP_ERR_INVALID_ARG, "negative capacity");
@@ -486,6 +515,7 @@ int ep_combine(ep_ctx* c, const uint16_t* y, int64_t num_recv_rows, const ep_han
                const float* recv_topk_weights, const uint16_t* bias0, const uint16_t* bias1,
                uint16_t* out_x, float* out_topk_weights, ep_stream_t stream, ep_event_t wait_event) {
     if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (c->num_shards > 1) return fail(c, EP_ERR_INVALID_ARG, "sharded context: use the ep_sharded_* calls");
     if (h == nullptr || (c->G > 0 && h->send_head == nullptr) || h->recv_rank_offset == nullptr)
         return fail(c, EP_ERR_HANDLE_MISMATCH, "handle send_head / recv_rank_offset missing");
     if (num_recv_rows < 0) return fail(c, EP_ERR_INVALID_ARG, "negative row count");
@@ -524,6 +554,7 @@ int ll_dispatch_impl(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint
                      uint8_t* packed_fp8, float* packed_scales, int32_t* packed_recv_count,
                      int32_t* src_info, int32_t* layout_range, ep_stream_t stream, ep_event_t wait_event) {
     if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (c->num_shards > 1) return fail(c, EP_ERR_INVALID_ARG, "sharded context: use the ep_sharded_* calls");
     const bool fp8 = packed_fp8 != nullptr || packed_scales != nullptr;
     if (packed_recv_count == nullptr || layout_range == nullptr || src_info == nullptr)
         return fail(c, EP_ERR_INVALID_ARG, "low-latency outputs missing");
@@ -593,6 +624,7 @@ int ep_ll_combine(ep_ctx* c, const uint16_t* y, const int64_t* topk_idx, const f
                   const int32_t* src_info, const int32_t* layout_range, uint16_t* out_x,
                   ep_stream_t stream, ep_event_t wait_event) {
     if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (c->num_shards > 1) return fail(c, EP_ERR_INVALID_ARG, "sharded context: use the ep_sharded_* calls");
     if (c->G > 0 && (y == nullptr || topk_idx == nullptr || topk_weights == nullptr || src_info == nullptr ||
                      layout_range == nullptr || out_x == nullptr))
         return fail(c, EP_ERR_INVALID_ARG, "low-latency combine argument missing");
@@ -676,6 +708,186 @@ int ep_ll_clean_mask(ep_ctx* c, ep_stream_t stream) {
     return cuda_check(c, cudaMemsetAsync(c->rank_mask, 0, sizeof(int) * c->R, reinterpret_cast<cudaStream_t>(stream)),
                       "clear rank mask");
 }
+
+// ------------------------------------------------------------ sharded exchange
+
+int ep_sharded_handle(ep_ctx* c, const uint8_t* is_token_in_rank, const int32_t* num_tokens_per_rank_all,
+                      const int32_t* num_tokens_per_expert_all, int32_t* send_head, int64_t* dst_offset,
+                      int64_t* num_recv_rows, int32_t* num_recv_tokens_per_expert, ep_stream_t stream,
+                      ep_event_t wait_event) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (num_tokens_per_rank_all == nullptr || num_tokens_per_expert_all == nullptr || dst_offset == nullptr)
+        return fail(c, EP_ERR_INVALID_ARG, "gathered counts / dst_offset missing");
+    if (c->G > 0 && (is_token_in_rank == nullptr || send_head == nullptr))
+        return fail(c, EP_ERR_INVALID_ARG, "is_token_in_rank / send_head missing");
+    if (!aligned(is_token_in_rank, 4) || !aligned(dst_offset, 8) || !aligned(num_recv_rows, 8))
+        return fail(c, EP_ERR_ALIGNMENT, "sharded handle arrays misaligned");
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
+    if (rc != EP_OK) return rc;
+    ep::ShardOffsetsParams op{num_tokens_per_rank_all, num_tokens_per_expert_all, c->shard_base,
+                              reinterpret_cast<long long*>(dst_offset), reinterpret_cast<long long*>(num_recv_rows),
+                              num_recv_tokens_per_expert, c->R, c->E, c->L, c->r0, c->Rl};
+    rc = launch(c, -1, true, s, [&] { return ep::launch_shard_offsets(op, s); });
+    if (rc != EP_OK || c->G == 0) return rc;
+    ep::ScanParams sp{};
+    sp.is_token_in_rank = is_token_in_rank;
+    sp.status = c->scan_status;
+    sp.ticket = c->scan_ticket;
+    sp.rank_start = c->rank_start;
+    sp.base = c->shard_base;
+    sp.send_head = send_head;
+    sp.err = c->err;
+    sp.G = c->G;
+    sp.R = c->R; sp.E = c->E; sp.L = c->L; sp.T = c->T; sp.C = c->C;
+    sp.q = (c->T + c->C - 1) / c->C;
+    sp.num_tiles = c->scan_tiles;
+    return launch(c, kScan, true, s, [&] { return ep::launch_scan(sp, s); });
+}
+
+namespace {
+
+int check_shard_table(ep_ctx* c, int num_shards, const void* const* table, bool required, const char* what,
+                      size_t align) {
+    if (table == nullptr) {
+        if (required) return fail(c, EP_ERR_INVALID_ARG, "%s pointer table missing", what);
+        return EP_OK;
+    }
+    for (int w = 0; w < num_shards; ++w) {
+        if (table[w] == nullptr) return fail(c, EP_ERR_INVALID_ARG, "%s of shard %d missing", what, w);
+        if (!aligned(table[w], align)) return fail(c, EP_ERR_ALIGNMENT, "%s of shard %d misaligned", what, w);
+    }
+    return EP_OK;
+}
+
+}  // namespace
+
+int ep_sharded_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, const float* topk_weights,
+                        const int32_t* send_head, const int64_t* dst_offset, int num_shards,
+                        uint16_t* const* recv_x, int64_t* const* recv_topk_idx,
+                        float* const* recv_topk_weights, int32_t* const* recv_src_idx,
+                        int64_t recv_capacity_rows, ep_stream_t stream, ep_event_t wait_event) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (num_shards != c->num_shards) return fail(c, EP_ERR_INVALID_ARG, "%d shard tables for %d shards",
+                                                 num_shards, c->num_shards);
+    if (recv_capacity_rows < 0) return fail(c, EP_ERR_INVALID_ARG, "negative capacity");
+    if (c->G > 0 && (x == nullptr || topk_idx == nullptr || send_head == nullptr || dst_offset == nullptr))
+        return fail(c, EP_ERR_INVALID_ARG, "x / topk_idx / send_head / dst_offset missing");
+    if (recv_topk_weights != nullptr && topk_weights == nullptr)
+        return fail(c, EP_ERR_INVALID_ARG, "recv_topk_weights needs topk_weights");
+    if (!aligned16(x) || !aligned(topk_idx, 8) || !aligned(topk_weights, 4) || !aligned(dst_offset, 8))
+        return fail(c, EP_ERR_ALIGNMENT, "inputs misaligned");
+    int rc = check_shard_table(c, num_shards, reinterpret_cast<const void* const*>(recv_x), true, "recv_x", 16);
+    if (rc == EP_OK)
+        rc = check_shard_table(c, num_shards, reinterpret_cast<const void* const*>(recv_topk_idx), false,
+                               "recv_topk_idx", 8);
+    if (rc == EP_OK)
+        rc = check_shard_table(c, num_shards, reinterpret_cast<const void* const*>(recv_topk_weights), false,
+                               "recv_topk_weights", 4);
+    if (rc == EP_OK)
+        rc = check_shard_table(c, num_shards, reinterpret_cast<const void* const*>(recv_src_idx), false,
+                               "recv_src_idx", 4);
+    if (rc != EP_OK) return rc;
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
+    if (rc != EP_OK) return rc;
+    ep::DispatchParams dp{};
+    dp.x = x;
+    dp.send_head = send_head;
+    dp.recv_capacity = recv_capacity_rows;
+    dp.topk_idx = topk_idx;
+    dp.topk_weights = topk_weights;
+    dp.dst_offset = reinterpret_cast<const long long*>(dst_offset);
+    dp.ranks_per_shard = c->Rl;
+    for (int w = 0; w < num_shards; ++w) {
+        dp.shard_rows[w] = recv_x[w];
+        dp.shard_idx[w] = recv_topk_idx ? recv_topk_idx[w] : nullptr;
+        dp.shard_w[w] = recv_topk_weights ? recv_topk_weights[w] : nullptr;
+        dp.shard_src[w] = recv_src_idx ? recv_src_idx[w] : nullptr;
+    }
+    dp.err = c->err;
+    dp.G = c->G;
+    dp.R = c->R; dp.E = c->E; dp.L = c->L; dp.T = c->T; dp.K = c->K; dp.H = c->H;
+    dp.splits = ep::dispatch_splits(c->H);
+    return launch(c, kDispatch, c->G > 0, s, [&] { return ep::launch_dispatch(ep::kModeSharded, dp, s); });
+}
+
+int ep_sharded_combine(ep_ctx* c, int num_shards, const uint16_t* const* y, const float* const* recv_topk_weights,
+                       int64_t y_capacity_rows, const int32_t* send_head, const int64_t* dst_offset,
+                       const uint16_t* bias0, const uint16_t* bias1, uint16_t* out_x, float* out_topk_weights,
+                       ep_stream_t stream, ep_event_t wait_event) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (num_shards != c->num_shards) return fail(c, EP_ERR_INVALID_ARG, "%d shard tables for %d shards",
+                                                 num_shards, c->num_shards);
+    if (y_capacity_rows < 0) return fail(c, EP_ERR_INVALID_ARG, "negative capacity");
+    if (c->G > 0 && (send_head == nullptr || dst_offset == nullptr || out_x == nullptr))
+        return fail(c, EP_ERR_INVALID_ARG, "send_head / dst_offset / out_x missing");
+    if (out_topk_weights != nullptr && recv_topk_weights == nullptr)
+        return fail(c, EP_ERR_INVALID_ARG, "out_topk_weights needs the shards' recv_topk_weights");
+    if (!aligned16(out_x) || !aligned16(bias0) || !aligned16(bias1) || !aligned(out_topk_weights, 4) ||
+        !aligned(dst_offset, 8))
+        return fail(c, EP_ERR_ALIGNMENT, "arrays misaligned");
+    int rc = check_shard_table(c, num_shards, reinterpret_cast<const void* const*>(y), true, "y", 16);
+    if (rc == EP_OK)
+        rc = check_shard_table(c, num_shards, reinterpret_cast<const void* const*>(recv_topk_weights), false,
+                               "recv_topk_weights", 4);
+    if (rc != EP_OK) return rc;
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
+    if (rc != EP_OK) return rc;
+    ep::CombineParams p{};
+    p.y_rows = y_capacity_rows;
+    p.send_head = send_head;
+    p.bias0 = bias0;
+    p.bias1 = bias1;
+    p.out_x = out_x;
+    p.out_topk_weights = out_topk_weights;
+    p.sharded = true;
+    p.dst_offset = reinterpret_cast<const long long*>(dst_offset);
+    p.ranks_per_shard = c->Rl;
+    for (int w = 0; w < num_shards; ++w) {
+        p.shard_y[w] = y[w];
+        p.shard_w[w] = recv_topk_weights ? recv_topk_weights[w] : nullptr;
+    }
+    p.err = c->err;
+    p.G = c->G;
+    p.R = c->R; p.K = c->K; p.H = c->H;
+    p.splits = ep::combine_splits(c->H);
+    return launch(c, kCombine, c->G > 0, s, [&] { return ep::launch_combine(p, c->num_sms, s); });
+}
+
+// Device memory that another process can map (CUDA IPC): one cudaMalloc per
+// buffer, so the handle covers exactly the buffer.
+int ep_shared_alloc(size_t bytes, void** ptr, uint8_t* ipc_handle) {
+    if (ptr == nullptr || ipc_handle == nullptr || bytes == 0) return EP_ERR_INVALID_ARG;
+    *ptr = nullptr;
+    void* p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) return EP_ERR_CUDA;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, p) != cudaSuccess) {
+        cudaFree(p);
+        return EP_ERR_CUDA;
+    }
+    static_assert(sizeof(h) == EP_IPC_HANDLE_BYTES, "IPC handle size");
+    std::memcpy(ipc_handle, &h, sizeof h);
+    *ptr = p;
+    return EP_OK;
+}
+
+int ep_shared_free(void* ptr) { return cudaFree(ptr) == cudaSuccess ? EP_OK : EP_ERR_CUDA; }
+
+int ep_ipc_open(const uint8_t* ipc_handle, void** ptr) {
+    if (ipc_handle == nullptr || ptr == nullptr) return EP_ERR_INVALID_ARG;
+    *ptr = nullptr;
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, ipc_handle, sizeof h);
+    return cudaIpcOpenMemHandle(ptr, h, cudaIpcMemLazyEnablePeerAccess) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+int ep_ipc_close(void* ptr) { return cudaIpcCloseMemHandle(ptr) == cudaSuccess ? EP_OK : EP_ERR_CUDA; }
 
 int ep_profile_enable(ep_ctx* c, int enable) {
     if (c == nullptr) return EP_ERR_INVALID_ARG;

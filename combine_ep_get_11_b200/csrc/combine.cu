@@ -18,7 +18,9 @@
 // every U-vector slab it issues the loads of a group of 4 rows at once
 // (4 x 4 vectors; measured best on B200 for fan-ins of 3.6 and 5.2), then adds
 // them in rank order, group after group.  Traffic per token: fan-out *
-// H*2 bytes read (streaming), H*2 written.
+// H*2 bytes read (streaming), H*2 written.  The sharded form reads rank d's
+// rows from the GPU hosting d (its own memory or a peer's, mapped into this
+// process): the return exchange happens inside the reduction.
 
 #include "common.cuh"
 #include "kernels.h"
@@ -42,10 +44,11 @@ __device__ __forceinline__ void add_bf16x8(float* acc, const uint4& v) {
     acc[7] = __fadd_rn(acc[7], bf16_hi(v.w));
 }
 
-template <int U, int kGroup = kRowsPerGroup>
+template <int U, bool kSharded, int kGroup = kRowsPerGroup>
 __global__ void __launch_bounds__(kCombineThreads, 2)
 combine_kernel(const CombineParams p) {
-    __shared__ long long s_rows[kCombineWarps][32];
+    __shared__ long long s_rows[kCombineWarps][32];             // row index, or (sharded) row address
+    __shared__ long long s_wrow[kSharded ? kCombineWarps : 1][32];   // sharded: weight-row address
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const long long wid = (long long)blockIdx.x * kCombineWarps + warp;
     const long long g = wid / p.splits;          // token
@@ -57,7 +60,7 @@ combine_kernel(const CombineParams p) {
     if (lane < R) {
         const int h = p.send_head[g * R + lane];
         if (h >= 0) {
-            row = p.recv_rank_offset[lane] + h;
+            row = (kSharded ? p.dst_offset[lane] : p.recv_rank_offset[lane]) + h;
             if (row >= p.y_rows) {
                 record_error(p.err, EP_ERR_CAPACITY);
                 row = -1;
@@ -66,7 +69,17 @@ combine_kernel(const CombineParams p) {
     }
     const uint32_t m = __ballot_sync(kFullMask, row >= 0);
     const int f = __popc(m);
-    if (row >= 0) s_rows[warp][__popc(m & lanemask_lt())] = row;
+    if (row >= 0) {
+        const int at = __popc(m & lanemask_lt());
+        if constexpr (kSharded) {   // rank d's rows are in shard d / ranks_per_shard (own or peer memory)
+            const int shard = lane / p.ranks_per_shard;
+            s_rows[warp][at] = (long long)reinterpret_cast<uintptr_t>(p.shard_y[shard] + row * p.H);
+            s_wrow[warp][at] =
+                p.shard_w[shard] ? (long long)reinterpret_cast<uintptr_t>(p.shard_w[shard] + row * p.K) : 0;
+        } else {
+            s_rows[warp][at] = row;
+        }
+    }
     __syncwarp();
 
     const uint4* b0 = p.bias0 ? reinterpret_cast<const uint4*>(p.bias0 + g * p.H) : nullptr;
@@ -89,7 +102,9 @@ combine_kernel(const CombineParams p) {
 #pragma unroll
             for (int i = 0; i < kGroup; ++i) {
                 if (i0 + i < f) {
-                    const uint4* src = reinterpret_cast<const uint4*>(p.y + s_rows[warp][i0 + i] * p.H);
+                    const uint4* src =
+                        kSharded ? reinterpret_cast<const uint4*>(static_cast<uintptr_t>(s_rows[warp][i0 + i]))
+                                 : reinterpret_cast<const uint4*>(p.y + s_rows[warp][i0 + i] * p.H);
 #pragma unroll
                     for (int u = 0; u < U; ++u) {
                         const int c = c0 + lane + 32 * u;
@@ -121,7 +136,15 @@ combine_kernel(const CombineParams p) {
         }
     }
 
-    if (part == 0 && p.recv_topk_weights != nullptr && p.out_topk_weights != nullptr && lane < p.K) {
+    if constexpr (kSharded) {
+        // weight rows are given for every shard whenever out_topk_weights is asked for
+        if (part == 0 && p.out_topk_weights != nullptr && lane < p.K) {
+            float w = 0.f;
+            for (int i = 0; i < f; ++i)
+                w = __fadd_rn(w, reinterpret_cast<const float*>(static_cast<uintptr_t>(s_wrow[warp][i]))[lane]);
+            p.out_topk_weights[g * p.K + lane] = w;
+        }
+    } else if (part == 0 && p.recv_topk_weights != nullptr && p.out_topk_weights != nullptr && lane < p.K) {
         float w = 0.f;
         for (int i = 0; i < f; ++i) w = __fadd_rn(w, p.recv_topk_weights[s_rows[warp][i] * p.K + lane]);
         p.out_topk_weights[g * p.K + lane] = w;
@@ -136,7 +159,10 @@ cudaError_t launch_combine(const CombineParams& p, int num_sms, cudaStream_t str
     // one warp per token (or column slice): the block scheduler balances the work
     (void)num_sms;
     const long long blocks = (p.G * p.splits + kCombineWarps - 1) / kCombineWarps;
-    combine_kernel<U><<<(unsigned)blocks, kCombineThreads, 0, stream>>>(p);
+    if (p.sharded)
+        combine_kernel<U, true><<<(unsigned)blocks, kCombineThreads, 0, stream>>>(p);
+    else
+        combine_kernel<U, false><<<(unsigned)blocks, kCombineThreads, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

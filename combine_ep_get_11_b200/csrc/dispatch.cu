@@ -25,7 +25,11 @@
 //   * lane d (destination rank), or lane k (top-k slot) in the packed form,
 //     resolves its destination row; a ballot compacts the rows in lane order;
 //   * in the normal form the destination lanes also write the receive
-//     metadata: local top-k ids, weights, and recv_src_idx.
+//     metadata: local top-k ids, weights, and recv_src_idx;
+//   * the sharded form is the normal form for virtual ranks spread over
+//     several GPUs: destination d's rows and metadata go straight into the
+//     receive buffers of the GPU hosting d (its own memory, or a peer's mapped
+//     into this process), so the exchange happens inside the copy.
 // Per token the HBM traffic is H*2 bytes read + fan-out * H*2 bytes written
 // (fan-out * (H + H/32) bytes in the FP8 packed form).
 
@@ -76,35 +80,45 @@ dispatch_kernel(const DispatchParams p) {
     } else if (lane < p.R) {
         const int h = p.send_head[g * p.R + lane];
         if (h >= 0) {
-            row = p.recv_rank_offset[lane] + h;
+            row = (kMode == kModeSharded ? p.dst_offset[lane] : p.recv_rank_offset[lane]) + h;
             if (row >= p.recv_capacity) {
                 record_error(p.err, EP_ERR_CAPACITY);
                 row = -1;
             }
         }
     }
+    // sharded: lane d's destination buffers are those of shard d / ranks_per_shard
+    const int shard = (kMode == kModeSharded && row >= 0) ? lane / p.ranks_per_shard : 0;
 
-    if (kMode == kModeNormal && part == 0) {
+    if ((kMode == kModeNormal || kMode == kModeSharded) && part == 0) {
+        int* r_src = p.recv_src_idx;
+        int64_t* r_idx = p.recv_topk_idx;
+        float* r_w = p.recv_topk_weights;
+        if (kMode == kModeSharded) {
+            r_src = p.shard_src[shard];
+            r_idx = p.shard_idx[shard];
+            r_w = p.shard_w[shard];
+        }
         long long e = -1;
         float w = 0.f;
         if (lane < p.K) {
             e = p.topk_idx[g * p.K + lane];
             if (p.topk_weights != nullptr) w = p.topk_weights[g * p.K + lane];
         }
-        if (row >= 0 && p.recv_src_idx != nullptr) p.recv_src_idx[row] = (int)(g % p.T);
+        if (row >= 0 && r_src != nullptr) r_src[row] = (int)(g % p.T);
         for (int k = 0; k < p.K; ++k) {
             const long long ek = __shfl_sync(kFullMask, e, k);
             const float wk = __shfl_sync(kFullMask, w, k);
             if (row >= 0) {
                 const bool here = ek >= 0 && ek < p.E && (int)ek / p.L == lane;
-                if (p.recv_topk_idx != nullptr)
-                    p.recv_topk_idx[row * p.K + k] = here ? (long long)((int)ek % p.L) : -1LL;
-                if (p.recv_topk_weights != nullptr)
-                    p.recv_topk_weights[row * p.K + k] = here ? wk : 0.f;
+                if (r_idx != nullptr) r_idx[row * p.K + k] = here ? (long long)((int)ek % p.L) : -1LL;
+                if (r_w != nullptr) r_w[row * p.K + k] = here ? wk : 0.f;
             }
         }
     }
     if (kMode == kModeNormal && p.recv_x == nullptr) return;   // metadata only
+    if (kMode == kModeSharded && row >= 0)                     // keep the row's address
+        row = (long long)reinterpret_cast<uintptr_t>(p.shard_rows[shard] + row * p.H);
 
     const uint32_t m = __ballot_sync(kFullMask, row >= 0);
     const int f = __popc(m);
@@ -181,7 +195,9 @@ dispatch_kernel(const DispatchParams p) {
                 if (c < hi) v[u] = ld_nc_v4(src + c);
             }
             for (int i = 0; i < f; ++i) {
-                uint4* dst = reinterpret_cast<uint4*>(p.recv_x + s_rows[warp][i] * p.H);
+                uint4* dst = kMode == kModeSharded
+                                 ? reinterpret_cast<uint4*>(static_cast<uintptr_t>(s_rows[warp][i]))
+                                 : reinterpret_cast<uint4*>(p.recv_x + s_rows[warp][i] * p.H);
 #pragma unroll
                 for (int u = 0; u < kVec; ++u) {
                     const int c = c0 + lane + 32 * u;
@@ -210,6 +226,7 @@ cudaError_t launch_dispatch(int mode, const DispatchParams& p, cudaStream_t stre
         case kModeCached: return launch_mode<kModeCached>(p, stream);
         case kModeLowLatency: return launch_mode<kModeLowLatency>(p, stream);
         case kModeLowLatencyFp8: return launch_mode<kModeLowLatencyFp8>(p, stream);
+        case kModeSharded: return launch_mode<kModeSharded>(p, stream);
         default: return cudaErrorInvalidValue;
     }
 }

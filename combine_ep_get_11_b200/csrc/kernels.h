@@ -17,12 +17,13 @@ inline int combine_splits(int) { return 1; }
 
 // ------------------------------------------------------------------ layout
 struct LayoutParams {
-    const int64_t* topk_idx;   // [G][K]
-    uint8_t* is_token_in_rank; // [G][R]
-    int* num_tokens_per_rank;  // [R][R], zeroed before launch
-    int* num_tokens_per_expert;// [R][E], zeroed before launch
+    const int64_t* topk_idx;   // [S][T][K]   (S source ranks in this launch)
+    uint8_t* is_token_in_rank; // [S][T][R]
+    int* num_tokens_per_rank;  // [S][R], zeroed before launch
+    int* num_tokens_per_expert;// [S][E], zeroed before launch
     int* err;
     int R, E, L, T, K;
+    int num_src;               // S: R, or the ranks of one shard
 };
 constexpr int kLayoutThreads = 256;
 cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream);
@@ -38,6 +39,7 @@ struct ScanParams {
     unsigned long long* status;        // [num_tiles][R] call-tagged words (zero words never match)
     unsigned long long* ticket;        // block ticket: only incremented (or zeroed with status)
     unsigned long long* rank_start;    // [R][R] call-tagged P(s*T)[d] (zeroed with the ticket if at all)
+    const int* base;                   // [R] or null: added to every P value (tokens of earlier shards)
     int* send_head;                    // [G][R]
     int* rank_prefix_matrix;           // [R][R]
     int* channel_prefix_matrix;        // [R][R][C]
@@ -48,11 +50,15 @@ struct ScanParams {
     long long G;
     int R, E, L, T, C, q, num_tiles;
 };
+// The handle matrices, recv_rank_offset and num_recv_tokens_per_expert may be
+// null (a sharded exchange takes its offsets from launch_shard_offsets).
 constexpr int kScanTile = 256;   // tokens per tile == threads per block
 cudaError_t launch_scan(const ScanParams& p, cudaStream_t stream);
 
 // ---------------------------------------------------- dispatch (row copies)
-enum DispatchMode { kModeNormal = 0, kModeCached = 1, kModeLowLatency = 2, kModeLowLatencyFp8 = 3 };
+enum DispatchMode { kModeNormal = 0, kModeCached = 1, kModeLowLatency = 2, kModeLowLatencyFp8 = 3,
+                    kModeSharded = 4 };
+constexpr int kMaxShards = 32;   // GPUs of a sharded exchange (each hosts >= 1 virtual rank)
 constexpr int kFp8Block = 128;   // hidden channels per FP8 scale
 
 struct DispatchParams {
@@ -75,6 +81,14 @@ struct DispatchParams {
     // low latency, FP8 form (recv_x unused)
     uint8_t* recv_fp8;                 // [E][ll_cap][H] E4M3 codes
     float* recv_scales;                // [E][ll_cap][H/128]
+    // sharded: destination d's rows live in shard d / ranks_per_shard's buffers,
+    // starting at row dst_offset[d] (pointers valid on this GPU: own or peer memory)
+    const long long* dst_offset;       // [R]
+    int ranks_per_shard;
+    uint16_t* shard_rows[kMaxShards];  // [cap][H] per shard
+    int64_t* shard_idx[kMaxShards];    // [cap][K] per shard, or null
+    float* shard_w[kMaxShards];        // [cap][K] per shard, or null
+    int* shard_src[kMaxShards];        // [cap] per shard, or null
     int* err;
     long long G;
     int R, E, L, T, K, H;
@@ -93,12 +107,35 @@ struct CombineParams {
     const uint16_t* bias1;             // [G][H] or null
     uint16_t* out_x;                   // [G][H]
     float* out_topk_weights;           // [G][K] or null
+    // sharded: the rows of destination d are read from shard d / ranks_per_shard
+    // (own or peer memory), from row dst_offset[d]; recv_rank_offset / y unused
+    bool sharded;
+    const long long* dst_offset;       // [R]
+    int ranks_per_shard;
+    const uint16_t* shard_y[kMaxShards];   // [y_rows][H] per shard
+    const float* shard_w[kMaxShards];      // [y_rows][K] per shard, or null
     int* err;
     long long G;
     int R, K, H;
     int splits;                        // warps per token (column slices of the row)
 };
 cudaError_t launch_combine(const CombineParams& p, int num_sms, cudaStream_t stream);
+
+// ---------------------------------------------------------- sharded offsets
+// From the gathered layout counts of all R ranks, for the shard hosting ranks
+// [r0, r0 + ranks_per_shard): the tokens of earlier shards per destination (the
+// scan's base), each destination's first row in its shard's receive buffer,
+// this shard's receive rows and its local experts' receive counts.
+struct ShardOffsetsParams {
+    const int* num_tokens_per_rank_all;    // [R][R]
+    const int* num_tokens_per_expert_all;  // [R][E]
+    int* base;                             // [R]
+    long long* dst_offset;                 // [R]
+    long long* num_recv_rows;              // [1] or null
+    int* num_recv_tokens_per_expert;       // [ranks_per_shard][L] or null
+    int R, E, L, r0, ranks_per_shard;
+};
+cudaError_t launch_shard_offsets(const ShardOffsetsParams& p, cudaStream_t stream);
 
 // ------------------------------------------------------------ low latency
 // Low-latency slot assignment: a decoupled-lookback scan over 256-token tiles

@@ -9,7 +9,8 @@
 // token is a 32-bit mask (R <= 32);
 // per-rank counts come from warp ballots + popc, per-expert counts from shared
 // memory atomics, and each block adds its counts to the global histograms.
-// The grid is (token blocks, source rank), so a block never straddles ranks.
+// The grid is (token blocks, source rank), so a block never straddles ranks; the
+// sources are all R ranks, or those of one shard of a sharded exchange.
 // Traffic: K*8 bytes read and R bytes written per token; latency-bound.
 
 #include "common.cuh"
@@ -79,7 +80,8 @@ layout_kernel(const LayoutParams p) {
 
 cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream) {
     if (p.T == 0) return cudaSuccess;
-    dim3 grid((p.T + kLayoutThreads - 1) / kLayoutThreads, p.R);
+    if (p.num_src == 0) return cudaSuccess;
+    dim3 grid((p.T + kLayoutThreads - 1) / kLayoutThreads, p.num_src);
     const size_t smem = (32 + (size_t)p.E) * sizeof(int);
     if (p.K <= 8)
         layout_kernel<8><<<grid, kLayoutThreads, smem, stream>>>(p);

@@ -155,7 +155,7 @@ scan_kernel(const ScanParams p) {
             }
             st_relaxed_u64(mine, tag | kFlagInclusive | (unsigned)(excl + agg));
         }
-        s_excl[lane] = excl;
+        s_excl[lane] = excl + (p.base != nullptr ? p.base[lane] : 0);
     }
     __syncthreads();
 
@@ -176,54 +176,56 @@ scan_kernel(const ScanParams p) {
     // (gb == G belongs to the last tile); P(gb)[d] = s_excl[d] + members before gb
     const bool last_tile = tile == p.num_tiles - 1;
     const int T = p.T, C = p.C;
-    const int s_lo = max(0, gt / T - 1);
-    const int s_hi = min(R - 1, (gt + kScanTile) / T);
-    const int per_src = (C + 1) * R;
-    const int nb = (s_hi - s_lo + 1) * per_src;
-    for (int i = tid; i < nb; i += kScanTile) {
-        const int s = s_lo + i / per_src;
-        const int rem = i - (i / per_src) * per_src;
-        const int c = rem / R, d = rem - (rem / R) * R;
-        const int gb = s * T + min(c * p.q, T);
-        const bool here = (gb >= gt && gb < gt + kScanTile && gb < G) || (gb == G && last_tile);
-        if (!here) continue;
-        const int rel = gb - gt;   // 0..256
-        const int w = rel >> 5, b = rel & 31;
-        const int pv = s_excl[d] + ((w < kWordsPerTile) ? s_wpref[d][w] + __popc(s_bits[d][w] & ((1u << b) - 1u))
-                                                         : s_wpref[d][kWordsPerTile]);
-        if (c == 0 && s > 0) st_relaxed_u64(p.rank_start + (size_t)s * R + d, tag | kFlagInclusive | (unsigned)pv);
-        if (c < C) p.recv_channel_prefix_matrix[((long long)d * R + s) * C + c] = pv;
-        if (c == C) p.rank_prefix_matrix[s * R + d] = pv;
-        if (c > 0) {
-            // the rank's start P(s*T)[d]: in this tile, or published by an earlier one
-            int start = 0;
-            const int gs = s * T;
-            if (s == 0) {
-                start = 0;
-            } else if (gs >= gt) {
-                const int rs = gs - gt, ws = rs >> 5, bs = rs & 31;
-                start = s_excl[d] + s_wpref[d][ws] + __popc(s_bits[d][ws] & ((1u << bs) - 1u));
-            } else {
-                unsigned long long v = ld_relaxed_u64(p.rank_start + (size_t)s * R + d);
-                uint64_t t0 = 0;
-                uint32_t spins = 0;
-                while (!published(v, tag)) {
-                    if (spins == 0) t0 = globaltimer_ns();
-                    ++spins;
-                    if (spins > kWaitLimitIters ||
-                        ((spins & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs)) {
-                        record_error(p.err, EP_ERR_TIMEOUT);
-                        break;
+    if (p.recv_channel_prefix_matrix != nullptr) {
+        const int s_lo = max(0, gt / T - 1);
+        const int s_hi = min(R - 1, (gt + kScanTile) / T);
+        const int per_src = (C + 1) * R;
+        const int nb = (s_hi - s_lo + 1) * per_src;
+        for (int i = tid; i < nb; i += kScanTile) {
+            const int s = s_lo + i / per_src;
+            const int rem = i - (i / per_src) * per_src;
+            const int c = rem / R, d = rem - (rem / R) * R;
+            const int gb = s * T + min(c * p.q, T);
+            const bool here = (gb >= gt && gb < gt + kScanTile && gb < G) || (gb == G && last_tile);
+            if (!here) continue;
+            const int rel = gb - gt;   // 0..256
+            const int w = rel >> 5, b = rel & 31;
+            const int pv = s_excl[d] + ((w < kWordsPerTile) ? s_wpref[d][w] + __popc(s_bits[d][w] & ((1u << b) - 1u))
+                                                             : s_wpref[d][kWordsPerTile]);
+            if (c == 0 && s > 0) st_relaxed_u64(p.rank_start + (size_t)s * R + d, tag | kFlagInclusive | (unsigned)pv);
+            if (c < C) p.recv_channel_prefix_matrix[((long long)d * R + s) * C + c] = pv;
+            if (c == C) p.rank_prefix_matrix[s * R + d] = pv;
+            if (c > 0) {
+                // the rank's start P(s*T)[d]: in this tile, or published by an earlier one
+                int start = 0;
+                const int gs = s * T;
+                if (s == 0) {
+                    start = 0;
+                } else if (gs >= gt) {
+                    const int rs = gs - gt, ws = rs >> 5, bs = rs & 31;
+                    start = s_excl[d] + s_wpref[d][ws] + __popc(s_bits[d][ws] & ((1u << bs) - 1u));
+                } else {
+                    unsigned long long v = ld_relaxed_u64(p.rank_start + (size_t)s * R + d);
+                    uint64_t t0 = 0;
+                    uint32_t spins = 0;
+                    while (!published(v, tag)) {
+                        if (spins == 0) t0 = globaltimer_ns();
+                        ++spins;
+                        if (spins > kWaitLimitIters ||
+                            ((spins & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs)) {
+                            record_error(p.err, EP_ERR_TIMEOUT);
+                            break;
+                        }
+                        v = ld_relaxed_u64(p.rank_start + (size_t)s * R + d);
                     }
-                    v = ld_relaxed_u64(p.rank_start + (size_t)s * R + d);
+                    start = (int)(uint32_t)v;
                 }
-                start = (int)(uint32_t)v;
+                p.channel_prefix_matrix[((long long)s * R + d) * C + (c - 1)] = pv - start;
             }
-            p.channel_prefix_matrix[((long long)s * R + d) * C + (c - 1)] = pv - start;
         }
     }
 
-    if (!last_tile) return;
+    if (!last_tile || p.recv_rank_offset == nullptr) return;
     // P(G)[d] = N_d: receive offsets; per-expert receive counts from the layout
     __shared__ long long s_total[32];
     if (tid < R) s_total[tid] = s_excl[tid] + s_wpref[tid][kWordsPerTile];

@@ -347,6 +347,91 @@ EP_API int ep_ll_update_mask(ep_ctx* ctx, int32_t rank, int32_t masked, ep_strea
 EP_API int ep_ll_query_mask(ep_ctx* ctx, int32_t* host_out, ep_stream_t stream);
 EP_API int ep_ll_clean_mask(ep_ctx* ctx, ep_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Sharded exchange: the R virtual ranks spread over W GPUs of one node, GPU w
+ * hosting ranks [w*R/W, (w+1)*R/W) -- the pages' ranks are GPUs joined by
+ * NVLink, with buffers allocated per rank and their IPC handles exchanged
+ * ([API] "Construction and Resource Allocation"; [ARCH] intranode mode).
+ * Each GPU keeps registered receive buffers (one cudaMalloc each, see
+ * ep_shared_alloc) that every other GPU maps with ep_ipc_open.  Dispatch writes
+ * every row straight into the receive buffer of the GPU hosting its
+ * destination, and combine reads the expert outputs back from there: the
+ * all-to-all happens inside the copy and the reduction, over NVLink.  The
+ * receive order is the one-GPU order, so send_head and the rows of rank d
+ * equal those ep_dispatch gives for the whole problem.
+ *
+ * Per step, on every GPU (shard w, Rl = R/W local ranks, local tokens G = Rl*T):
+ *   1. ep_get_dispatch_layout on the shard's topk_idx [Rl][T][K] gives
+ *      is_token_in_rank [Rl][T][R], num_tokens_per_rank [Rl][R],
+ *      num_tokens_per_expert [Rl][E];
+ *   2. the caller gathers the W layouts' counts in shard order into
+ *      num_tokens_per_rank_all [R][R] and num_tokens_per_expert_all [R][E]
+ *      (an all-gather of a few KB);
+ *   3. ep_sharded_handle -> send_head [Rl][T][R] (P(g)[d] over all R*T tokens),
+ *      dst_offset [R] (first row of rank d in its GPU's receive buffer),
+ *      num_recv_rows (rows this GPU receives), num_recv_tokens_per_expert
+ *      [Rl][L] for this GPU's experts;
+ *   4. ep_sharded_dispatch writes the rows (and metadata) into the GPUs' buffers;
+ *   5. a barrier across the GPUs (every dispatch finished) before the experts
+ *      read their rows, and again (every expert output written) before
+ *   6. ep_sharded_combine, which reduces, for each local token, the rows of its
+ *      destination ranks in ascending rank order (fp32, one rounding), reading
+ *      them from the GPUs hosting them.
+ * Pointer tables (`num_shards` entries, indexed by shard) hold device pointers
+ * valid in the calling process: its own buffer at its own index, the mapped
+ * peers' elsewhere.  Every buffer of a table has at least `capacity` rows.
+ * The kernels never wait on another GPU; the barriers are the caller's.
+ * Rows from or to a row index >= capacity record EP_ERR_CAPACITY. */
+
+/* Context for shard `shard` of `num_shards` (1 <= W <= 32, R % W == 0) on the
+ * current device.  cfg describes the whole problem (R, E, T per rank, ...).
+ * ep_get_dispatch_layout works on the shard's ranks; ep_dispatch,
+ * ep_dispatch_cached, ep_combine and the low-latency calls are refused
+ * (EP_ERR_INVALID_ARG) on a context of W > 1. */
+EP_API int ep_create_sharded(const ep_config* cfg, int num_shards, int shard, ep_ctx** out);
+
+/* Step 3 above.  num_tokens_per_rank_all i32 [R][R], num_tokens_per_expert_all
+ * i32 [R][E] (inputs, gathered); send_head i32 [Rl][T][R], dst_offset i64 [R],
+ * num_recv_rows i64 [1] (nullable), num_recv_tokens_per_expert i32 [Rl][L]
+ * (nullable): outputs on this device. */
+EP_API int ep_sharded_handle(ep_ctx* ctx, const uint8_t* is_token_in_rank, const int32_t* num_tokens_per_rank_all,
+                             const int32_t* num_tokens_per_expert_all, int32_t* send_head, int64_t* dst_offset,
+                             int64_t* num_recv_rows, int32_t* num_recv_tokens_per_expert,
+                             ep_stream_t stream, ep_event_t wait_event);
+
+/* Step 4.  x bf16 [Rl][T][H], topk_idx i64 [Rl][T][K], topk_weights f32
+ * [Rl][T][K] (nullable unless recv_topk_weights is given).  Tables of
+ * num_shards pointers: recv_x bf16 [capacity][H] (required), recv_topk_idx
+ * i64 [capacity][K], recv_topk_weights f32 [capacity][K], recv_src_idx i32
+ * [capacity] (each table nullable; written as by ep_dispatch, in the receive
+ * buffer of the GPU hosting the destination). */
+EP_API int ep_sharded_dispatch(ep_ctx* ctx, const uint16_t* x, const int64_t* topk_idx, const float* topk_weights,
+                               const int32_t* send_head, const int64_t* dst_offset, int num_shards,
+                               uint16_t* const* recv_x, int64_t* const* recv_topk_idx,
+                               float* const* recv_topk_weights, int32_t* const* recv_src_idx,
+                               int64_t capacity, ep_stream_t stream, ep_event_t wait_event);
+
+/* Step 6.  Tables of num_shards pointers: y bf16 [capacity][H] (the expert
+ * outputs, row for row as received; required), recv_topk_weights f32
+ * [capacity][K] (required iff out_topk_weights is given).  bias0 / bias1 bf16
+ * [Rl][T][H] nullable; out_x bf16 [Rl][T][H]; out_topk_weights f32 [Rl][T][K]
+ * nullable.  Same arithmetic as ep_combine. */
+EP_API int ep_sharded_combine(ep_ctx* ctx, int num_shards, const uint16_t* const* y,
+                              const float* const* recv_topk_weights, int64_t capacity, const int32_t* send_head,
+                              const int64_t* dst_offset, const uint16_t* bias0, const uint16_t* bias1,
+                              uint16_t* out_x, float* out_topk_weights, ep_stream_t stream, ep_event_t wait_event);
+
+/* Registered buffers: ep_shared_alloc makes one device allocation of `bytes`
+ * on the current device and writes its CUDA IPC handle (EP_IPC_HANDLE_BYTES
+ * bytes) to ipc_handle; release it with ep_shared_free.  Another process maps
+ * it with ep_ipc_open (peer access enabled on demand) and unmaps it with
+ * ep_ipc_close.  A process cannot open its own handles. */
+#define EP_IPC_HANDLE_BYTES 64
+EP_API int ep_shared_alloc(size_t bytes, void** ptr, uint8_t* ipc_handle);
+EP_API int ep_shared_free(void* ptr);
+EP_API int ep_ipc_open(const uint8_t* ipc_handle, void** ptr);
+EP_API int ep_ipc_close(void* ptr);
+
 /* Optional per-kernel timing (CUDA events around each launch on the call's
  * stream; inside a stream capture they become event-record nodes, recorded
  * each time the graph runs).  ep_profile_read synchronizes the recorded events and returns,

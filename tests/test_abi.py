@@ -72,3 +72,21 @@ def test_null_arguments(lib):
 
 def test_no_kernels_launched_on_cpu(lib):
     assert lib.ep_kernel_launch_count() == 0
+
+
+@pytest.mark.parametrize("shards,shard", [(3, 0), (0, 0), (2, 2), (2, -1), (33, 0)])
+def test_bad_shard_split_is_rejected_on_the_host(lib, shards, shard):
+    import combine_ep_get_11_b200 as ep
+    c = ep.ep_config(8, 64, 16, 256, 2, 10, 0)
+    out = ctypes.c_void_p()
+    assert lib.ep_create_sharded(ctypes.byref(c), shards, shard, ctypes.byref(out)) == 1
+    assert out.value is None
+
+
+def test_sharded_null_arguments(lib):
+    assert lib.ep_sharded_handle(None, *([None] * 9)) == 1
+    assert lib.ep_sharded_dispatch(None, None, None, None, None, None, 1, None, None, None, None, 0,
+                                   None, None) == 1
+    assert lib.ep_sharded_combine(None, 1, None, None, 0, None, None, None, None, None, None, None, None) == 1
+    assert lib.ep_shared_alloc(0, None, None) == 1
+    assert lib.ep_ipc_open(None, None) == 1
