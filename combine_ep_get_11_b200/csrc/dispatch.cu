@@ -206,6 +206,10 @@ dispatch_kernel(const DispatchParams p) {
             }
         }
     }
+    // sharded: rows and metadata may sit in other GPUs' memory; make them
+    // visible system-wide before the kernel ends (a peer reads them after the
+    // caller's cross-GPU barrier)
+    if (kMode == kModeSharded) __threadfence_system();
 }
 
 template <int kMode>
