@@ -480,7 +480,8 @@ int ep_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, const flo
     dp.G = c->G;
     dp.R = c->R; dp.E = c->E; dp.L = c->L; dp.T = c->T; dp.K = c->K; dp.H = c->H;
     dp.splits = ep::dispatch_splits(c->H);
-    return launch(c, kDispatch, true, s, [&] { return ep::launch_dispatch(ep::kModeNormal, dp, s); });
+    return launch(c, kDispatch, true, s,
+                  [&] { return ep::launch_dispatch(ep::kModeNormal, dp, s, num_recv_host == nullptr); });
 }
 
 int ep_dispatch_cached(ep_ctx* c, const uint16_t* x, const ep_handle* h, uint16_t* recv_x,
@@ -595,7 +596,7 @@ int ll_dispatch_impl(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint
     dp.R = c->R; dp.E = c->E; dp.L = c->L; dp.T = c->T; dp.K = c->K; dp.H = c->H;
     dp.splits = ep::dispatch_splits(c->H);
     const int mode = fp8 ? ep::kModeLowLatencyFp8 : ep::kModeLowLatency;
-    return launch(c, fp8 ? kLLCopyFp8 : kLLCopy, true, s, [&] { return ep::launch_dispatch(mode, dp, s); });
+    return launch(c, fp8 ? kLLCopyFp8 : kLLCopy, true, s, [&] { return ep::launch_dispatch(mode, dp, s, true); });
 }
 
 }  // namespace

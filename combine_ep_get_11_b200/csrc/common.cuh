@@ -88,6 +88,24 @@ __device__ __forceinline__ void st_stream_v4(uint4* p, const uint4& v) {
                  : "memory");
 }
 
+// ----------------------------------------- programmatic dependent launch
+// A kernel launched with the programmatic stream-serialization attribute may
+// start while the previous kernel on its stream is still running, once every
+// block of that kernel has executed pdl_launch_dependents (or exited).  It
+// must execute pdl_wait before it reads anything the previous kernel writes;
+// the wait returns when that kernel has completed and its writes are visible.
+// Both are no-ops for kernels launched without the attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned, bytes % 16 == 0).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // bf16 pair (packed in a u32, low half first) -> two floats (exact).
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }

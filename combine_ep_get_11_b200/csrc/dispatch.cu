@@ -58,6 +58,19 @@ dispatch_kernel(const DispatchParams p) {
     const int part = (int)(wid % p.splits);      // column slice of its row
     if (g >= p.G) return;   // whole warp
 
+    // The normal and packed forms are launched right behind the handle / slot
+    // scan and may start before it ends: pull this warp's slice of the source
+    // row (never written by the scan) into L2 meanwhile, then wait for the scan.
+    if constexpr (kMode == kModeNormal || kMode == kModeLowLatency || kMode == kModeLowLatencyFp8) {
+        if (lane == 0) {
+            const int nv = p.H / 8;
+            const int per = ((nv + p.splits - 1) / p.splits + 31) / 32 * 32;
+            const int lo = part * per, hi = min(nv, lo + per);
+            if (lo < hi) prefetch_l2(p.x + g * p.H + (long long)lo * 8, (uint32_t)(hi - lo) * 16u);
+        }
+        pdl_wait();
+    }
+
     constexpr bool kPacked = kMode == kModeLowLatency || kMode == kModeLowLatencyFp8;
     long long row = -1;
     if (kPacked) {
@@ -213,24 +226,33 @@ dispatch_kernel(const DispatchParams p) {
 }
 
 template <int kMode>
-cudaError_t launch_mode(const DispatchParams& p, cudaStream_t stream) {
+cudaError_t launch_mode(const DispatchParams& p, cudaStream_t stream, bool after_scan) {
     const long long blocks = (p.G * p.splits + kDispatchWarps - 1) / kDispatchWarps;
     // the FP8 form also keeps the codes and scales live: hold 14 vectors per pass
     constexpr int kVec = kMode == kModeLowLatencyFp8 ? 14 : kVecPerLane;
-    dispatch_kernel<kMode, kVec><<<(unsigned)blocks, kDispatchThreads, 0, stream>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(kDispatchThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_scan ? 1 : 0;   // may overlap the scan's tail (see pdl_wait above)
+    return cudaLaunchKernelEx(&cfg, dispatch_kernel<kMode, kVec>, p);
 }
 
 }  // namespace
 
-cudaError_t launch_dispatch(int mode, const DispatchParams& p, cudaStream_t stream) {
+cudaError_t launch_dispatch(int mode, const DispatchParams& p, cudaStream_t stream, bool after_scan) {
     if (p.G == 0) return cudaSuccess;
     switch (mode) {
-        case kModeNormal: return launch_mode<kModeNormal>(p, stream);
-        case kModeCached: return launch_mode<kModeCached>(p, stream);
-        case kModeLowLatency: return launch_mode<kModeLowLatency>(p, stream);
-        case kModeLowLatencyFp8: return launch_mode<kModeLowLatencyFp8>(p, stream);
-        case kModeSharded: return launch_mode<kModeSharded>(p, stream);
+        case kModeNormal: return launch_mode<kModeNormal>(p, stream, after_scan);
+        case kModeCached: return launch_mode<kModeCached>(p, stream, false);
+        case kModeLowLatency: return launch_mode<kModeLowLatency>(p, stream, after_scan);
+        case kModeLowLatencyFp8: return launch_mode<kModeLowLatencyFp8>(p, stream, after_scan);
+        case kModeSharded: return launch_mode<kModeSharded>(p, stream, false);
         default: return cudaErrorInvalidValue;
     }
 }

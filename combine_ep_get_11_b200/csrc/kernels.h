@@ -94,7 +94,10 @@ struct DispatchParams {
     int R, E, L, T, K, H;
     int splits;                        // warps per token (column slices of the row)
 };
-cudaError_t launch_dispatch(int mode, const DispatchParams& p, cudaStream_t stream);
+// after_scan: launched right behind the handle / slot scan kernel, which lets
+// it start early (programmatic dependent launch); only the normal and packed
+// forms make use of it.
+cudaError_t launch_dispatch(int mode, const DispatchParams& p, cudaStream_t stream, bool after_scan = false);
 
 // ----------------------------------------------------------------- combine
 struct CombineParams {

@@ -79,6 +79,7 @@ ll_slot_kernel(const LLCountParams p) {
     __shared__ int s_tile;
     __shared__ unsigned long long s_tag;
     const int tid = threadIdx.x;
+    pdl_launch_dependents();   // the packed copy may start prefetching its rows
     if (tid == 0) {
         const unsigned long long tk = atomicAdd(p.ticket, 1ull);
         s_tile = (int)(tk % (unsigned long long)p.num_tiles);

@@ -62,6 +62,7 @@ scan_kernel(const ScanParams p) {
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int R = p.R;
+    pdl_launch_dependents();   // the dispatch kernel may start prefetching its rows
     if (tid == 0) {
         const unsigned long long tk = atomicAdd(p.ticket, 1ull);
         s_tile = (int)(tk % (unsigned long long)p.num_tiles);
