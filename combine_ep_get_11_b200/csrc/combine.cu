@@ -17,7 +17,8 @@
 // shared memory.  Each lane then owns 16-byte columns of the hidden row; for
 // every U-vector slab it issues the loads of a group of 4 rows at once
 // (4 x 4 vectors; measured best on B200 for fan-ins of 3.6 and 5.2), then adds
-// them in rank order, group after group.  Traffic per token: fan-out *
+// them in rank order, group after group.  Lane i also asks for the next column
+// slab of row i ahead of time (a bulk L2 prefetch), so the slab's loads hit L2.  Traffic per token: fan-out *
 // H*2 bytes read (streaming), H*2 written.  The sharded form reads rank d's
 // rows from the GPU hosting d (its own memory or a peer's, mapped into this
 // process): the return exchange happens inside the reduction.
@@ -90,7 +91,14 @@ combine_kernel(const CombineParams p) {
     const int nvec = p.H / 8;
     const int per = ((nvec + p.splits - 1) / p.splits + 31) / 32 * 32;
     const int lo = part * per, hi = min(nvec, lo + per);
+    // rows' next column slab into L2 ahead of its loads (lane i: row i of the token)
+    // (not in the sharded form, whose rows may live in a peer GPU's memory)
+    const uint4* pf_row = nullptr;
+    if (!kSharded && lane < f) pf_row = reinterpret_cast<const uint4*>(p.y + s_rows[warp][lane] * p.H);
+    if (pf_row != nullptr && lo < hi) prefetch_l2(pf_row + lo, (uint32_t)min(32 * U, hi - lo) * 16u);
     for (int c0 = lo; c0 < hi; c0 += 32 * U) {
+        const int nxt = c0 + 32 * U;
+        if (pf_row != nullptr && nxt < hi) prefetch_l2(pf_row + nxt, (uint32_t)min(32 * U, hi - nxt) * 16u);
         float acc[U][8];
 #pragma unroll
         for (int u = 0; u < U; ++u)

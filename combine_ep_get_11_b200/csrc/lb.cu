@@ -126,7 +126,13 @@ lb_reduce_kernel(const LBParams p) {
         acc[u][0] = bf16_lo(g0.x); acc[u][1] = bf16_hi(g0.x); acc[u][2] = bf16_lo(g0.y); acc[u][3] = bf16_hi(g0.y);
         acc[u][4] = bf16_lo(g0.z); acc[u][5] = bf16_hi(g0.z); acc[u][6] = bf16_lo(g0.w); acc[u][7] = bf16_hi(g0.w);
     }
+    // each replica's chunk into L2 one replica ahead of its loads
+    const long long chunk0 = (long long)blockIdx.x * kLBChunk;
+    const uint32_t chunk_bytes = (uint32_t)(min(kLBChunk, p.Wv - chunk0) * 16);
+    if (tid == 0 && n > 0 && chunk0 < p.Wv) prefetch_l2(red + (long long)s_list[0] * p.Wv + chunk0, chunk_bytes);
     for (int j = 0; j < n; ++j) {      // replicas in ascending order; all loads of one replica in flight
+        if (tid == 0 && j + 1 < n && chunk0 < p.Wv)
+            prefetch_l2(red + (long long)s_list[j + 1] * p.Wv + chunk0, chunk_bytes);
         const uint4* r = red + (long long)s_list[j] * p.Wv;
         uint4 v[kLBVec];
 #pragma unroll
