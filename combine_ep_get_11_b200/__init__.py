@@ -68,6 +68,7 @@ _SIGNATURES = {
     "ep_last_error": (ctypes.c_char_p, [_vp]),
     "ep_sync_status": (ctypes.c_int, [_vp, _vp]),
     "ep_kernel_launch_count": (ctypes.c_uint64, []),
+    "ep_test_offset_tickets": (ctypes.c_int, [_vp, _i64]),
     "ep_get_dispatch_layout": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "ep_dispatch": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(ep_handle),
                                    _vp, _vp, _vp, _i64, ctypes.POINTER(_i64), _vp, _vp]),

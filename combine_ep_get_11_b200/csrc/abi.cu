@@ -332,6 +332,41 @@ int ep_handle_layout(const ep_ctx* c, ep_handle_sizes* s) {
 
 const char* ep_last_error(const ep_ctx* c) { return c == nullptr ? "null context" : c->last_error; }
 
+namespace {
+
+int realign_tickets(ep_ctx* c) {
+    struct { unsigned long long* ticket; long long tiles; } t[2] = {
+        {c->scan_ticket, c->scan_tiles}, {c->ll_ticket, c->ll_tiles}};
+    for (auto& x : t) {
+        if (x.tiles <= 0) continue;
+        unsigned long long v = 0;
+        int rc = cuda_check(c, cudaMemcpy(&v, x.ticket, sizeof v, cudaMemcpyDeviceToHost), "read ticket");
+        if (rc != EP_OK) return rc;
+        const unsigned long long n = (unsigned long long)x.tiles;
+        v = (v + n - 1) / n * n;
+        rc = cuda_check(c, cudaMemcpy(x.ticket, &v, sizeof v, cudaMemcpyHostToDevice), "write ticket");
+        if (rc != EP_OK) return rc;
+    }
+    return EP_OK;
+}
+
+}  // namespace
+
+int ep_test_offset_tickets(ep_ctx* c, int64_t delta) {
+    if (c == nullptr || delta < 0) return EP_ERR_INVALID_ARG;
+    DeviceGuard guard(c->device);
+    int rc = cuda_check(c, cudaDeviceSynchronize(), "cudaDeviceSynchronize");
+    for (unsigned long long* tk : {c->scan_ticket, c->ll_ticket}) {
+        if (rc != EP_OK) return rc;
+        unsigned long long v = 0;
+        rc = cuda_check(c, cudaMemcpy(&v, tk, sizeof v, cudaMemcpyDeviceToHost), "read ticket");
+        if (rc != EP_OK) return rc;
+        v += (unsigned long long)delta;
+        rc = cuda_check(c, cudaMemcpy(tk, &v, sizeof v, cudaMemcpyHostToDevice), "write ticket");
+    }
+    return rc;
+}
+
 int ep_sync_status(ep_ctx* c, ep_stream_t stream) {
     if (c == nullptr) return EP_ERR_INVALID_ARG;
     DeviceGuard guard(c->device);
@@ -343,6 +378,10 @@ int ep_sync_status(ep_ctx* c, ep_stream_t stream) {
     if (rc != EP_OK) return rc;
     if (code != 0) {
         rc = cuda_check(c, cudaMemset(c->err, 0, sizeof(int)), "clear error word");
+        // a scan that gave up leaves its ticket possibly off a multiple of its tile
+        // count: move each ticket up to the next multiple (a new call number that
+        // no status word carries yet), so the next calls start consistent
+        if (rc == EP_OK && code == EP_ERR_TIMEOUT) rc = realign_tickets(c);
         if (rc != EP_OK) return rc;
         return fail(c, code, "device reported %s", ep_status_string(code));
     }

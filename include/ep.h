@@ -160,6 +160,18 @@ EP_API const char* ep_last_error(const ep_ctx* ctx);
  * no kernel recorded an error since the last call).  The only blocking call
  * besides ep_dispatch with num_recv_host. */
 EP_API int ep_sync_status(ep_ctx* ctx, ep_stream_t stream);
+/* (When it reports EP_ERR_TIMEOUT it also moves the scans' ticket counters up
+ * to the next multiple of their tile counts, so the following calls start from
+ * a consistent state.) */
+
+/* Test support for the bounded waits.  Synchronizes the device, then adds
+ * `delta` to the ticket counters of the handle scan and the low-latency slot
+ * scan.  A delta that is not a multiple of a scan's tile count makes the
+ * scan's next call give its tiles two different call tags: the tiles waiting
+ * for a word tagged with the other number give up after the wait limit (about
+ * a second) and record EP_ERR_TIMEOUT; that call's outputs are then undefined.
+ * ep_sync_status realigns the counters. */
+EP_API int ep_test_offset_tickets(ep_ctx* ctx, int64_t delta);
 
 /* Number of kernels this library has launched in this process (all contexts). */
 EP_API uint64_t ep_kernel_launch_count(void);

@@ -206,6 +206,54 @@ def test_repeated_calls_on_one_context(ep):
     buf.destroy()
 
 
+# ----------------------------------------------------------------------------- bounded waits
+
+def test_bounded_wait_runs_out_and_context_recovers(ep):
+    """Failure detection without a fault: shift the scans' ticket counters by one,
+    so the next scan's tiles carry two different call tags and the tiles waiting
+    for a word tagged with the other number give up after the wait limit.  The
+    call must end (no hang), report EP_ERR_TIMEOUT, and the context must give
+    correct results afterwards (ep_sync_status realigns the counters)."""
+    import time
+    w = synth.Workload("wait", 4, 16, 300, 64, 4, "uniform", 81)   # 5 handle tiles, 8 slot tiles
+    inp = Inputs(w)
+    buf = make_buffer(ep, w)
+    ll = oracle.ll_dispatch(inp.x_u16, inp.topk, w.num_experts, w.tmax)
+    _, h, (o_recv_x, _, _) = oracle_normal(inp)
+    N = int(h["recv_rank_offset"][-1])
+    handle = ep.Handle.empty(w.num_ranks, w.num_tokens, w.num_channels, w.local_experts, N, "cuda")
+    recv_x = torch.empty((N, w.hidden), dtype=torch.bfloat16, device="cuda")
+
+    def dispatch():
+        ep.ep_dispatch(buf.ctx, inp.x_d, inp.topk_d, None, None, None, None, handle, recv_x, None, None, N)
+
+    def check_ll():
+        _, count, (src_info, layout_range) = buf.low_latency_dispatch(inp.x_d, inp.topk_d)
+        assert buf.sync_status() == 0
+        np.testing.assert_array_equal(count.cpu().numpy(), ll["packed_recv_count"])
+        np.testing.assert_array_equal(layout_range.cpu().numpy(), ll["layout_range"])
+
+    def check_normal():
+        dispatch()
+        assert buf.sync_status() == 0
+        for key in ("send_head", "rank_prefix_matrix", "channel_prefix_matrix", "recv_rank_offset"):
+            np.testing.assert_array_equal(getattr(handle, key).cpu().numpy(), h[key], err_msg=key)
+        np.testing.assert_array_equal(u16(recv_x), o_recv_x)
+
+    check_ll()
+    check_normal()
+    lib = ep.load()
+    for skewed in (lambda: buf.low_latency_dispatch(inp.x_d, inp.topk_d), dispatch):
+        assert lib.ep_test_offset_tickets(buf.ctx, 1) == 0
+        t0 = time.monotonic()
+        skewed()                              # outputs undefined: some tiles give up
+        assert buf.sync_status() == 6         # EP_ERR_TIMEOUT
+        assert time.monotonic() - t0 < 60
+        check_ll()
+        check_normal()
+    buf.destroy()
+
+
 # ----------------------------------------------------------------------------- edge cases
 
 def test_no_tokens(ep):
