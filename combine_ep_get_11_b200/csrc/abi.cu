@@ -674,7 +674,7 @@ int ep_ll_combine(ep_ctx* c, const uint16_t* y, const int64_t* topk_idx, const f
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     int rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
     if (rc != EP_OK) return rc;
-    ep::LLCombineParams p{y, topk_idx, topk_weights, src_info, layout_range, c->rank_mask, out_x, c->err,
+    ep::LLCombineParams p{y, topk_idx, topk_weights, src_info, layout_range, c->rank_mask, c->slot_map, out_x, c->err,
                           c->G, c->R, c->E, c->T, c->K, c->H, c->ll_cap,
                           ep::combine_splits(c->H)};
     return launch(c, kLLCombine, c->G > 0, s, [&] { return ep::launch_ll_combine(p, c->num_sms, s); });

@@ -171,6 +171,7 @@ struct LLCombineParams {
     const int* src_info;        // [E][ll_cap]
     const int* layout_range;    // [E][R][2]
     const int* rank_mask;       // [R], 0 active / 1 masked
+    const int* slot_hint;       // [G][K] slots of the last low-latency dispatch, or null (checked against the handle)
     uint16_t* out_x;            // [G][H]
     int* err;
     long long G;

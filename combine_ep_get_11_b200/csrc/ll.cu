@@ -16,9 +16,10 @@
 // slot map for the copy kernel (the dispatch kernel's packed mode).  No atomic
 // decides an order, so the packing is deterministic.
 //
-// ll_combine_kernel: one warp per token.  Lane k finds the slot of its expert
-// by binary search in src_info inside layout_range[e][s] (ascending token
-// ids), the valid slots are ranked by (expert id, k), and the rows are reduced
+// ll_combine_kernel: one warp per token.  Lane k finds the slot of its expert:
+// the slot the last low-latency dispatch on the context gave (token, k), if the
+// handle confirms it (inside layout_range[e][s] and holding the token), else by
+// binary search in src_info inside layout_range[e][s] (ascending token ids), the valid slots are ranked by (expert id, k), and the rows are reduced
 // with an fp32 fused multiply-add chain in that order.
 
 #include "common.cuh"
@@ -253,24 +254,36 @@ ll_combine_kernel(const LLCombineParams p) {
         const bool src_masked = p.rank_mask[s] != 0;   // warp-uniform: the token took no part
         long long e = -1;
         float w = 0.f;
+        int hint = -1;
         if (lane < p.K && !src_masked) {
             e = p.topk_idx[g * p.K + lane];
             w = p.topk_weights[g * p.K + lane];
+            if (p.slot_hint != nullptr) hint = p.slot_hint[g * p.K + lane];
         }
         bool valid = e >= 0 && e < p.E && p.rank_mask[(int)e / (p.E / p.R)] == 0;
         long long row = -1;
         if (valid) {
             const int* range = p.layout_range + ((long long)e * p.R + s) * 2;
+            const int* info = p.src_info + e * cap;
+            // the slot the last dispatch gave (token, k), if it is this token's
+            // slot under this handle: inside source s's range and holding t (a
+            // token appears once per list, so that slot is the one)
+            const int hint_t = (hint >= 0 && hint < cap) ? info[hint] : -1;
             int lo = max(range[0], 0);
             const int end = (int)min((long long)lo + max(range[1], 0), cap);
-            const int* info = p.src_info + e * cap;
-            int hi = end;
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (info[mid] < t) lo = mid + 1; else hi = mid;
+            int slot = -1;
+            if (hint >= lo && hint < end && hint_t == t) {
+                slot = hint;
+            } else {   // binary search of t in the source's ascending token ids
+                int hi = end;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (info[mid] < t) lo = mid + 1; else hi = mid;
+                }
+                if (lo < end && info[lo] == t) slot = lo;
             }
-            if (lo < end && info[lo] == t) {
-                row = e * cap + lo;
+            if (slot >= 0) {
+                row = e * cap + slot;
             } else {
                 record_error(p.err, EP_ERR_HANDLE_MISMATCH);
                 valid = false;

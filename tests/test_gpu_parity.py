@@ -206,6 +206,27 @@ def test_repeated_calls_on_one_context(ep):
     buf.destroy()
 
 
+def test_ll_combine_with_an_older_handle(ep):
+    """The low-latency combine takes the last dispatch's slots only where the
+    handle it is given confirms them: combining routing A's rows with A's handle
+    after a dispatch of routing B must still give A's result."""
+    w = synth.Workload("ll-old", 8, 64, 96, 128, 6, "uniform_masked", 80, mask_prob=0.1)
+    a = Inputs(w)
+    b = Inputs(dataclasses.replace(w, seed=w.seed + 1))
+    buf = make_buffer(ep, w)
+    packed_a, _, handle_a = buf.low_latency_dispatch(a.x_d, a.topk_d)
+    buf.low_latency_dispatch(b.x_d, b.topk_d)                     # the context now holds B's slots
+    out = buf.low_latency_combine(packed_a, a.topk_d, a.weights_d, handle_a)
+    assert buf.sync_status() == 0
+    ll = oracle.ll_dispatch(a.x_u16, a.topk, w.num_experts, w.tmax)
+    ref = oracle.ll_combine(ll["packed_recv_x"], a.topk, a.weights, ll["src_info"], ll["layout_range"],
+                            w.num_experts, w.tmax)
+    abs_ref = oracle.ll_combine(bf16_abs(ll["packed_recv_x"]), a.topk, np.abs(a.weights), ll["src_info"],
+                                ll["layout_range"], w.num_experts, w.tmax)
+    assert_combine_close(u16(out), ref, abs_ref, w.topk, "ll combine, older handle")
+    buf.destroy()
+
+
 # ----------------------------------------------------------------------------- bounded waits
 
 def test_bounded_wait_runs_out_and_context_recovers(ep):
