@@ -69,6 +69,7 @@ _SIGNATURES = {
     "ep_sync_status": (ctypes.c_int, [_vp, _vp]),
     "ep_kernel_launch_count": (ctypes.c_uint64, []),
     "ep_test_offset_tickets": (ctypes.c_int, [_vp, _i64]),
+    "ep_check_handle": (ctypes.c_int, [_vp, _vp, ctypes.POINTER(ep_handle), _vp, _vp]),
     "ep_get_dispatch_layout": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "ep_dispatch": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(ep_handle),
                                    _vp, _vp, _vp, _i64, ctypes.POINTER(_i64), _vp, _vp]),
@@ -393,6 +394,17 @@ class Buffer:
                     recv_w if recv_capacity else None, recv_capacity, stream=stream)
         handle.num_recv_rows = recv_capacity
         return recv_x, recv_idx, recv_w, handle
+
+    def check_handle(self, topk_idx, handle: Handle, stream=None) -> bool:
+        """True if `handle` is the dispatch handle of this routing (the reuse
+        contract); synchronizes the stream to read the verdict."""
+        hs = handle.c_struct()
+        _check(load().ep_check_handle(self.ctx, _ptr(topk_idx), ctypes.byref(hs), _stream(stream), None),
+               "ep_check_handle", self.ctx)
+        rc = ep_sync_status(self.ctx, stream)
+        if rc not in (EP_OK, 5):
+            _check(rc, "device status", self.ctx)
+        return rc == EP_OK
 
     def dispatch_cached(self, x, handle: Handle, stream=None):
         recv_x = torch.empty((handle.num_recv_rows, self.H), dtype=torch.bfloat16, device=self.device)

@@ -17,8 +17,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build", "libep")
 LIB = os.path.join(PKG, "libep.so")
-SOURCES = ["abi.cu", "layout.cu", "scan.cu", "dispatch.cu", "combine.cu", "ll.cu", "lb.cu", "noalloc.cu", "shard.cu"]
-HEADERS = ["common.cuh", "kernels.h"]
+SOURCES = ["abi.cu", "layout.cu", "scan.cu", "dispatch.cu", "combine.cu", "ll.cu", "lb.cu", "noalloc.cu", "shard.cu", "check.cu"]
+HEADERS = ["common.cuh", "kernels.h", "check.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 NVCC_FLAGS = [

@@ -19,6 +19,7 @@
 #include <vector>
 
 #include "../../include/ep.h"
+#include "check.h"
 #include "kernels.h"
 
 struct ep_prof_rec {
@@ -928,6 +929,24 @@ int ep_ipc_open(const uint8_t* ipc_handle, void** ptr) {
 }
 
 int ep_ipc_close(void* ptr) { return cudaIpcCloseMemHandle(ptr) == cudaSuccess ? EP_OK : EP_ERR_CUDA; }
+
+int ep_check_handle(ep_ctx* c, const int64_t* topk_idx, const ep_handle* h, ep_stream_t stream,
+                    ep_event_t wait_event) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (c->num_shards > 1) return fail(c, EP_ERR_INVALID_ARG, "sharded context: the handle check is one-GPU");
+    int rc = check_handle(c, h);
+    if (rc != EP_OK) return rc;
+    if (c->G > 0 && topk_idx == nullptr) return fail(c, EP_ERR_INVALID_ARG, "topk_idx missing");
+    if (!aligned(topk_idx, 8)) return fail(c, EP_ERR_ALIGNMENT, "topk_idx misaligned");
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
+    if (rc != EP_OK) return rc;
+    ep::HandleCheckParams p{topk_idx, h->is_token_in_rank, h->send_head,
+                            reinterpret_cast<const long long*>(h->recv_rank_offset), c->err, c->G,
+                            c->R, c->E, c->L, c->K};
+    return launch(c, -1, c->G > 0, s, [&] { return ep::launch_handle_check(p, s); });
+}
 
 int ep_profile_enable(ep_ctx* c, int enable) {
     if (c == nullptr) return EP_ERR_INVALID_ARG;

@@ -176,6 +176,17 @@ EP_API int ep_test_offset_tickets(ep_ctx* ctx, int64_t delta);
 /* Number of kernels this library has launched in this process (all contexts). */
 EP_API uint64_t ep_kernel_launch_count(void);
 
+/* Handle check for the reuse contract ([REUSE] "Performance Contract and
+ * Constraints": a handle stays valid only while topk_idx is unchanged).
+ * Recomputes each token's destination ranks from topk_idx (i64 [R][T][K]) and
+ * compares them with the handle's is_token_in_rank and send_head (>= 0 exactly
+ * for those ranks, and below each rank's receive count from recv_rank_offset).
+ * A difference records EP_ERR_HANDLE_MISMATCH for ep_sync_status.  Reads
+ * G*(K*8 + R*5) bytes; stream-ordered; blocks nothing.  Not on a sharded
+ * context. */
+EP_API int ep_check_handle(ep_ctx* ctx, const int64_t* topk_idx, const ep_handle* handle,
+                           ep_stream_t stream, ep_event_t wait_event);
+
 /* Dispatch layout ([API] "Configuration and Layout Helpers", [ARCH] table
  * "Buffer.get_dispatch_layout").
  *   topk_idx              i64 [R][T][K]  input

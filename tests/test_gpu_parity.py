@@ -227,6 +227,36 @@ def test_ll_combine_with_an_older_handle(ep):
     buf.destroy()
 
 
+def test_handle_check(ep):
+    """The reuse contract: a handle checks out against its own routing, or one that
+    sends every token to the same ranks, and fails against any other."""
+    w = W["dsv3"].scaled(num_tokens=300, hidden=64)
+    a = Inputs(w)
+    b = Inputs(dataclasses.replace(w, seed=w.seed + 1))
+    buf = make_buffer(ep, w)
+    _, _, _, handle = buf.dispatch(a.x_d, a.topk_d, a.weights_d)
+    assert buf.check_handle(a.topk_d, handle)
+    assert not buf.check_handle(b.topk_d, handle)
+    L = w.local_experts
+    topk = a.topk.copy()
+    flat = topk.reshape(-1, w.topk)
+    # same ranks: swap one expert for another expert of the same rank
+    g = int(np.nonzero(flat[:, 0] >= 0)[0][0])
+    e = int(flat[g, 0])
+    flat[g, 0] = e // L * L + (e % L + 1) % L
+    assert buf.check_handle(torch.from_numpy(topk).cuda(), handle)
+    # another rank: one token's set of destination ranks changes
+    for g in range(flat.shape[0]):
+        ranks = {int(x) // L for x in flat[g] if x >= 0}
+        if len(ranks) < w.num_ranks and flat[g, 0] >= 0:
+            break
+    r = next(r for r in range(w.num_ranks) if r not in ranks)
+    flat[g, 0] = r * L
+    assert not buf.check_handle(torch.from_numpy(topk).cuda(), handle)
+    assert buf.sync_status() == 0
+    buf.destroy()
+
+
 # ----------------------------------------------------------------------------- bounded waits
 
 def test_bounded_wait_runs_out_and_context_recovers(ep):
