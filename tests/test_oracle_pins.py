@@ -206,6 +206,45 @@ def test_handle_matches_sort_formulation(R, E, T, K, C, mask_p):
                                   exp_nte.sum(0).reshape(R, L))
 
 
+def _random_shape(seed):
+    rng = np.random.default_rng(0xC0FFEE + seed)
+    R = int(rng.integers(1, 9))
+    E = R * int(rng.integers(1, 5))
+    T = int(rng.integers(0, 21))
+    K = int(rng.integers(1, min(E, 6) + 1))
+    C = int(rng.integers(1, 9))
+    mask_p = float(rng.choice([0.0, 0.2, 0.5, 1.0]))
+    distinct = bool(rng.integers(0, 2))
+    return rng, R, E, T, K, C, mask_p, distinct
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_random_shapes_match_the_independent_formulations(seed):
+    """Forty seeded tiny shapes, T = 0, fully masked and repeated experts included:
+    the handle against the sort formulation, the low-latency lists against the
+    per-expert enumeration."""
+    rng, R, E, T, K, C, mask_p, distinct = _random_shape(seed)
+    topk = random_topk(rng, R, E, T, K, mask_p, distinct=distinct)
+    if distinct:
+        _, _, _, h, _ = run_oracle_dispatch(topk, E, C)
+        b = brute_handle(topk, E, C)
+        for key in ("send_head", "recv_src_idx", "recv_rank_offset", "rank_prefix_matrix",
+                    "channel_prefix_matrix", "recv_channel_prefix_matrix"):
+            np.testing.assert_array_equal(h[key], b[key], err_msg=f"{key} {(R, E, T, K, C, mask_p)}")
+    x = f32_to_bf16_torch(rng.standard_normal((R, T, 8)).astype(np.float32))
+    ll = oracle.ll_dispatch(x, topk, E, max(T, 1))
+    L = E // R
+    for e, lst in brute_ll(topk, E).items():
+        d, j = divmod(e, L)
+        assert ll["packed_recv_count"][d, j] == len(lst)
+        for slot, (s_, t) in enumerate(lst):
+            assert ll["src_info"][d, j, slot] == t
+        for s_ in range(R):
+            begin = sum(1 for (ss, _) in lst if ss < s_)
+            cnt = sum(1 for (ss, _) in lst if ss == s_)
+            assert ll["layout_range"][d, j, s_].tolist() == [begin, cnt]
+
+
 def test_dispatch_rows_and_combine_integer_rows():
     """Rows carry exact small integers; the combine sum and every row copy are exact."""
     rng = np.random.default_rng(7)
