@@ -5,12 +5,18 @@
 // Entry point -> kernels (all on the caller's stream):
 //   ep_get_dispatch_layout : memset(histograms) + layout_kernel
 //   ep_dispatch            : [layout_kernel] + scan_kernel (call-tagged scan state, nothing to clear)
-//                            [+ one host read of N] + dispatch_kernel<normal>
+//                            [+ one host read of N] + dispatch_kernel<normal> (programmatic
+//                            launch behind the scan)
 //   ep_dispatch_cached     : dispatch_kernel<cached>
 //   ep_combine             : combine_kernel
-//   ep_ll_dispatch[_fp8]   : ll_slot_kernel (call-tagged scan state, nothing to clear) + dispatch_kernel<packed[, FP8]>
+//   ep_ll_dispatch[_fp8]   : ll_slot_kernel (call-tagged scan state, nothing to clear) +
+//                            dispatch_kernel<packed[, FP8]> (programmatic launch behind the scan)
 //   ep_ll_combine          : ll_combine_kernel
 //   ep_lb_prefetch_weights : lb_prefetch_kernel;  ep_lb_reduce_grads : lb_reduce_kernel
+//   ep_sharded_handle      : shard_offsets_kernel + scan_kernel (with the shard's base)
+//   ep_sharded_dispatch    : dispatch_kernel<sharded>;  ep_sharded_combine : combine_kernel<sharded>
+//   ep_check_handle        : handle_check_kernel
+//   ep_ll_update_mask / ep_ll_clean_mask : set_mask_kernel / memset
 
 #include <atomic>
 #include <cstdarg>
