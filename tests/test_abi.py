@@ -90,3 +90,8 @@ def test_sharded_null_arguments(lib):
     assert lib.ep_sharded_combine(None, 1, None, None, 0, None, None, None, None, None, None, None, None) == 1
     assert lib.ep_shared_alloc(0, None, None) == 1
     assert lib.ep_ipc_open(None, None) == 1
+
+
+def test_check_and_test_support_null_arguments(lib):
+    assert lib.ep_check_handle(None, None, None, None, None) == 1
+    assert lib.ep_test_offset_tickets(None, 1) == 1
