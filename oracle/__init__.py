@@ -41,19 +41,22 @@ def load_library(path: str):
                                            _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr]
     L.oracle_combine.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _ptr, _c_i64, _ptr, _ptr,
                                      _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _c_i64]
+    L.oracle_combine_fp32.argtypes = L.oracle_combine.argtypes
     L.oracle_ll_dispatch.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
                                          _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr]
     L.oracle_ll_combine.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
                                         _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _c_i64, _ptr]
+    L.oracle_ll_combine_fp32.argtypes = L.oracle_ll_combine.argtypes
     L.oracle_fp8_e4m3_encode.argtypes = [_ptr, _ptr, _c_i64]
     L.oracle_fp8_e4m3_encode.restype = None
     L.oracle_quantize_e4m3_blocks.argtypes = [_ptr, _c_i64, _c_i32, _c_i32, _ptr, _ptr]
     L.oracle_lb_prefetch_weights.argtypes = [_ptr, _c_i32, _c_i64, _ptr, _c_i32, _ptr]
     L.oracle_lb_reduce_grads.argtypes = [_ptr, _ptr, _c_i32, _ptr, _c_i32, _c_i64]
+    L.oracle_lb_reduce_grads_fp32.argtypes = L.oracle_lb_reduce_grads.argtypes
     for name in ("oracle_layout", "oracle_dispatch_handle", "oracle_dispatch_rows",
-                 "oracle_combine", "oracle_ll_dispatch", "oracle_ll_combine",
-                 "oracle_quantize_e4m3_blocks", "oracle_lb_prefetch_weights",
-                 "oracle_lb_reduce_grads"):
+                 "oracle_combine", "oracle_combine_fp32", "oracle_ll_dispatch", "oracle_ll_combine",
+                 "oracle_ll_combine_fp32", "oracle_quantize_e4m3_blocks", "oracle_lb_prefetch_weights",
+                 "oracle_lb_reduce_grads", "oracle_lb_reduce_grads_fp32"):
         getattr(L, name).restype = ctypes.c_int
     return L
 
@@ -152,8 +155,12 @@ def dispatch_rows(x, topk_idx: np.ndarray, topk_weights, handle: dict, num_exper
 
 
 def combine(y: np.ndarray, handle: dict, recv_topk_weights=None, bias0=None, bias1=None,
-            tokens=None, topk: int | None = None):
-    """y [N,H] u16 -> (out_x [R,T,H] u16 or [n,H] for a token list, out_w or None)."""
+            tokens=None, topk: int | None = None, fp32: bool = False):
+    """y [N,H] u16 -> (out_x [R,T,H] u16 or [n,H] for a token list, out_w or None).
+
+    fp32=False: the exact sum (fp64 accumulation, one bf16 rounding).
+    fp32=True: the fixed-order fp32 definition (ascending destination rank, then
+    the biases; binary32 additions from +0, one bf16 rounding)."""
     y = np.ascontiguousarray(y, dtype=np.uint16)
     sh = handle["send_head"]
     R, T, _ = sh.shape
@@ -170,10 +177,11 @@ def combine(y: np.ndarray, handle: dict, recv_topk_weights=None, bias0=None, bia
     out_w = np.empty((n, K), np.float32) if rw is not None else None
     b0 = None if bias0 is None else np.ascontiguousarray(bias0, dtype=np.uint16)
     b1 = None if bias1 is None else np.ascontiguousarray(bias1, dtype=np.uint16)
-    _check(lib().oracle_combine(
+    fn = lib().oracle_combine_fp32 if fp32 else lib().oracle_combine
+    _check(fn(
         R, T, K, H, _p(y), y.shape[0], _p(sh), _p(handle["recv_rank_offset"]), _p(rw),
         _p(b0), _p(b1), _p(out), _p(out_w), _p(tok), 0 if tok is None else tok.size),
-        "oracle_combine")
+        "oracle_combine" + ("_fp32" if fp32 else ""))
     if tok is None:
         out = out.reshape(R, T, H)
         if out_w is not None:
@@ -212,7 +220,10 @@ def ll_dispatch(x, topk_idx, num_experts: int, max_tokens_per_rank: int, with_ro
 
 
 def ll_combine(y, topk_idx, topk_weights, src_info, layout_range, num_experts: int,
-               max_tokens_per_rank: int, tokens=None, rank_mask=None):
+               max_tokens_per_rank: int, tokens=None, rank_mask=None, fp32: bool = False):
+    """Weighted low-latency combine.  fp32=False: the exact sum (fp64, one bf16
+    rounding); fp32=True: the fixed-order definition (binary32 fused multiply-add
+    chain from +0 over ascending (expert id, k), one bf16 rounding)."""
     y = np.ascontiguousarray(y, dtype=np.uint16)
     topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int64)
     w = np.ascontiguousarray(topk_weights, dtype=np.float32)
@@ -221,11 +232,13 @@ def ll_combine(y, topk_idx, topk_weights, src_info, layout_range, num_experts: i
     tok = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int64)
     n = R * T if tok is None else tok.size
     out = np.empty((n, H), np.uint16)
-    _check(lib().oracle_ll_combine(
+    fn = lib().oracle_ll_combine_fp32 if fp32 else lib().oracle_ll_combine
+    _check(fn(
         R, num_experts, T, K, H, max_tokens_per_rank, _p(y), _p(topk_idx), _p(w),
         _p(np.ascontiguousarray(src_info, dtype=np.int32)),
         _p(np.ascontiguousarray(layout_range, dtype=np.int32)), _p(out), _p(tok),
-        0 if tok is None else tok.size, _p(_mask(rank_mask, R))), "oracle_ll_combine")
+        0 if tok is None else tok.size, _p(_mask(rank_mask, R))),
+        "oracle_ll_combine" + ("_fp32" if fp32 else ""))
     return out.reshape(R, T, H) if tok is None else out
 
 
@@ -259,12 +272,15 @@ def lb_prefetch_weights(expert_weights, mapping, redundant_weights):
     return out
 
 
-def lb_reduce_grads(redundant_grads, mapping, expert_grads):
-    """redundant_grads [N, W] u16, mapping [N] i32, expert_grads [E, W] u16 -> new expert_grads."""
+def lb_reduce_grads(redundant_grads, mapping, expert_grads, fp32: bool = False):
+    """redundant_grads [N, W] u16, mapping [N] i32, expert_grads [E, W] u16 -> new expert_grads.
+    fp32=False: the exact sum (fp64); fp32=True: the fixed-order definition (binary32
+    additions from the original gradient over ascending replica index)."""
     rg = np.ascontiguousarray(redundant_grads, dtype=np.uint16)
     m = np.ascontiguousarray(mapping, dtype=np.int32)
     out = np.array(expert_grads, dtype=np.uint16, copy=True, order="C")
     E, W = out.shape
-    _check(lib().oracle_lb_reduce_grads(_p(rg), _p(m), m.size, _p(out), E, W),
-           "oracle_lb_reduce_grads")
+    fn = lib().oracle_lb_reduce_grads_fp32 if fp32 else lib().oracle_lb_reduce_grads
+    _check(fn(_p(rg), _p(m), m.size, _p(out), E, W),
+           "oracle_lb_reduce_grads" + ("_fp32" if fp32 else ""))
     return out

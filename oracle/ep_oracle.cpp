@@ -28,13 +28,27 @@
 // x[s][0..T).  A global token id is g = s * T + t.  rank(e) = e / L,
 // loc(e) = e mod L, an expert id of -1 marks an unused slot.
 //
-// Floating point: the combines are accumulated in double (fp64) and rounded
-// once to bf16 (round to nearest, ties to even).  bf16 values are passed as
-// their raw 16-bit patterns.
+// Floating point: every reduction is stated twice.
+//   * The fixed-order fp32 definition (oracle_combine_fp32,
+//     oracle_ll_combine_fp32, oracle_lb_reduce_grads_fp32): an fp32
+//     accumulator starting at +0 (or at the original gradient), one IEEE
+//     binary32 operation per term in the stated order (round to nearest even;
+//     the low-latency combine uses a fused multiply-add, one rounding per
+//     term), then one rounding to bf16.  This is the result the method
+//     computes, bit for bit, so the CUDA path must match it exactly.
+//   * The exact sum (oracle_combine, oracle_ll_combine, oracle_lb_reduce_grads):
+//     accumulated in double (exact for these term counts and magnitudes up to
+//     the last bits) and rounded once to bf16.  It is the reference for the
+//     "within one bf16 ulp" accuracy statement.
+// bf16 values are passed as their raw 16-bit patterns.  Built with
+// -ffp-contract=off so no multiply and add is fused unless written as fma.
 //
 // Parity status: every function here is pinned by tests/test_oracle_pins.py
 // (brute force with an independent sort-based formulation, closed forms,
-// invariants, special cases and a hand-worked fixture).
+// invariants, special cases and hand-worked fixtures; the summation order and
+// the fused multiply-add of the fp32 reductions by hand-worked cancellation
+// cases in tests/golden/fp32_order.txt), and tests/test_oracle_mutations.py
+// checks that planted mistakes fail those pins.
 
 #include <cmath>
 #include <cstdint>
@@ -83,6 +97,18 @@ uint16_t double_to_bf16_bits(double v) {
     uint16_t b = static_cast<uint16_t>(u >> 16);
     return neg ? static_cast<uint16_t>(b | 0x8000) : b;
 }
+
+// bf16 bits -> float (exact: bf16 is the upper half of a binary32 pattern).
+float bf16_bits_to_float(uint16_t b) {
+    uint32_t u = static_cast<uint32_t>(b) << 16;
+    float f;
+    std::memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+// float -> bf16 bits, nearest even.  A float is exactly a double, so the
+// one-step double rounding above rounds the float itself.
+uint16_t float_to_bf16_bits(float f) { return double_to_bf16_bits(static_cast<double>(f)); }
 
 bool shape_ok(int32_t R, int32_t E, int32_t T, int32_t K) {
     return R >= 1 && E >= 1 && E % R == 0 && T >= 0 && K >= 1;
@@ -323,6 +349,58 @@ int oracle_combine(int32_t R, int32_t T, int32_t K, int32_t H,
     return ORACLE_OK;
 }
 
+// Combine, fixed-order fp32 definition (same arguments as oracle_combine).
+// The reduction of [API] "Combine Operation" taken as the method computes it:
+// an fp32 accumulator starting at +0 adds, one binary32 addition each (round
+// to nearest even), the token's received rows in ascending destination rank,
+// then bias0, then bias1, and is rounded once to bf16:
+//   acc = +0;  for d = 0, 1, ..., R-1 with h = send_head[s][t][d] >= 0:
+//                  acc = acc + y[off_d + h][i]
+//   acc = acc + bias0[s][t][i];  acc = acc + bias1[s][t][i];  out = bf16(acc)
+// The combined weights take the same ascending-rank fp32 sum of the received
+// weight rows.
+int oracle_combine_fp32(int32_t R, int32_t T, int32_t K, int32_t H,
+                        const uint16_t* y, int64_t y_rows, const int32_t* send_head,
+                        const int64_t* recv_rank_offset, const float* recv_topk_weights,
+                        const uint16_t* bias0, const uint16_t* bias1,
+                        uint16_t* out_x, float* out_topk_weights,
+                        const int64_t* tokens, int64_t n_tokens) {
+    if (R < 1 || T < 0 || K < 1 || H < 1) return ORACLE_BAD_ARG;
+    const int64_t G = (int64_t)R * T;
+    const int64_t n = tokens != nullptr ? n_tokens : G;
+    std::vector<float> sum32(H);
+    for (int64_t i = 0; i < n; ++i) {
+        const int64_t g = tokens != nullptr ? tokens[i] : i;
+        if (g < 0 || g >= G) return ORACLE_BAD_ARG;
+        std::fill(sum32.begin(), sum32.end(), 0.0f);
+        for (int32_t dst = 0; dst < R; ++dst) {          // ascending destination rank
+            const int32_t h = send_head[g * R + dst];
+            if (h < 0) continue;
+            const int64_t row = recv_rank_offset[dst] + h;
+            if (row >= y_rows) return ORACLE_CAPACITY;
+            for (int32_t c = 0; c < H; ++c) sum32[c] = sum32[c] + bf16_bits_to_float(y[row * H + c]);
+        }
+        if (bias0 != nullptr)
+            for (int32_t c = 0; c < H; ++c) sum32[c] = sum32[c] + bf16_bits_to_float(bias0[g * H + c]);
+        if (bias1 != nullptr)
+            for (int32_t c = 0; c < H; ++c) sum32[c] = sum32[c] + bf16_bits_to_float(bias1[g * H + c]);
+        if (out_x != nullptr)
+            for (int32_t c = 0; c < H; ++c) out_x[i * H + c] = float_to_bf16_bits(sum32[c]);
+        if (out_topk_weights != nullptr && recv_topk_weights != nullptr) {
+            for (int32_t k = 0; k < K; ++k) {
+                float w32 = 0.0f;
+                for (int32_t dst = 0; dst < R; ++dst) {
+                    const int32_t h = send_head[g * R + dst];
+                    if (h < 0) continue;
+                    w32 = w32 + recv_topk_weights[(recv_rank_offset[dst] + h) * K + k];
+                }
+                out_topk_weights[i * K + k] = w32;
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
 // Low-latency dispatch.  [API] "IB-GDA Kernels" and "Low-Latency Inference
 // with FP8": tokens are streamed into per-expert packed receive buffers bounded
 // by num_max_dispatch_tokens_per_rank (Tmax); the call returns the packed rows,
@@ -425,6 +503,57 @@ int oracle_ll_combine(int32_t R, int32_t E, int32_t T, int32_t K, int32_t H, int
             for (int32_t c = 0; c < H; ++c) acc[c] += w * bf16_bits_to_double(row[c]);
         }
         for (int32_t c = 0; c < H; ++c) out[i * H + c] = double_to_bf16_bits(acc[c]);
+    }
+    return ORACLE_OK;
+}
+
+// Low-latency combine, fixed-order fp32 definition (same arguments as
+// oracle_ll_combine).  The weighted reduction of [API] "IB-GDA Kernels" taken
+// as the method computes it: the token's valid slots are visited in ascending
+// (expert id, slot k), and each adds w * y with one fused multiply-add
+// (binary32, one rounding of the exact w * y + acc), starting from +0; the
+// result is rounded once to bf16:
+//   acc = +0;  for (e, k) ascending:  acc = fma(w[s][t][k], y[e][slot][i], acc)
+//   out = bf16(acc)
+int oracle_ll_combine_fp32(int32_t R, int32_t E, int32_t T, int32_t K, int32_t H, int32_t Tmax,
+                           const uint16_t* y, const int64_t* topk_idx, const float* topk_weights,
+                           const int32_t* src_info, const int32_t* layout_range, uint16_t* out,
+                           const int64_t* tokens, int64_t n_tokens, const int32_t* rank_mask) {
+    if (!shape_ok(R, E, T, K) || H < 1 || Tmax < T) return ORACLE_BAD_ARG;
+    const int32_t L = E / R;
+    const int64_t cap = (int64_t)R * Tmax;
+    const int64_t G = (int64_t)R * T;
+    const int64_t n = tokens != nullptr ? n_tokens : G;
+    std::vector<float> chain(H);
+    std::vector<std::pair<int64_t, int32_t>> visit;   // (expert id, k), sorted
+    for (int64_t i = 0; i < n; ++i) {
+        const int64_t g = tokens != nullptr ? tokens[i] : i;
+        if (g < 0 || g >= G) return ORACLE_BAD_ARG;
+        const int32_t s = (int32_t)(g / T), t = (int32_t)(g % T);
+        visit.clear();
+        for (int32_t k = 0; k < K; ++k) {
+            const int64_t e = topk_idx[g * K + k];
+            if (e == -1) continue;
+            if (e < -1 || e >= E) return ORACLE_BAD_TOPK;
+            if (rank_mask != nullptr && (rank_mask[s] != 0 || rank_mask[e / L] != 0)) continue;
+            visit.emplace_back(e, k);
+        }
+        std::sort(visit.begin(), visit.end());
+        std::fill(chain.begin(), chain.end(), 0.0f);
+        for (const auto& slot_of : visit) {
+            const int64_t e = slot_of.first;
+            const int32_t k = slot_of.second;
+            const int32_t first = layout_range[(e * R + s) * 2 + 0];
+            const int32_t count = layout_range[(e * R + s) * 2 + 1];
+            int64_t slot = -1;
+            for (int32_t p = first; p < first + count; ++p)
+                if (src_info[e * cap + p] == t) { slot = p; break; }
+            if (slot < 0) return ORACLE_NOT_FOUND;
+            const float w32 = topk_weights[g * K + k];
+            const uint16_t* yrow = y + (e * cap + slot) * H;
+            for (int32_t c = 0; c < H; ++c) chain[c] = std::fma(w32, bf16_bits_to_float(yrow[c]), chain[c]);
+        }
+        for (int32_t c = 0; c < H; ++c) out[i * H + c] = float_to_bf16_bits(chain[c]);
     }
     return ORACLE_OK;
 }
@@ -533,6 +662,30 @@ int oracle_lb_reduce_grads(const uint16_t* redundant_grads, const int32_t* mappi
             for (int32_t i = 0; i < N; ++i)
                 if (mapping[i] == e) acc += bf16_bits_to_double(redundant_grads[(int64_t)i * W + c]);
             expert_grads[(int64_t)e * W + c] = double_to_bf16_bits(acc);
+        }
+    }
+    return ORACLE_OK;
+}
+
+// Gradient reduction, fixed-order fp32 definition (same arguments as
+// oracle_lb_reduce_grads): an fp32 accumulator starts at the original
+// gradient and adds, one binary32 addition each, the replicas' gradients in
+// ascending replica index; one rounding to bf16 at the end.
+int oracle_lb_reduce_grads_fp32(const uint16_t* redundant_grads, const int32_t* mapping, int32_t N,
+                                uint16_t* expert_grads, int32_t E, int64_t W) {
+    if (E < 1 || W < 1 || N < 0) return ORACLE_BAD_ARG;
+    for (int32_t i = 0; i < N; ++i)
+        if (mapping[i] < -1 || mapping[i] >= E) return ORACLE_BAD_TOPK;
+    std::vector<int32_t> replicas;
+    for (int32_t e = 0; e < E; ++e) {
+        replicas.clear();
+        for (int32_t i = 0; i < N; ++i)
+            if (mapping[i] == e) replicas.push_back(i);     // ascending replica index
+        if (replicas.empty()) continue;                     // untouched
+        for (int64_t c = 0; c < W; ++c) {
+            float g32 = bf16_bits_to_float(expert_grads[(int64_t)e * W + c]);
+            for (const int32_t i : replicas) g32 = g32 + bf16_bits_to_float(redundant_grads[(int64_t)i * W + c]);
+            expert_grads[(int64_t)e * W + c] = float_to_bf16_bits(g32);
         }
     }
     return ORACLE_OK;

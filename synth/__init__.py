@@ -43,6 +43,7 @@ _KIND_Y = 5
 _KIND_BIAS = 6
 _KIND_PERM = 7
 _KIND_REDUNDANCY = 8
+_KIND_CANCEL = 9
 
 
 @dataclasses.dataclass(frozen=True)
@@ -187,6 +188,41 @@ def expert_rows(seed: int, num_rows: int, hidden: int, chunk: int = 65536):
 
     with _cf.ThreadPoolExecutor(min(8, max(1, parts))) as ex:
         list(ex.map(one, range(parts)))
+    return y
+
+
+def cancel_rows(seed: int, num_rows: int, hidden: int, p_big: float = 0.5, big_exp: int = 25):
+    """[num_rows, H] numpy uint16 bf16 bit patterns whose sums cancel: each value
+    is +-2^big_exp (random sign) with probability p_big, else an N(0,1) draw
+    rounded to bf16.  Where the large terms of a sum cancel, the small ones that
+    were added next to a large one lost their low bits (binary32 keeps 24
+    significant bits), so the result depends on the order of the additions.
+    N(0,1) rows seldom show the order: their sums of a few terms are mostly
+    exact in binary32."""
+    import torch
+    rng = _rng(seed, 0, _KIND_CANCEL)
+    big = rng.random((num_rows, hidden)) < p_big
+    sign = np.where(rng.random((num_rows, hidden)) < 0.5, -1.0, 1.0)
+    small = rng.standard_normal((num_rows, hidden), dtype=np.float32)
+    v = np.where(big, sign * 2.0 ** big_exp, small).astype(np.float32)
+    return torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def cancel_rows_device(seed: int, num_rows: int, hidden: int, device="cuda", p_big: float = 0.5,
+                       big_exp: int = 25, chunk_rows: int = 1 << 16):
+    """cancel_rows' distribution drawn on the GPU with torch's seeded generator (bf16
+    tensor [num_rows, H]) for full-size workloads."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    y = torch.empty((num_rows, hidden), dtype=torch.bfloat16, device=device)
+    for lo in range(0, num_rows, chunk_rows):
+        hi = min(num_rows, lo + chunk_rows)
+        shape = (hi - lo, hidden)
+        big = torch.rand(shape, generator=gen, device=device) < p_big
+        sign = torch.where(torch.rand(shape, generator=gen, device=device) < 0.5, -1.0, 1.0)
+        small = torch.randn(shape, generator=gen, device=device)
+        y[lo:hi] = torch.where(big, sign * float(2 ** big_exp), small)
     return y
 
 

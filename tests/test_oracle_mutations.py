@@ -67,6 +67,30 @@ MUTANTS = {
         "double acc = bf16_bits_to_double(expert_grads[(int64_t)e * W + c]);", "double acc = 0.0;"),
     "weights leak to other ranks": (
         "here ? topk_weights[g * K + k] : 0.0f;", "topk_weights[g * K + k];"),
+    "fp32 combine in descending rank order": (
+        "for (int32_t dst = 0; dst < R; ++dst) {          // ascending destination rank",
+        "for (int32_t dst = R - 1; dst >= 0; --dst) {"),
+    "fp32 combine accumulates in double": (
+        "std::vector<float> sum32(H);", "std::vector<double> sum32(H);"),
+    "fp32 combine adds bias1 before bias0": (
+        "            for (int32_t c = 0; c < H; ++c) sum32[c] = sum32[c] + bf16_bits_to_float(bias0[g * H + c]);\n"
+        "        if (bias1 != nullptr)\n"
+        "            for (int32_t c = 0; c < H; ++c) sum32[c] = sum32[c] + bf16_bits_to_float(bias1[g * H + c]);",
+        "            for (int32_t c = 0; c < H; ++c) sum32[c] = sum32[c] + bf16_bits_to_float(bias1[g * H + c]);\n"
+        "        if (bias1 != nullptr)\n"
+        "            for (int32_t c = 0; c < H; ++c) sum32[c] = sum32[c] + bf16_bits_to_float(bias0[g * H + c]);"),
+    "fp32 combined weights skip the last rank": (
+        "w32 = w32 + recv_topk_weights[(recv_rank_offset[dst] + h) * K + k];",
+        "if (dst < R - 1) w32 = w32 + recv_topk_weights[(recv_rank_offset[dst] + h) * K + k];"),
+    "fp32 ll combine in k order": ("std::sort(visit.begin(), visit.end());", ""),
+    "fp32 ll combine rounds the product": (
+        "chain[c] = std::fma(w32, bf16_bits_to_float(yrow[c]), chain[c]);",
+        "chain[c] = w32 * bf16_bits_to_float(yrow[c]) + chain[c];"),
+    "fp32 lb reduce in descending replica order": (
+        "if (replicas.empty()) continue;                     // untouched",
+        "if (replicas.empty()) continue; std::reverse(replicas.begin(), replicas.end());"),
+    "fp32 lb reduce starts from zero": (
+        "float g32 = bf16_bits_to_float(expert_grads[(int64_t)e * W + c]);", "float g32 = 0.0f;"),
 }
 
 

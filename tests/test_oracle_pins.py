@@ -683,3 +683,198 @@ def test_lb_reduce_rounds_once():
     assert bf16_to_f64(out)[0, 0] == 1.0 + 2.0 ** -6
     with pytest.raises(oracle.OracleError):
         oracle.lb_reduce_grads(r, np.array([0, 9, 0], np.int32), g)
+
+
+# ----------------------------------------------------------------------------
+# fixed-order fp32 reductions (the arithmetic the method performs)
+
+GOLDEN_FP32 = os.path.join(os.path.dirname(__file__), "golden", "fp32_order.txt")
+
+
+def load_golden_fp32():
+    vals = {}
+    with open(GOLDEN_FP32) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *rest = line.split()
+            vals[key] = [int(v, 16) if v.lower().startswith(("0x", "-0x")) else int(v) for v in rest]
+    return vals
+
+
+def _f32(bits):
+    return np.array(bits, np.uint32).view(np.float32)
+
+
+def test_golden_fp32_combine_order():
+    """Ascending destination ranks, then bias0, then bias1, in binary32 from +0:
+    the hand-worked cancellation cases of tests/golden/fp32_order.txt."""
+    g = load_golden_fp32()
+    R, T, H, K = (g[f"combine_{k}"][0] for k in ("R", "T", "H", "K"))
+    h = {"send_head": np.array(g["combine_send_head"], np.int32).reshape(R, T, R),
+         "recv_rank_offset": np.array(g["combine_recv_rank_offset"], np.int64)}
+    y = np.array(g["combine_y"], np.uint16).reshape(-1, H)
+    b0 = np.array(g["combine_bias0"], np.uint16).reshape(R, T, H)
+    b1 = np.array(g["combine_bias1"], np.uint16).reshape(R, T, H)
+    rw = _f32(g["combine_recv_w"]).reshape(-1, K)
+    out, out_w = oracle.combine(y, h, rw, bias0=b0, bias1=b1, fp32=True)
+    assert out.ravel().tolist() == g["combine_out_fp32"]
+    assert out_w.ravel().view(np.uint32).tolist() == g["combine_w_fp32"]
+    out, out_w = oracle.combine(y, h, rw, bias0=b0, bias1=b1)
+    assert out.ravel().tolist() == g["combine_out_exact"]
+    assert out_w.ravel().view(np.uint32).tolist() == g["combine_w_exact"]
+
+
+def test_golden_fp32_ll_combine_order_and_fma():
+    """Ascending expert id (not k), one fused multiply-add per slot."""
+    g = load_golden_fp32()
+    R, E, T, K, Tmax, H = (g[f"ll_{k}"][0] for k in ("R", "E", "T", "K", "TMAX", "H"))
+    topk = np.array(g["ll_topk_idx"], np.int64).reshape(R, T, K)
+    ll = oracle.ll_dispatch(None, topk, E, Tmax, with_rows=False)
+    y = np.array(g["ll_y"], np.uint16).reshape(R, E // R, R * Tmax, H)
+    w = _f32(g["ll_w"]).reshape(R, T, K)
+    out = oracle.ll_combine(y, topk, w, ll["src_info"], ll["layout_range"], E, Tmax, fp32=True)
+    assert out.ravel().tolist() == g["ll_out_fp32"]
+    out = oracle.ll_combine(y, topk, w, ll["src_info"], ll["layout_range"], E, Tmax)
+    assert out.ravel().tolist() == g["ll_out_exact"]
+
+
+def test_golden_fp32_lb_reduce_order():
+    g = load_golden_fp32()
+    m = np.array(g["lb_mapping"], np.int32)
+    grads = np.array(g["lb_grads"], np.uint16).reshape(1, 1)
+    red = np.array(g["lb_redundant"], np.uint16).reshape(-1, 1)
+    assert oracle.lb_reduce_grads(red, m, grads, fp32=True).ravel().tolist() == g["lb_out_fp32"]
+    assert oracle.lb_reduce_grads(red, m, grads).ravel().tolist() == g["lb_out_exact"]
+
+
+def test_fp32_reductions_exact_on_integer_rows():
+    """Small integers and power-of-two weights: every binary32 operation is exact, so
+    the fixed-order results equal the exact sums counted by brute force."""
+    rng = np.random.default_rng(41)
+    R, E, T, K, C, H = 4, 16, 10, 3, 3, 16
+    topk = random_topk(rng, R, E, T, K, mask_p=0.15)
+    w = (2.0 ** rng.integers(-4, 3, (R, T, K))).astype(np.float32)
+    x = f32_to_bf16_torch(rng.integers(-20, 21, (R, T, H)).astype(np.float32))
+    _, _, _, h, (recv_x, _, recv_w) = run_oracle_dispatch(topk, E, C, x, w)
+    b = brute_handle(topk, E, C)
+    yv = rng.integers(-8, 9, size=recv_x.shape).astype(np.float32)
+    b0v = rng.integers(-3, 4, (R, T, H)).astype(np.float32)
+    b1v = rng.integers(-3, 4, (R, T, H)).astype(np.float32)
+    out, out_w = oracle.combine(f32_to_bf16_torch(yv), h, recv_w, bias0=f32_to_bf16_torch(b0v),
+                                bias1=f32_to_bf16_torch(b1v), fp32=True)
+    exp = b0v.astype(np.float64) + b1v
+    for row, (d, s, t) in enumerate(b["triples"]):
+        exp[s, t] += yv[row]
+    np.testing.assert_array_equal(bf16_to_f64(out), exp)
+    np.testing.assert_array_equal(out_w, np.where(topk != -1, w, 0.0).astype(np.float32))
+
+    ll = oracle.ll_dispatch(None, topk, E, T, with_rows=False)
+    L, cap = E // R, R * T
+    ylv = rng.integers(-6, 7, size=(R, L, cap, H)).astype(np.float32)
+    out = oracle.ll_combine(f32_to_bf16_torch(ylv), topk, w, ll["src_info"], ll["layout_range"], E, T,
+                            fp32=True)
+    lists = brute_ll(topk, E)
+    exp = np.zeros((R, T, H))
+    for s in range(R):
+        for t in range(T):
+            for k in range(K):
+                e = int(topk[s, t, k])
+                if e != -1:
+                    exp[s, t] += float(w[s, t, k]) * ylv[e // L, e % L, lists[e].index((s, t))]
+    # every term and partial sum is exact in binary32; only the final bf16 rounding acts
+    np.testing.assert_array_equal(out, f32_to_bf16_torch(exp.astype(np.float32)))
+
+    m = rng.integers(-1, 5, 11).astype(np.int32)
+    gv = rng.integers(-20, 21, (5, 24)).astype(np.float32)
+    rv = rng.integers(-20, 21, (11, 24)).astype(np.float32)
+    out = oracle.lb_reduce_grads(f32_to_bf16_torch(rv), m, f32_to_bf16_torch(gv), fp32=True)
+    exp = gv.astype(np.float64).copy()
+    for i in range(11):
+        if m[i] >= 0:
+            exp[m[i]] += rv[i]
+    np.testing.assert_array_equal(bf16_to_f64(out), exp)
+
+
+def test_fp32_identity_combines_closed_form():
+    """Identity experts: f-fold binary32 sums of one bf16 value are exact, so the
+    fixed-order combine is bf16(f * x); weights 1/8 give bf16(valid/8 * x)."""
+    w_ = synth.WORKLOADS["dsv3"].scaled(num_tokens=40, hidden=64)
+    topk = synth.topk_idx(w_)
+    x = synth.hidden_rows(w_).view(torch.int16).numpy().view(np.uint16)
+    _, _, tin, h, (recv_x, _, _) = run_oracle_dispatch(topk, w_.num_experts, w_.num_channels, x)
+    out, _ = oracle.combine(recv_x, h, fp32=True)
+    fan = tin.sum(-1).astype(np.float32)
+    exp = f32_to_bf16_torch(fan[..., None] * bf16_to_f64(x).astype(np.float32))
+    exp[exp == 0x8000] = 0
+    np.testing.assert_array_equal(out, exp)
+
+    w_ = synth.WORKLOADS["ll"].scaled(num_tokens=12, hidden=32)
+    topk = synth.topk_idx(w_)
+    x = synth.hidden_rows(w_).view(torch.int16).numpy().view(np.uint16)
+    ll = oracle.ll_dispatch(x, topk, w_.num_experts, w_.tmax)
+    out = oracle.ll_combine(ll["packed_recv_x"], topk, np.full(topk.shape, 0.125, np.float32),
+                            ll["src_info"], ll["layout_range"], w_.num_experts, w_.tmax, fp32=True)
+    exp = f32_to_bf16_torch((topk != -1).sum(-1).astype(np.float32)[..., None] / 8
+                            * bf16_to_f64(x).astype(np.float32))
+    np.testing.assert_array_equal(out, exp)
+
+
+def _within_fp32_bound(got, exact, abs_sum, n_terms):
+    """|bf16(fp32 sum) - bf16(exact)| <= half a bf16 ulp of each + n * 2^-24 * sum|terms|:
+    the recursive-summation error bound (each binary32 operation errs by at most a
+    relative 2^-24), plus the two final roundings."""
+    def ulp(v):
+        a = np.abs(v)
+        e = np.maximum(np.floor(np.log2(np.where(a > 0, a, 1.0))), -126.0)
+        return np.where(a > 0, 2.0 ** (e - 7), 2.0 ** -133)
+    g, r = bf16_to_f64(got), bf16_to_f64(exact)
+    tol = 0.5 * ulp(g) + 0.5 * ulp(r) + 1.01 * n_terms * 2.0 ** -24 * bf16_to_f64(abs_sum)
+    return np.abs(g - r) <= tol
+
+
+def test_fp32_reductions_within_the_summation_bound():
+    """On random N(0,1) rows the fixed-order results stay within the binary32
+    summation error bound of the exact sums (any dropped, doubled or misplaced
+    term would break it by a whole term)."""
+    w_ = synth.WORKLOADS["dsv3"].scaled(num_tokens=50, hidden=64)
+    topk = synth.topk_idx(w_)
+    x = synth.hidden_rows(w_).view(torch.int16).numpy().view(np.uint16)
+    _, _, _, h, (recv_x, _, _) = run_oracle_dispatch(topk, w_.num_experts, w_.num_channels, x)
+    y = synth.expert_rows(w_.seed + 1, recv_x.shape[0], w_.hidden).view(torch.int16).numpy().view(np.uint16)
+    b0 = synth.bias_rows(w_, 0).view(torch.int16).numpy().view(np.uint16)
+    got, _ = oracle.combine(y, h, bias0=b0, fp32=True)
+    exact, _ = oracle.combine(y, h, bias0=b0)
+    abs_sum, _ = oracle.combine(y & np.uint16(0x7FFF), h, bias0=b0 & np.uint16(0x7FFF))
+    assert _within_fp32_bound(got, exact, abs_sum, 9).all()
+    # rows whose large terms cancel: the binary32 sums lose low bits, so the
+    # fixed-order result differs from the exact one in places, within the bound
+    yw = synth.cancel_rows(w_.seed + 3, recv_x.shape[0], w_.hidden)
+    got, _ = oracle.combine(yw, h, fp32=True)
+    exact, _ = oracle.combine(yw, h)
+    abs_sum, _ = oracle.combine(yw & np.uint16(0x7FFF), h)
+    assert _within_fp32_bound(got, exact, abs_sum, 8).all()
+    assert (got != exact).mean() > 0.05
+
+    w_ = synth.WORKLOADS["ll"].scaled(num_tokens=20, hidden=64)
+    topk = synth.topk_idx(w_)
+    wts = synth.topk_weights(w_)
+    ll = oracle.ll_dispatch(None, topk, w_.num_experts, w_.tmax, with_rows=False)
+    R, L, cap = w_.num_ranks, w_.local_experts, w_.num_ranks * w_.tmax
+    y = synth.expert_rows(w_.seed + 2, R * L * cap, w_.hidden).view(torch.int16).numpy().view(np.uint16)
+    y = y.reshape(R, L, cap, w_.hidden)
+    args = (ll["src_info"], ll["layout_range"], w_.num_experts, w_.tmax)
+    got = oracle.ll_combine(y, topk, wts, *args, fp32=True)
+    exact = oracle.ll_combine(y, topk, wts, *args)
+    abs_sum = oracle.ll_combine(y & np.uint16(0x7FFF), topk, np.abs(wts), *args)
+    assert _within_fp32_bound(got, exact, abs_sum, w_.topk).all()
+
+    rng = np.random.default_rng(43)
+    m = rng.integers(0, 3, 12).astype(np.int32)
+    g = f32_to_bf16_torch(rng.standard_normal((3, 256)).astype(np.float32))
+    r = f32_to_bf16_torch(rng.standard_normal((12, 256)).astype(np.float32))
+    got = oracle.lb_reduce_grads(r, m, g, fp32=True)
+    exact = oracle.lb_reduce_grads(r, m, g)
+    abs_sum = oracle.lb_reduce_grads(r & np.uint16(0x7FFF), m, g & np.uint16(0x7FFF))
+    assert _within_fp32_bound(got, exact, abs_sum, 13).all()
