@@ -343,7 +343,7 @@ class Path:
         nte = torch.empty((R, E), dtype=torch.int32, device=dev)
         tin = torch.empty((R, T, R), dtype=torch.uint8, device=dev)
         ep.ep_get_dispatch_layout(ctx, topk_d, ntr, nte, tin)
-        N = self.N = int(ntr.sum().item())    # receive rows of this routing (sizing read, untimed)
+        N = self.N = ep.ep_get_num_recv(ctx, ntr, R)[0]   # receive rows of this routing (sizing read, untimed)
         handle = ep.Handle.empty(R, T, C, E // R, N, dev)
         handle.is_token_in_rank = tin
         recv_x = torch.empty((N, H), dtype=torch.bfloat16, device=dev)

@@ -1,8 +1,9 @@
 """Python binding of libep.so: MoE dispatch / combine on virtual EP ranks (B200).
 
-Argument marshalling only.  Every step of the path runs in the library's CUDA
-kernels; torch supplies device memory and the current stream.  The entry points
-keep the C names (``ep_create``, ``ep_get_dispatch_layout``, ``ep_dispatch``,
+Argument marshalling only.  Every step of the path runs in the library (its CUDA
+kernels, and its host code for the receive count); torch supplies device memory
+and the current stream.  The entry points keep the C names (``ep_create``,
+``ep_get_dispatch_layout``, ``ep_get_num_recv``, ``ep_dispatch``,
 ``ep_dispatch_cached``, ``ep_combine``, ``ep_ll_dispatch``, ``ep_ll_combine``,
 ``ep_sync_status``); ``Buffer`` wraps them with output allocation, in the shape
 of DeepEP's ``Buffer`` API.  There is no CPU fallback: if the library is
@@ -73,6 +74,7 @@ _SIGNATURES = {
     "ep_get_dispatch_layout": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "ep_dispatch": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(ep_handle),
                                    _vp, _vp, _vp, _i64, ctypes.POINTER(_i64), _vp, _vp]),
+    "ep_get_num_recv": (ctypes.c_int, [_vp, _vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), _vp, _vp]),
     "ep_dispatch_cached": (ctypes.c_int, [_vp, _vp, ctypes.POINTER(ep_handle), _vp, _i64, _vp, _vp]),
     "ep_combine": (ctypes.c_int, [_vp, _vp, _i64, ctypes.POINTER(ep_handle), _vp, _vp, _vp, _vp,
                                   _vp, _vp, _vp]),
@@ -217,6 +219,16 @@ def ep_dispatch(ctx, x, topk_idx, topk_weights, num_tokens_per_rank, num_tokens_
                               ctypes.byref(n) if want_num_recv else None,
                               _stream(stream), _event(wait_event)), "ep_dispatch", ctx)
     return int(n.value) if want_num_recv else None
+
+
+def ep_get_num_recv(ctx, num_tokens_per_rank, num_ranks: int, stream=None, wait_event=None):
+    """(N, [N_0 .. N_{R-1}]): receive rows in all and per destination rank, from the
+    layout's per-rank counts (one host synchronisation, inside the library)."""
+    n = _i64(-1)
+    per = (_i64 * num_ranks)()
+    _check(load().ep_get_num_recv(ctx, _ptr(num_tokens_per_rank), ctypes.byref(n), per, _stream(stream),
+                                  _event(wait_event)), "ep_get_num_recv", ctx)
+    return int(n.value), [int(v) for v in per]
 
 
 def ep_dispatch_cached(ctx, x, handle: Handle, recv_x, recv_capacity_rows, stream=None,
@@ -382,7 +394,7 @@ class Buffer:
             layout = self.get_dispatch_layout(topk_idx, stream)
         ntr, nte, tin = layout
         if recv_capacity is None:
-            recv_capacity = int(ntr.sum().item())
+            recv_capacity, _ = ep_get_num_recv(self.ctx, ntr, self.R, stream)
         handle = Handle.empty(self.R, self.T, self.C, self.L, recv_capacity, self.device)
         handle.is_token_in_rank = tin
         recv_x = torch.empty((recv_capacity, self.H), dtype=torch.bfloat16, device=self.device)

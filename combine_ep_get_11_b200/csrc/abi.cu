@@ -7,6 +7,7 @@
 //   ep_dispatch            : [layout_kernel] + scan_kernel (call-tagged scan state, nothing to clear)
 //                            [+ one host read of N] + dispatch_kernel<normal> (programmatic
 //                            launch behind the scan)
+//   ep_get_num_recv        : one device-to-host copy of the [R][R] counts + a stream sync
 //   ep_dispatch_cached     : dispatch_kernel<cached>
 //   ep_combine             : combine_kernel
 //   ep_ll_dispatch[_fp8]   : ll_slot_kernel (call-tagged scan state, nothing to clear) +
@@ -528,6 +529,32 @@ int ep_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, const flo
     dp.splits = ep::dispatch_splits(c->H);
     return launch(c, kDispatch, true, s,
                   [&] { return ep::launch_dispatch(ep::kModeNormal, dp, s, num_recv_host == nullptr); });
+}
+
+int ep_get_num_recv(ep_ctx* c, const int32_t* num_tokens_per_rank, int64_t* num_recv_host,
+                    int64_t* num_recv_per_rank_host, ep_stream_t stream, ep_event_t wait_event) {
+    if (c == nullptr) return EP_ERR_INVALID_ARG;
+    if (c->num_shards > 1) return fail(c, EP_ERR_INVALID_ARG, "sharded context: ep_sharded_handle gives the count");
+    if (num_tokens_per_rank == nullptr || num_recv_host == nullptr)
+        return fail(c, EP_ERR_INVALID_ARG, "num_tokens_per_rank / num_recv_host missing");
+    DeviceGuard guard(c->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
+    if (rc != EP_OK) return rc;
+    std::vector<int32_t> ntr((size_t)c->R * c->R);
+    rc = cuda_check(c, cudaMemcpyAsync(ntr.data(), num_tokens_per_rank, sizeof(int32_t) * ntr.size(),
+                                       cudaMemcpyDeviceToHost, s), "read num_tokens_per_rank");
+    if (rc == EP_OK) rc = cuda_check(c, cudaStreamSynchronize(s), "cudaStreamSynchronize");
+    if (rc != EP_OK) return rc;
+    int64_t total = 0;
+    for (int d = 0; d < c->R; ++d) {
+        int64_t nd = 0;
+        for (int src = 0; src < c->R; ++src) nd += ntr[(size_t)src * c->R + d];
+        if (num_recv_per_rank_host != nullptr) num_recv_per_rank_host[d] = nd;
+        total += nd;
+    }
+    *num_recv_host = total;
+    return EP_OK;
 }
 
 int ep_dispatch_cached(ep_ctx* c, const uint16_t* x, const ep_handle* h, uint16_t* recv_x,

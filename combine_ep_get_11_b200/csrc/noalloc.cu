@@ -14,7 +14,10 @@
 // In host code `g_static_scratch` names a host-side stand-in, not device
 // memory; its device address is looked up once per device with
 // cudaGetSymbolAddress (on the first call on that device, with that device
-// current) and passed to the kernel.
+// current) and passed to the kernel.  The looked-up address is kept for the
+// life of the process; a reset of the device's primary context (for example
+// cudaDeviceReset) reloads the module and invalidates it, which the header
+// states as a limit of this entry point.
 
 #include <cstdint>
 #include <mutex>
@@ -69,8 +72,8 @@ extern "C" EP_API int ep_dispatch_handle_static(int32_t num_ranks, int32_t num_e
         handle->recv_rank_offset == nullptr || handle->num_recv_tokens_per_expert == nullptr ||
         num_tokens_per_expert == nullptr)
         return EP_ERR_INVALID_ARG;
-    if (G > 0 && (is_token_in_rank == nullptr || handle->send_head == nullptr))
-        return EP_ERR_INVALID_ARG;
+    if (G > 0 && (is_token_in_rank == nullptr || handle->send_head == nullptr || error_word == nullptr))
+        return EP_ERR_INVALID_ARG;   // (a timeout of the scan's waits is reported through error_word)
     if ((reinterpret_cast<uintptr_t>(is_token_in_rank) & 3u) != 0 ||
         (reinterpret_cast<uintptr_t>(handle->recv_rank_offset) & 7u) != 0)
         return EP_ERR_ALIGNMENT;

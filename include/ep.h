@@ -136,7 +136,17 @@ typedef struct ep_handle_sizes {
  * "Memory Alignment and Validation": rows must be whole 16-byte vectors) and
  * allocates the fixed device workspace (scan state, error word, internal
  * layout arrays).  *out is set only on EP_OK.  Host-only validation runs
- * before any CUDA call, so a bad shape fails without a GPU. */
+ * before any CUDA call, so a bad shape fails without a GPU.
+ *
+ * Concurrency: a context's workspace is shared by its calls -- the handle
+ * scan's ticket counter and status words, the low-latency slot scan's counter,
+ * status words and slot map (which ep_ll_combine reads as a hint), the rank
+ * mask, the internal layout arrays and the error word.  Calls on one context
+ * must therefore be ordered with respect to each other on the GPU: issue them
+ * on one stream (or order the streams with events), and from one host thread
+ * at a time.  Two dispatches of one context running at once would interleave
+ * their tickets and break the scans' call tags.  Different contexts are
+ * independent and may run concurrently. */
 EP_API int ep_create(const ep_config* cfg, ep_ctx** out);
 
 /* Free the context and its workspace ([API] "Explicit Resource Cleanup").
@@ -158,7 +168,7 @@ EP_API const char* ep_last_error(const ep_ctx* ctx);
 
 /* Synchronize `stream`, then return and clear the device error word (EP_OK if
  * no kernel recorded an error since the last call).  The only blocking call
- * besides ep_dispatch with num_recv_host. */
+ * besides ep_get_num_recv, ep_dispatch with num_recv_host and the mask query. */
 EP_API int ep_sync_status(ep_ctx* ctx, ep_stream_t stream);
 /* (When it reports EP_ERR_TIMEOUT it also moves the scans' ticket counters up
  * to the next multiple of their tile counts, so the following calls start from
@@ -227,6 +237,19 @@ EP_API int ep_dispatch(ep_ctx* ctx, const uint16_t* x, const int64_t* topk_idx, 
                 uint16_t* recv_x, int64_t* recv_topk_idx, float* recv_topk_weights,
                 int64_t recv_capacity_rows, int64_t* num_recv_host,
                 ep_stream_t stream, ep_event_t wait_event);
+
+/* Receive counts from a layout ([REUSE] "Performance Contract and Constraints":
+ * the number of tokens each rank receives is only known after the layout, and
+ * learning it costs one CPU-GPU synchronisation).  Copies num_tokens_per_rank
+ * (i32 [R][R], device, from ep_get_dispatch_layout on this stream) to the host,
+ * synchronizes the stream once, and writes
+ *   *num_recv_host               = N = sum over s, d of num_tokens_per_rank[s][d]
+ *   num_recv_per_rank_host[d]    = N_d = sum over s of num_tokens_per_rank[s][d]
+ *                                  (nullable; R int64 values in host memory)
+ * N is the receive capacity ep_dispatch needs.  Not on a sharded context
+ * (ep_sharded_handle returns each GPU's count). */
+EP_API int ep_get_num_recv(ep_ctx* ctx, const int32_t* num_tokens_per_rank, int64_t* num_recv_host,
+                           int64_t* num_recv_per_rank_host, ep_stream_t stream, ep_event_t wait_event);
 
 /* Cached dispatch ([REUSE] "Fast Path Dispatch with Handle Reuse"): scatter
  * new rows x with a handle from an earlier ep_dispatch of the same routing.
@@ -341,14 +364,20 @@ EP_API int ep_lb_reduce_grads(ep_ctx* ctx, const uint16_t* redundant_grads, int6
  *                         channel_prefix_matrix, recv_channel_prefix_matrix,
  *                         recv_rank_offset, num_recv_tokens_per_expert
  *                         (recv_src_idx and is_token_in_rank are not touched)
- *   error_word            nullable device int32, zeroed by the caller; a device
- *                         wait that runs out stores EP_ERR_TIMEOUT there
+ *   error_word            device int32, zeroed by the caller; a device wait that
+ *                         runs out stores EP_ERR_TIMEOUT there.  Required when
+ *                         R * T > 0 (EP_ERR_INVALID_ARG if null): without it a
+ *                         timeout could not be reported
  * Limits as for ep_config; in addition the scratch it needs,
  *   256 + round_up(8 * R * ceil(R*T / 256), 256) + 8 * R * R bytes,
  * must fit in EP_STATIC_SCRATCH_BYTES, or the call returns EP_ERR_CAPACITY
- * before launching anything (R = 32, T = 8192, C = 10 needs about 300 KiB).
+ * before launching anything (R = 32, T = 8192 needs 270,592 bytes = 264.25 KiB;
+ * the channel count does not enter).
  * The first call on a device looks up the array's device address (once, with
- * that device current); make that first call before any stream capture.
+ * that device current); make that first call before any stream capture.  The
+ * address is kept for the life of the process: a cudaDeviceReset (or any reset
+ * of the device's primary context) invalidates it, so do not call this entry
+ * point again after one.
  * Every call shares the one array, and each call clears what must start at
  * zero: calls that may overlap on the GPU (other streams, other threads) race
  * and must be serialised by the caller. */

@@ -21,3 +21,17 @@ def cuda_lib():
     import combine_ep_get_11_b200 as ep
     ep.load()
     return ep
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Combine error statistics of the GPU tests (bit-exact against the oracle's
+    fixed-order fp32 definition; these figures are against the exact sums)."""
+    helpers = sys.modules.get("helpers")
+    rows = getattr(helpers, "COMBINE_REPORT", None) if helpers is not None else None
+    if not rows:
+        return
+    tr = terminalreporter
+    tr.section("combine error against the exact sum (results equal the fixed-order fp32 oracle bit for bit)")
+    for what, st in rows:
+        tr.write_line(f"{what:64s} n={st['n']:>10d}  max_ulp={st['max_ulp']:<7.3g} "
+                      f"max_rel={st['max_rel']:<9.3g} mean_abs={st['mean_abs']:.3e}")

@@ -1,6 +1,8 @@
 """Shared test utilities: bf16 bit views, the combine tolerance, GPU runners."""
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -54,6 +56,57 @@ def assert_combine_close(got: np.ndarray, ref: np.ndarray, abs_sum=None, n_terms
             f"got {bf16_to_f64(got)[tuple(i)]!r} ref {bf16_to_f64(ref)[tuple(i)]!r} tol {tol[tuple(i)]!r}")
     ulps = diff / bf16_ulp(bf16_to_f64(ref))
     return float(ulps.max()) if ulps.size else 0.0, float(diff.mean()) if diff.size else 0.0
+
+
+GOLDEN_FP32 = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "fp32_order.txt")
+
+
+def load_golden_fp32() -> dict:
+    """The hand-worked fp32 summation-order cases (tests/golden/fp32_order.txt):
+    key -> list of ints (hex bit patterns or decimals)."""
+    vals = {}
+    with open(GOLDEN_FP32) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *rest = line.split()
+            vals[key] = [int(v, 16) if v.lower().startswith(("0x", "-0x")) else int(v) for v in rest]
+    return vals
+
+
+# (case, statistics) of every combine checked in this session; printed in the
+# test summary by conftest.py
+COMBINE_REPORT: list = []
+
+
+def combine_stats(got: np.ndarray, exact: np.ndarray) -> dict:
+    """Error of bf16 results against the exact sums rounded to bf16: max error in
+    bf16 ulps (of the exact value), max relative error, mean absolute error."""
+    g, r = bf16_to_f64(got), bf16_to_f64(exact)
+    diff = np.abs(g - r)
+    if diff.size == 0:
+        return {"n": 0, "max_ulp": 0.0, "max_rel": 0.0, "mean_abs": 0.0}
+    nz = r != 0
+    rel = np.where(nz, diff / np.where(nz, np.abs(r), 1.0), np.where(diff > 0, np.inf, 0.0))
+    return {"n": int(diff.size), "max_ulp": float((diff / bf16_ulp(r)).max()),
+            "max_rel": float(rel.max()), "mean_abs": float(diff.mean())}
+
+
+def check_combine(what: str, got: np.ndarray, fp32_ref: np.ndarray, exact: np.ndarray,
+                  abs_sum=None, n_terms: int = 8, one_ulp: bool = False) -> dict:
+    """A GPU combine result: bit-exact against the oracle's fixed-order fp32
+    definition; against the exact sum either within one bf16 ulp (one_ulp: the
+    accuracy bar for N(0,1) rows) or within the binary32 summation bound
+    (abs_sum: rows whose terms cancel).  The error statistics are recorded."""
+    np.testing.assert_array_equal(got, fp32_ref, err_msg=f"{what}: fixed-order fp32 definition")
+    st = combine_stats(got, exact)
+    if one_ulp:
+        assert st["max_ulp"] <= 1.0, f"{what}: {st['max_ulp']} ulp from the exact sum"
+    if abs_sum is not None:
+        assert_combine_close(got, exact, abs_sum, n_terms, what)
+    COMBINE_REPORT.append((what, st))
+    return st
 
 
 class Inputs:

@@ -95,3 +95,4 @@ def test_sharded_null_arguments(lib):
 def test_check_and_test_support_null_arguments(lib):
     assert lib.ep_check_handle(None, None, None, None, None) == 1
     assert lib.ep_test_offset_tickets(None, 1) == 1
+    assert lib.ep_get_num_recv(None, None, None, None, None, None) == 1

@@ -1,8 +1,11 @@
 """GPU parity: the CUDA path (through the C ABI) against the CPU oracle, element by
 element, on seeded inputs small enough for the oracle, spanning several scan tiles,
-several dispatch CTAs and ragged tails.  Integer, index and copied-row outputs must
-be bit-exact; the combines must be within one bf16 ulp plus the fp32 accumulation
-bound (see tests/helpers.py)."""
+several dispatch CTAs and ragged tails.  Everything is bit-exact: integer, index and
+copied-row outputs, and the combines against the oracle's fixed-order fp32
+definition (ascending ranks / expert ids, binary32, one bf16 rounding).  Rows whose
+large terms cancel make the summation order visible; against the exact sums the
+combines are also checked within one bf16 ulp (N(0,1) rows) or the binary32
+summation bound (cancelling rows), and the error statistics are reported."""
 import dataclasses
 
 import numpy as np
@@ -11,7 +14,7 @@ import torch
 
 import oracle
 import synth
-from helpers import Inputs, assert_combine_close, bf16_abs, to_bf16_tensor, u16
+from helpers import Inputs, bf16_abs, check_combine, load_golden_fp32, to_bf16_tensor, u16
 
 pytestmark = pytest.mark.gpu
 
@@ -71,6 +74,8 @@ def test_layout_handle_dispatch_combine(ep, w):
     layout = buf.get_dispatch_layout(inp.topk_d)
     for got, exp, name in zip(layout, (ntr, nte, tin), ("ntr", "nte", "is_token_in_rank")):
         np.testing.assert_array_equal(got.cpu().numpy(), exp, err_msg=name)
+    n_all, n_per = ep.ep_get_num_recv(buf.ctx, layout[0], w.num_ranks)
+    assert n_all == N and n_per == np.diff(h["recv_rank_offset"]).tolist()
 
     recv_x, recv_idx, recv_w, handle = buf.dispatch(inp.x_d, inp.topk_d, inp.weights_d, layout=layout)
     assert buf.sync_status() == 0
@@ -92,9 +97,22 @@ def test_layout_handle_dispatch_combine(ep, w):
     y = synth.expert_rows(w.seed + 1, N, w.hidden)
     b0, b1 = synth.bias_rows(w, 0), synth.bias_rows(w, 1)
     out2, _ = buf.combine(y.cuda(), handle, None, bias=(b0.cuda(), b1.cuda()))
-    ref, _ = oracle.combine(u16(y), h, bias0=u16(b0), bias1=u16(b1))
-    abs_sum, _ = oracle.combine(bf16_abs(u16(y)), h, bias0=bf16_abs(u16(b0)), bias1=bf16_abs(u16(b1)))
-    assert_combine_close(u16(out2), ref, abs_sum, min(w.num_ranks, w.topk) + 2, "combine")
+    bias = dict(bias0=u16(b0), bias1=u16(b1))
+    check_combine(f"{w.name}: combine, N(0,1) rows + 2 biases", u16(out2),
+                  oracle.combine(u16(y), h, fp32=True, **bias)[0], oracle.combine(u16(y), h, **bias)[0],
+                  one_ulp=True)
+    # rows whose large terms cancel (the order of the additions shows), and received
+    # weight rows that cancel too (the weights' sum order shows)
+    yc = synth.cancel_rows(w.seed + 2, N, w.hidden)
+    wc = synth.cancel_rows(w.seed + 3, N, w.topk)
+    wc = ((wc.astype(np.uint32) << 16).view(np.float32)).copy()
+    out3, out3_w = buf.combine(to_bf16_tensor(yc).cuda(), handle, torch.from_numpy(wc).cuda())
+    ref32, ref32_w = oracle.combine(yc, h, wc, fp32=True)
+    exact, _ = oracle.combine(yc, h, wc)
+    abs_sum, _ = oracle.combine(bf16_abs(yc), h)
+    check_combine(f"{w.name}: combine, cancelling rows", u16(out3), ref32, exact, abs_sum,
+                  min(w.num_ranks, w.topk))
+    np.testing.assert_array_equal(out3_w.cpu().numpy(), ref32_w, err_msg="combined weights, fixed order")
 
     # cached dispatch of new rows with the same handle
     x2 = synth.hidden_rows(dataclasses.replace(w, seed=w.seed + 17))
@@ -102,6 +120,71 @@ def test_layout_handle_dispatch_combine(ep, w):
     e_x2, _, _ = oracle.dispatch_rows(u16(x2), inp.topk, None, h, w.num_experts)
     np.testing.assert_array_equal(u16(recv_x2), e_x2)
     assert buf.sync_status() == 0
+    buf.destroy()
+
+
+def test_hand_worked_fp32_cases(ep):
+    """The hand-worked cancellation cases of tests/golden/fp32_order.txt through the C
+    ABI: the combine adds in ascending rank order with the biases last, the
+    low-latency combine is a fused multiply-add chain over ascending expert ids, the
+    gradient reduction adds replicas in ascending order.  The fixtures' columns come
+    first in rows of 8 (whole 16-byte vectors); the other columns are zero."""
+    g = load_golden_fp32()
+    H = 8
+
+    def rows(bits, n, width):
+        a = np.zeros((n, H), np.uint16)
+        a[:, :width] = np.array(bits, np.uint16).reshape(n, width)
+        return a
+
+    # combine: token (0, 0) of three ranks names experts 0, 1, 2 (one per rank)
+    R, T, K, hc = g["combine_R"][0], g["combine_T"][0], 3, g["combine_H"][0]
+    buf = ep.Buffer(R, R, T, H, K, 1)
+    topk = torch.tensor([[[0, 1, 2]], [[-1, -1, -1]], [[-1, -1, -1]]], dtype=torch.int64, device="cuda")
+    x = torch.zeros((R, T, H), dtype=torch.bfloat16, device="cuda")
+    _, _, _, handle = buf.dispatch(x, topk)
+    assert handle.send_head.cpu().numpy().ravel().tolist() == g["combine_send_head"]
+    assert handle.recv_rank_offset.cpu().numpy().tolist() == g["combine_recv_rank_offset"]
+    y = to_bf16_tensor(rows(g["combine_y"], 3, hc)).cuda()
+    b0 = to_bf16_tensor(rows(g["combine_bias0"], R * T, hc).reshape(R, T, H)).cuda()
+    b1 = to_bf16_tensor(rows(g["combine_bias1"], R * T, hc).reshape(R, T, H)).cuda()
+    rw = np.zeros((3, K), np.float32)
+    rw[:, 0] = np.array(g["combine_recv_w"], np.uint32).view(np.float32)
+    out, out_w = buf.combine(y, handle, torch.from_numpy(rw).cuda(), bias=(b0, b1))
+    assert buf.sync_status() == 0
+    got = u16(out).reshape(R * T, H)
+    assert got[:, :hc].ravel().tolist() == g["combine_out_fp32"]
+    assert not got[:, hc:].any()
+    ow = out_w.cpu().numpy().reshape(R * T, K)
+    assert ow[:, 0].view(np.uint32).tolist() == g["combine_w_fp32"]
+    assert not ow[:, 1:].any()
+    buf.destroy()
+
+    # low-latency combine
+    R, E, T, K, Tmax = (g[f"ll_{k}"][0] for k in ("R", "E", "T", "K", "TMAX"))
+    buf = ep.Buffer(R, E, T, H, K, 1, Tmax)
+    topk = torch.tensor(g["ll_topk_idx"], dtype=torch.int64).reshape(R, T, K).cuda()
+    _, count, ll_handle = buf.low_latency_dispatch(torch.zeros((R, T, H), dtype=torch.bfloat16,
+                                                               device="cuda"), topk)
+    assert count.cpu().numpy().ravel().tolist() == [1, 2, 1, 1]
+    y = to_bf16_tensor(rows(g["ll_y"], E * R * Tmax, 1).reshape(R, E // R, R * Tmax, H)).cuda()
+    wts = torch.from_numpy(np.array(g["ll_w"], np.uint32).view(np.float32).reshape(R, T, K)).cuda()
+    out = buf.low_latency_combine(y, topk, wts, ll_handle)
+    assert buf.sync_status() == 0
+    got = u16(out).reshape(R * T, H)
+    assert got[:, 0].tolist() == g["ll_out_fp32"]
+    assert not got[:, 1:].any()
+    buf.destroy()
+
+    # gradient reduction: one expert, two replicas
+    buf = ep.Buffer(1, 1, 1, H, 1, 1)
+    grads = to_bf16_tensor(rows(g["lb_grads"], 1, 1)).cuda()
+    red = to_bf16_tensor(rows(g["lb_redundant"], 2, 1)).cuda()
+    buf.lb_reduce_grads(red, grads, torch.tensor(g["lb_mapping"], dtype=torch.int32, device="cuda"))
+    assert buf.sync_status() == 0
+    got = u16(grads)
+    assert got[:, 0].tolist() == g["lb_out_fp32"]
+    assert not got[:, 1:].any()
     buf.destroy()
 
 
@@ -156,16 +239,22 @@ def test_low_latency(ep, w):
             n = int(ll["packed_recv_count"][d, j])
             np.testing.assert_array_equal(si[d, j, :n], ll["src_info"][d, j, :n])
             np.testing.assert_array_equal(p[d, j, :n], ll["packed_recv_x"][d, j, :n])
-    # identity experts and independent expert outputs
-    for y_u16 in (p, u16(synth.expert_rows(w.seed + 3, R * L * w.tmax * w.num_ranks, w.hidden)
-                         ).reshape(p.shape)):
+    # identity experts and independent expert outputs (softmax weights), then rows
+    # whose large terms cancel with unit weights (the order of the chain shows)
+    rows = R * L * w.tmax * w.num_ranks
+    ones = np.ones_like(inp.weights)
+    for what, y_u16, wts in (
+            ("identity experts", p, inp.weights),
+            ("N(0,1) rows", u16(synth.expert_rows(w.seed + 3, rows, w.hidden)).reshape(p.shape), inp.weights),
+            ("cancelling rows, unit weights", synth.cancel_rows(w.seed + 4, rows, w.hidden).reshape(p.shape),
+             ones)):
         y_d = to_bf16_tensor(y_u16).cuda()
-        out = buf.low_latency_combine(y_d, inp.topk_d, inp.weights_d, (src_info, layout_range))
-        ref = oracle.ll_combine(y_u16, inp.topk, inp.weights, ll["src_info"], ll["layout_range"],
-                                w.num_experts, w.tmax)
-        abs_ref = oracle.ll_combine(bf16_abs(y_u16), inp.topk, np.abs(inp.weights), ll["src_info"],
-                                    ll["layout_range"], w.num_experts, w.tmax)
-        assert_combine_close(u16(out), ref, abs_ref, w.topk, "ll combine")
+        out = buf.low_latency_combine(y_d, inp.topk_d, torch.from_numpy(wts).cuda(), (src_info, layout_range))
+        args = (ll["src_info"], ll["layout_range"], w.num_experts, w.tmax)
+        ref32 = oracle.ll_combine(y_u16, inp.topk, wts, *args, fp32=True)
+        exact = oracle.ll_combine(y_u16, inp.topk, wts, *args)
+        abs_ref = oracle.ll_combine(bf16_abs(y_u16), inp.topk, np.abs(wts), *args)
+        check_combine(f"{w.name}: ll combine, {what}", u16(out), ref32, exact, abs_ref, w.topk)
     assert buf.sync_status() == 0
     buf.destroy()
 
@@ -219,11 +308,11 @@ def test_ll_combine_with_an_older_handle(ep):
     out = buf.low_latency_combine(packed_a, a.topk_d, a.weights_d, handle_a)
     assert buf.sync_status() == 0
     ll = oracle.ll_dispatch(a.x_u16, a.topk, w.num_experts, w.tmax)
-    ref = oracle.ll_combine(ll["packed_recv_x"], a.topk, a.weights, ll["src_info"], ll["layout_range"],
-                            w.num_experts, w.tmax)
-    abs_ref = oracle.ll_combine(bf16_abs(ll["packed_recv_x"]), a.topk, np.abs(a.weights), ll["src_info"],
-                                ll["layout_range"], w.num_experts, w.tmax)
-    assert_combine_close(u16(out), ref, abs_ref, w.topk, "ll combine, older handle")
+    args = (ll["src_info"], ll["layout_range"], w.num_experts, w.tmax)
+    check_combine("ll combine with an older handle", u16(out),
+                  oracle.ll_combine(ll["packed_recv_x"], a.topk, a.weights, *args, fp32=True),
+                  oracle.ll_combine(ll["packed_recv_x"], a.topk, a.weights, *args),
+                  oracle.ll_combine(bf16_abs(ll["packed_recv_x"]), a.topk, np.abs(a.weights), *args), w.topk)
     buf.destroy()
 
 
@@ -472,12 +561,13 @@ def test_low_latency_rank_mask(ep, masked):
     y_u16 = u16(synth.expert_rows(w.seed + 3, p.reshape(-1, w.hidden).shape[0], w.hidden)).reshape(p.shape)
     out = buf.low_latency_combine(to_bf16_tensor(y_u16).cuda(), inp.topk_d, inp.weights_d,
                                   (src_info, layout_range))
-    ref = oracle.ll_combine(y_u16, inp.topk, inp.weights, ll["src_info"], ll["layout_range"], E,
-                            w.tmax, rank_mask=mask)
-    abs_ref = oracle.ll_combine(bf16_abs(y_u16), inp.topk, np.abs(inp.weights), ll["src_info"],
-                                ll["layout_range"], E, w.tmax, rank_mask=mask)
+    args = (ll["src_info"], ll["layout_range"], E, w.tmax)
     got = u16(out)
-    assert_combine_close(got, ref, abs_ref, w.topk, "masked ll combine")
+    check_combine(f"ll combine, ranks {masked} masked", got,
+                  oracle.ll_combine(y_u16, inp.topk, inp.weights, *args, rank_mask=mask, fp32=True),
+                  oracle.ll_combine(y_u16, inp.topk, inp.weights, *args, rank_mask=mask),
+                  oracle.ll_combine(bf16_abs(y_u16), inp.topk, np.abs(inp.weights), *args, rank_mask=mask),
+                  w.topk)
     assert (got[mask.astype(bool)] == 0).all()
 
     (codes, scales), count8, _ = buf.low_latency_dispatch(inp.x_d, inp.topk_d, use_fp8=True)
@@ -523,18 +613,19 @@ def test_load_balance_prefetch_and_reduce(ep, E, W, N):
     assert buf.sync_status() == 0
     np.testing.assert_array_equal(u16(red), oracle.lb_prefetch_weights(u16(ew), mapping, u16(before)))
 
-    grads = synth.expert_rows(93, E, W)
-    rg = synth.expert_rows(94, N, W)
-    g_d = grads.clone().cuda()
-    buf.lb_reduce_grads(rg.cuda(), g_d, torch.from_numpy(mapping).cuda())
-    assert buf.sync_status() == 0
-    ref = oracle.lb_reduce_grads(u16(rg), mapping, u16(grads))
-    abs_ref = oracle.lb_reduce_grads(bf16_abs(u16(rg)), mapping, bf16_abs(u16(grads)))
-    got = u16(g_d)
     n_terms = 1 + int(np.bincount(mapping[mapping >= 0], minlength=E).max())
-    assert_combine_close(got, ref, abs_ref, n_terms, "lb reduce")
     untouched = np.setdiff1d(np.arange(E), mapping)
-    np.testing.assert_array_equal(got[untouched], u16(grads)[untouched])
+    for what, grads, rg in (("N(0,1) rows", u16(synth.expert_rows(93, E, W)), u16(synth.expert_rows(94, N, W))),
+                            ("cancelling rows", synth.cancel_rows(95, E, W), synth.cancel_rows(96, N, W))):
+        g_d = to_bf16_tensor(grads).cuda()
+        buf.lb_reduce_grads(to_bf16_tensor(rg).cuda(), g_d, torch.from_numpy(mapping).cuda())
+        assert buf.sync_status() == 0
+        got = u16(g_d)
+        check_combine(f"lb reduce E{E} W{W} N{N}, {what}", got,
+                      oracle.lb_reduce_grads(rg, mapping, grads, fp32=True),
+                      oracle.lb_reduce_grads(rg, mapping, grads),
+                      oracle.lb_reduce_grads(bf16_abs(rg), mapping, bf16_abs(grads)), n_terms)
+        np.testing.assert_array_equal(got[untouched], grads[untouched])
     buf.destroy()
 
 

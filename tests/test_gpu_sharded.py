@@ -16,7 +16,7 @@ import torch.multiprocessing as mp
 
 import oracle
 import synth
-from helpers import Inputs, assert_combine_close, bf16_abs, to_bf16_tensor, u16
+from helpers import Inputs, bf16_abs, check_combine, to_bf16_tensor, u16
 
 pytestmark = pytest.mark.gpu
 
@@ -114,19 +114,24 @@ def test_local_shards_match_one_gpu(ep, case):
         np.testing.assert_array_equal(u16(outs[s]), e_out[sl[s]])
         np.testing.assert_array_equal(out_ws[s].cpu().numpy(), e_w[sl[s]])
 
-    # independent expert outputs (placed row for row as received) and two bias terms
+    # independent expert outputs (placed row for row as received) and two bias terms:
+    # N(0,1) rows, then rows whose large terms cancel (the rank order shows)
     N = int(h["recv_rank_offset"][-1])
-    y = u16(synth.expert_rows(w.seed + 5, N, H))
     off = h["recv_rank_offset"]
-    for s, b in enumerate(group.shards):
-        for d in range(s * per, (s + 1) * per):
-            b.y[int(dst[d]):int(dst[d] + n[d])].copy_(to_bf16_tensor(y[off[d]:off[d + 1]]).cuda())
     b0, b1 = synth.bias_rows(w, 0), synth.bias_rows(w, 1)
-    group.combine(outs, None, [(b0[q].cuda(), b1[q].cuda()) for q in sl])
-    ref, _ = oracle.combine(y, h, bias0=u16(b0), bias1=u16(b1))
-    abs_sum, _ = oracle.combine(bf16_abs(y), h, bias0=bf16_abs(u16(b0)), bias1=bf16_abs(u16(b1)))
-    for s in range(nshards):
-        assert_combine_close(u16(outs[s]), ref[sl[s]], abs_sum[sl[s]], min(R, K) + 2, f"shard {s}")
+    bias = dict(bias0=u16(b0), bias1=u16(b1))
+    for what, y in (("N(0,1) rows", u16(synth.expert_rows(w.seed + 5, N, H))),
+                    ("cancelling rows", synth.cancel_rows(w.seed + 6, N, H))):
+        for s, b in enumerate(group.shards):
+            for d in range(s * per, (s + 1) * per):
+                b.y[int(dst[d]):int(dst[d] + n[d])].copy_(to_bf16_tensor(y[off[d]:off[d + 1]]).cuda())
+        group.combine(outs, None, [(b0[q].cuda(), b1[q].cuda()) for q in sl])
+        got = np.concatenate([u16(o) for o in outs])
+        check_combine(f"{w.name} over {nshards} shards: combine, {what} + 2 biases", got,
+                      oracle.combine(y, h, fp32=True, **bias)[0], oracle.combine(y, h, **bias)[0],
+                      oracle.combine(bf16_abs(y), h, bias0=bf16_abs(bias["bias0"]),
+                                     bias1=bf16_abs(bias["bias1"]))[0], min(R, K) + 2,
+                      one_ulp=what == "N(0,1) rows")
     for b in group.shards:
         assert b.sync_status() == 0
     group.destroy()

@@ -25,6 +25,7 @@ import torch
 
 import oracle
 import synth
+from helpers import load_golden_fp32
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "tiny_handle.txt")
 
@@ -687,21 +688,6 @@ def test_lb_reduce_rounds_once():
 
 # ----------------------------------------------------------------------------
 # fixed-order fp32 reductions (the arithmetic the method performs)
-
-GOLDEN_FP32 = os.path.join(os.path.dirname(__file__), "golden", "fp32_order.txt")
-
-
-def load_golden_fp32():
-    vals = {}
-    with open(GOLDEN_FP32) as f:
-        for line in f:
-            line = line.strip()
-            if not line or line.startswith("#"):
-                continue
-            key, *rest = line.split()
-            vals[key] = [int(v, 16) if v.lower().startswith(("0x", "-0x")) else int(v) for v in rest]
-    return vals
-
 
 def _f32(bits):
     return np.array(bits, np.uint32).view(np.float32)
