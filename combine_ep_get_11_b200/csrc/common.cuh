@@ -82,6 +82,13 @@ __device__ __forceinline__ uint4 ld_nc_v4(const uint4* p) {
     return v;
 }
 
+// 32 bytes in one load (sm_100 256-bit vector access; p 32-byte aligned).
+__device__ __forceinline__ void ld_nc_v8(const void* p, uint4& a, uint4& b) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(p));
+}
+
 __device__ __forceinline__ void st_stream_v4(uint4* p, const uint4& v) {
     asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
                  "r"(v.z), "r"(v.w)

@@ -1,4 +1,4 @@
-// Dispatch row scatter (normal, cached and low-latency packed).
+// Dispatch row scatter (normal, cached, low-latency packed, and its FP8 form).
 //
 // "DeepEP Buffer Class API ...", section "Dispatch Operation": each token row
 // goes, with its top-k ids and weights, to every rank that owns one of its
@@ -31,7 +31,7 @@
 //     receive buffers of the GPU hosting d (its own memory, or a peer's mapped
 //     into this process), so the exchange happens inside the copy.
 // Per token the HBM traffic is H*2 bytes read + fan-out * H*2 bytes written
-// (fan-out * (H + H/32) bytes in the FP8 packed form).
+// (fan-out * (H + H/32) bytes in the FP8 packed form, ll_fp8_copy_kernel below).
 
 #include <algorithm>
 
@@ -48,6 +48,30 @@ constexpr int kDispatchThreads = 256;
 constexpr int kDispatchWarps = kDispatchThreads / 32;
 constexpr int kVecPerLane = 28;   // 16-byte vectors held per lane per pass
 
+// Packed (low-latency) destination of lane k's top-k slot of token g: the row
+// of its expert's list that the slot scan gave it, or -1 (unused slot, a
+// repeated expert after its first slot, a masked source or destination rank,
+// or a slot past the capacity, which is recorded).
+__device__ __forceinline__ long long packed_row(const DispatchParams& p, long long g, int lane) {
+    long long e = -1;
+    if (lane < p.K) e = p.topk_idx[g * p.K + lane];
+    // slots from or to a masked rank are not sent
+    bool valid = e >= 0 && e < p.E && p.rank_mask[g / p.T] == 0 && p.rank_mask[(int)e / (p.E / p.R)] == 0;
+    for (int k = 0; k < p.K; ++k) {   // a repeated expert is sent once
+        const long long ek = __shfl_sync(kFullMask, e, k);
+        if (k < lane && ek == e) valid = false;
+    }
+    long long row = -1;
+    if (valid) {
+        const int slot = p.slot_map[g * p.K + lane];
+        if (slot >= 0 && slot < p.ll_capacity)
+            row = e * p.ll_capacity + slot;
+        else
+            record_error(p.err, EP_ERR_CAPACITY);
+    }
+    return row;
+}
+
 template <int kMode, int kVec = kVecPerLane>
 __global__ void __launch_bounds__(kDispatchThreads, 2)
 dispatch_kernel(const DispatchParams p) {
@@ -61,7 +85,7 @@ dispatch_kernel(const DispatchParams p) {
     // The normal and packed forms are launched right behind the handle / slot
     // scan and may start before it ends: pull this warp's slice of the source
     // row (never written by the scan) into L2 meanwhile, then wait for the scan.
-    if constexpr (kMode == kModeNormal || kMode == kModeLowLatency || kMode == kModeLowLatencyFp8) {
+    if constexpr (kMode == kModeNormal || kMode == kModeLowLatency) {
         if (lane == 0) {
             const int nv = p.H / 8;
             const int per = ((nv + p.splits - 1) / p.splits + 31) / 32 * 32;
@@ -71,25 +95,10 @@ dispatch_kernel(const DispatchParams p) {
         pdl_wait();
     }
 
-    constexpr bool kPacked = kMode == kModeLowLatency || kMode == kModeLowLatencyFp8;
+    constexpr bool kPacked = kMode == kModeLowLatency;
     long long row = -1;
     if (kPacked) {
-        long long e = -1;
-        if (lane < p.K) e = p.topk_idx[g * p.K + lane];
-        // slots from or to a masked rank are not sent
-        bool valid = e >= 0 && e < p.E && p.rank_mask[g / p.T] == 0 &&
-                     p.rank_mask[(int)e / (p.E / p.R)] == 0;
-        for (int k = 0; k < p.K; ++k) {   // a repeated expert is sent once
-            const long long ek = __shfl_sync(kFullMask, e, k);
-            if (k < lane && ek == e) valid = false;
-        }
-        if (valid) {
-            const int slot = p.slot_map[g * p.K + lane];
-            if (slot >= 0 && slot < p.ll_capacity)
-                row = e * p.ll_capacity + slot;
-            else
-                record_error(p.err, EP_ERR_CAPACITY);
-        }
+        row = packed_row(p, g, lane);
     } else if (lane < p.R) {
         const int h = p.send_head[g * p.R + lane];
         if (h >= 0) {
@@ -143,79 +152,21 @@ dispatch_kernel(const DispatchParams p) {
     const int per = ((nvec + p.splits - 1) / p.splits + 31) / 32 * 32;
     const int lo = part * per, hi = min(nvec, lo + per);
     const uint4* src = reinterpret_cast<const uint4*>(p.x + g * p.H);
-    if (kMode == kModeLowLatencyFp8) {
-        // Each half-warp holds 16 vectors = one 128-channel block: amax by xor
-        // shuffles within the half, scale = amax / 448, codes = E4M3(x * (448 /
-        // amax)) (round to nearest even, saturating), 8 code bytes per lane per
-        // vector.
-        const int nblk = p.H / kFp8Block;
-        for (int c0 = lo; c0 < hi; c0 += 32 * kVec) {
-            uint4 v[kVec];
+    for (int c0 = lo; c0 < hi; c0 += 32 * kVec) {
+        uint4 v[kVec];
 #pragma unroll
-            for (int u = 0; u < kVec; ++u) {
-                const int c = c0 + lane + 32 * u;
-                if (c < hi) v[u] = ld_nc_v4(src + c);
-            }
-#pragma unroll
-            for (int u = 0; u < kVec; ++u) {
-                const int c = c0 + lane + 32 * u;
-                if (c0 + 32 * u >= hi) break;               // warp-uniform
-                float xs[8];
-                xs[0] = bf16_lo(v[u].x); xs[1] = bf16_hi(v[u].x);
-                xs[2] = bf16_lo(v[u].y); xs[3] = bf16_hi(v[u].y);
-                xs[4] = bf16_lo(v[u].z); xs[5] = bf16_hi(v[u].z);
-                xs[6] = bf16_lo(v[u].w); xs[7] = bf16_hi(v[u].w);
-                float m = 0.f;
-                if (c < hi) {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(xs[i]));
-                }
-                m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 8));
-                m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 4));
-                m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 2));
-                m = fmaxf(m, __shfl_xor_sync(kFullMask, m, 1));
-                const float scale = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
-                const float inv = m > 0.f ? __fdiv_rn(448.f, m) : 0.f;
-                uint32_t packed[2];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t word = 0;
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        const float2 q = make_float2(__fmul_rn(xs[4 * h + 2 * i], inv),
-                                                     __fmul_rn(xs[4 * h + 2 * i + 1], inv));
-                        const __nv_fp8x2_storage_t pair = __nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
-                        word |= (uint32_t)pair << (16 * i);
-                    }
-                    packed[h] = word;
-                }
-                if (c < hi) {
-                    const uint2 codes = make_uint2(packed[0], packed[1]);
-                    for (int i = 0; i < f; ++i) {
-                        const long long r = s_rows[warp][i];
-                        *reinterpret_cast<uint2*>(p.recv_fp8 + r * p.H + (long long)c * 8) = codes;
-                        if ((lane & 15) == 0) p.recv_scales[r * nblk + c / 16] = scale;
-                    }
-                }
-            }
+        for (int u = 0; u < kVec; ++u) {
+            const int c = c0 + lane + 32 * u;
+            if (c < hi) v[u] = ld_nc_v4(src + c);
         }
-    } else {
-        for (int c0 = lo; c0 < hi; c0 += 32 * kVec) {
-            uint4 v[kVec];
+        for (int i = 0; i < f; ++i) {
+            uint4* dst = kMode == kModeSharded
+                             ? reinterpret_cast<uint4*>(static_cast<uintptr_t>(s_rows[warp][i]))
+                             : reinterpret_cast<uint4*>(p.recv_x + s_rows[warp][i] * p.H);
 #pragma unroll
             for (int u = 0; u < kVec; ++u) {
                 const int c = c0 + lane + 32 * u;
-                if (c < hi) v[u] = ld_nc_v4(src + c);
-            }
-            for (int i = 0; i < f; ++i) {
-                uint4* dst = kMode == kModeSharded
-                                 ? reinterpret_cast<uint4*>(static_cast<uintptr_t>(s_rows[warp][i]))
-                                 : reinterpret_cast<uint4*>(p.recv_x + s_rows[warp][i] * p.H);
-#pragma unroll
-                for (int u = 0; u < kVec; ++u) {
-                    const int c = c0 + lane + 32 * u;
-                    if (c < hi) st_stream_v4(dst + c, v[u]);
-                }
+                if (c < hi) st_stream_v4(dst + c, v[u]);
             }
         }
     }
@@ -225,11 +176,144 @@ dispatch_kernel(const DispatchParams p) {
     if (kMode == kModeSharded) __threadfence_system();
 }
 
+// ---------------------------------------------------------------- FP8 form
+//
+// "DeepEP Buffer Class API ...", "Low-Latency Inference with FP8": the packed
+// low-latency rows as OCP E4M3 codes with one fp32 scale per token per 128
+// hidden channels (scale = amax / 448, code = E4M3(x * (448 / amax)), each an
+// fp32 operation rounded to nearest even; E4M3 nearest even, saturating; an
+// all-zero block has scale 1 and zero codes).
+//
+// The row is walked in steps of 512 channels: in a step lane l holds channels
+// [16 l, 16 l + 16) (one 32-byte load), so the 8 lanes of an aligned group
+// hold one 128-channel block and find its amax with three xor shuffles.  A
+// lane turns its 16 values into 16 code bytes (one 16-byte store per
+// destination row and step, 512 contiguous bytes per warp instruction).  The
+// block scales of a pass (4 per step) are gathered one per lane, so each
+// destination row gets all of them from a single coalesced store.  A warp
+// holds up to kFp8Steps steps of its row (7: a 7168-wide row in two column
+// slices), loads them all before converting any, then streams the codes
+// to every destination.  Traffic per token: H*2 bytes read, fan-out * (H +
+// H/32) bytes written.
+#ifndef EP_FP8_STEPS
+#define EP_FP8_STEPS 7
+#endif
+constexpr int kFp8Steps = EP_FP8_STEPS;             // 512-channel steps held per warp per pass
+constexpr int kFp8LanesPerBlock = kFp8Block / 16;   // 8 lanes x 16 channels
+static_assert(kFp8LanesPerBlock == 8, "a block is 8 lanes of 16 channels");
+
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+    return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+__global__ void __launch_bounds__(kDispatchThreads, kFp8Steps <= 3 ? 4 : 2)
+ll_fp8_copy_kernel(const DispatchParams p) {
+    __shared__ long long s_rows[kDispatchWarps][32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const long long wid = (long long)blockIdx.x * kDispatchWarps + warp;
+    const long long g = wid / p.splits;          // token
+    const int part = (int)(wid % p.splits);      // column slice of its row (whole steps)
+    if (g >= p.G) return;   // whole warp
+
+    const int nvec = p.H / 8;                    // 16-byte vectors (8 channels) per row
+    const int nstep = (nvec + 63) / 64;
+    const int per = (nstep + p.splits - 1) / p.splits;
+    const int s_lo = part * per, s_hi = min(nstep, s_lo + per);
+    // launched right behind the slot scan: pull this warp's slice of the source
+    // row into L2 while the scan finishes, then wait for it
+    if (lane == 0 && s_lo < s_hi)
+        prefetch_l2(p.x + g * p.H + (long long)s_lo * 512, (uint32_t)(min(nvec, s_hi * 64) - s_lo * 64) * 16u);
+    pdl_wait();
+
+    const long long row = packed_row(p, g, lane);
+    const uint32_t m = __ballot_sync(kFullMask, row >= 0);
+    const int f = __popc(m);
+    if (row >= 0) s_rows[warp][__popc(m & lanemask_lt())] = row;
+    __syncwarp();
+
+    const int nblk = p.H / kFp8Block;
+    const uint4* src = reinterpret_cast<const uint4*>(p.x + g * p.H);
+    for (int st0 = s_lo; st0 < s_hi; st0 += kFp8Steps) {
+        uint4 a[kFp8Steps], b[kFp8Steps];
+#pragma unroll
+        for (int k = 0; k < kFp8Steps; ++k) {
+            const int c = (st0 + k) * 64 + 2 * lane;
+            if (st0 + k < s_hi && c < nvec) ld_nc_v8(src + c, a[k], b[k]);
+        }
+        uint4 codes[kFp8Steps];
+        float scale[kFp8Steps];
+#pragma unroll
+        for (int k = 0; k < kFp8Steps; ++k) {
+            scale[k] = 1.f;
+            if (st0 + k >= s_hi) break;                       // warp-uniform
+            const bool on = (st0 + k) * 64 + 2 * lane < nvec;
+            float xs[16];
+            xs[0] = bf16_lo(a[k].x);  xs[1] = bf16_hi(a[k].x);  xs[2] = bf16_lo(a[k].y);  xs[3] = bf16_hi(a[k].y);
+            xs[4] = bf16_lo(a[k].z);  xs[5] = bf16_hi(a[k].z);  xs[6] = bf16_lo(a[k].w);  xs[7] = bf16_hi(a[k].w);
+            xs[8] = bf16_lo(b[k].x);  xs[9] = bf16_hi(b[k].x);  xs[10] = bf16_lo(b[k].y); xs[11] = bf16_hi(b[k].y);
+            xs[12] = bf16_lo(b[k].z); xs[13] = bf16_hi(b[k].z); xs[14] = bf16_lo(b[k].w); xs[15] = bf16_hi(b[k].w);
+            float amax = 0.f;
+            if (on) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(xs[i]));
+            }
+            amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
+            amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 4));
+            scale[k] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+            const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                w[q] = e4m3x4(__fmul_rn(xs[4 * q], inv), __fmul_rn(xs[4 * q + 1], inv),
+                              __fmul_rn(xs[4 * q + 2], inv), __fmul_rn(xs[4 * q + 3], inv));
+            codes[k] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        // block j of this pass (step j / 4, block j % 4 of the step) -> lane j
+        float my_scale = 1.f;
+#pragma unroll
+        for (int k = 0; k < kFp8Steps; ++k) {
+            const float v = __shfl_sync(kFullMask, scale[k], (lane & 3) * kFp8LanesPerBlock);
+            if ((lane >> 2) == k) my_scale = v;
+        }
+        const int blk0 = st0 * 4;
+        const int nb = min(min(kFp8Steps, s_hi - st0) * 4, nblk - blk0);
+        for (int i = 0; i < f; ++i) {
+            const long long r = s_rows[warp][i];
+            uint8_t* dst = p.recv_fp8 + r * p.H;
+#pragma unroll
+            for (int k = 0; k < kFp8Steps; ++k) {
+                const int c = (st0 + k) * 64 + 2 * lane;
+                if (st0 + k < s_hi && c < nvec) st_stream_v4(reinterpret_cast<uint4*>(dst + (long long)c * 8), codes[k]);
+            }
+            if (lane < nb) __stcs(p.recv_scales + r * nblk + blk0 + lane, my_scale);
+        }
+    }
+}
+
+cudaError_t launch_ll_copy_fp8(DispatchParams p, cudaStream_t stream, bool after_scan) {
+    const int nstep = (p.H / 8 + 63) / 64;
+    p.splits = (nstep + kFp8Steps - 1) / kFp8Steps;   // the fewest column slices with one pass each
+    const long long blocks = (p.G * p.splits + kDispatchWarps - 1) / kDispatchWarps;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(kDispatchThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_scan ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, ll_fp8_copy_kernel, p);
+}
+
 template <int kMode>
 cudaError_t launch_mode(const DispatchParams& p, cudaStream_t stream, bool after_scan) {
     const long long blocks = (p.G * p.splits + kDispatchWarps - 1) / kDispatchWarps;
-    // the FP8 form also keeps the codes and scales live: hold 14 vectors per pass
-    constexpr int kVec = kMode == kModeLowLatencyFp8 ? 14 : kVecPerLane;
+    constexpr int kVec = kVecPerLane;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)blocks);
     cfg.blockDim = dim3(kDispatchThreads);
@@ -251,7 +335,7 @@ cudaError_t launch_dispatch(int mode, const DispatchParams& p, cudaStream_t stre
         case kModeNormal: return launch_mode<kModeNormal>(p, stream, after_scan);
         case kModeCached: return launch_mode<kModeCached>(p, stream, false);
         case kModeLowLatency: return launch_mode<kModeLowLatency>(p, stream, after_scan);
-        case kModeLowLatencyFp8: return launch_mode<kModeLowLatencyFp8>(p, stream, after_scan);
+        case kModeLowLatencyFp8: return launch_ll_copy_fp8(p, stream, after_scan);
         case kModeSharded: return launch_mode<kModeSharded>(p, stream, false);
         default: return cudaErrorInvalidValue;
     }

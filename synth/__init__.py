@@ -167,12 +167,20 @@ def _normal_bf16_rows(seed, kind, shape_per_rank, num_parts, torch_out):
     return torch_out
 
 
-def hidden_rows(w: Workload, pin_memory: bool = False):
-    """x [R, T, H] torch.bfloat16 on the CPU."""
+def hidden_rows(w: Workload, pin_memory: bool = False, ranks=None):
+    """x [R, T, H] torch.bfloat16 on the CPU (ranks: a range of source ranks, whose
+    rows are drawn alone: [len(ranks), T, H], the same values as in the full x)."""
     import torch
-    x = torch.empty((w.num_ranks, w.num_tokens, w.hidden), dtype=torch.bfloat16,
-                    pin_memory=pin_memory)
-    return _normal_bf16_rows(w.seed, _KIND_X, (w.num_tokens, w.hidden), w.num_ranks, x)
+    ranks = range(w.num_ranks) if ranks is None else ranks
+    x = torch.empty((len(ranks), w.num_tokens, w.hidden), dtype=torch.bfloat16, pin_memory=pin_memory)
+
+    def one(i):
+        a = _rng(w.seed, ranks[i], _KIND_X).standard_normal((w.num_tokens, w.hidden), dtype=np.float32)
+        x[i].copy_(torch.from_numpy(a).to(torch.bfloat16))
+
+    with _cf.ThreadPoolExecutor(min(8, max(1, len(ranks)))) as ex:
+        list(ex.map(one, range(len(ranks))))
+    return x
 
 
 def expert_rows(seed: int, num_rows: int, hidden: int, chunk: int = 65536):

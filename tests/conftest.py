@@ -32,6 +32,12 @@ def pytest_terminal_summary(terminalreporter, exitstatus, config):
         return
     tr = terminalreporter
     tr.section("combine error against the exact sum (results equal the fixed-order fp32 oracle bit for bit)")
+    tr.write_line("N(0,1) rows: max error in bf16 ulps of the exact sum, max relative error, mean abs error; "
+                  "cancelling rows: share of elements off the exact sum and the largest error as a "
+                  "fraction of the binary32 summation bound")
     for what, st in rows:
-        tr.write_line(f"{what:64s} n={st['n']:>10d}  max_ulp={st['max_ulp']:<7.3g} "
-                      f"max_rel={st['max_rel']:<9.3g} mean_abs={st['mean_abs']:.3e}")
+        if st.get("cancelling"):
+            tail = f"differ={st['differ']:<8.3g} max_err/bound={st['bound_used']:.3g}"
+        else:
+            tail = f"max_ulp={st['max_ulp']:<5.3g} max_rel={st['max_rel']:<9.3g} mean_abs={st['mean_abs']:.3e}"
+        tr.write_line(f"{what:72s} n={st['n']:>9d}  {tail}")

@@ -46,7 +46,8 @@ def combine_tolerance(ref: np.ndarray, got: np.ndarray, abs_sum: np.ndarray | No
     return np.abs(g - r), tol
 
 
-def assert_combine_close(got: np.ndarray, ref: np.ndarray, abs_sum=None, n_terms=8, what=""):
+def assert_combine_close(got: np.ndarray, ref: np.ndarray, abs_sum=None, n_terms=8, what="",
+                         return_ratio=False):
     diff, tol = combine_tolerance(ref, got, abs_sum, n_terms)
     bad = diff > tol
     if bad.any():
@@ -54,6 +55,8 @@ def assert_combine_close(got: np.ndarray, ref: np.ndarray, abs_sum=None, n_terms
         raise AssertionError(
             f"{what}: {bad.sum()} of {bad.size} elements outside tolerance; first at {tuple(i)}: "
             f"got {bf16_to_f64(got)[tuple(i)]!r} ref {bf16_to_f64(ref)[tuple(i)]!r} tol {tol[tuple(i)]!r}")
+    if return_ratio:
+        return diff, tol
     ulps = diff / bf16_ulp(bf16_to_f64(ref))
     return float(ulps.max()) if ulps.size else 0.0, float(diff.mean()) if diff.size else 0.0
 
@@ -94,17 +97,23 @@ def combine_stats(got: np.ndarray, exact: np.ndarray) -> dict:
 
 
 def check_combine(what: str, got: np.ndarray, fp32_ref: np.ndarray, exact: np.ndarray,
-                  abs_sum=None, n_terms: int = 8, one_ulp: bool = False) -> dict:
+                  abs_sum=None, n_terms: int = 8, one_ulp: bool = False, cancelling: bool = False) -> dict:
     """A GPU combine result: bit-exact against the oracle's fixed-order fp32
     definition; against the exact sum either within one bf16 ulp (one_ulp: the
     accuracy bar for N(0,1) rows) or within the binary32 summation bound
-    (abs_sum: rows whose terms cancel).  The error statistics are recorded."""
+    (abs_sum: a sum whose terms cancel can lose every bit of a small result, so
+    only the bound applies).  The error statistics are recorded for the test
+    summary: in ulps for ordinary rows, as a fraction of the bound for rows whose
+    terms cancel (cancelling)."""
     np.testing.assert_array_equal(got, fp32_ref, err_msg=f"{what}: fixed-order fp32 definition")
     st = combine_stats(got, exact)
+    st["differ"] = float(np.mean(got != exact)) if got.size else 0.0
     if one_ulp:
         assert st["max_ulp"] <= 1.0, f"{what}: {st['max_ulp']} ulp from the exact sum"
     if abs_sum is not None:
-        assert_combine_close(got, exact, abs_sum, n_terms, what)
+        diff, tol = assert_combine_close(got, exact, abs_sum, n_terms, what, return_ratio=True)
+        st["bound_used"] = float((diff / tol).max()) if diff.size else 0.0
+    st["cancelling"] = cancelling
     COMBINE_REPORT.append((what, st))
     return st
 

@@ -118,7 +118,7 @@ def check_normal_full(ep, w, y_source):
         check_combine(f"{w.name} full size: combine, {what}, {tokens.size} sampled tokens", got,
                       oracle.combine(y_u, h, tokens=tokens, fp32=True)[0], oracle.combine(y_u, h, tokens=tokens)[0],
                       oracle.combine(bf16_abs(y_u), h, tokens=tokens)[0], min(w.num_ranks, w.topk),
-                      one_ulp=what == "N(0,1) rows")
+                      one_ulp=what == "N(0,1) rows", cancelling=what == "cancelling rows")
         del y_u
     assert buf.sync_status() == 0
     buf.destroy()
@@ -250,7 +250,7 @@ def test_low_latency_full(ep):
                       got, oracle.ll_combine(y_u, inp.topk, wts, *args, tokens=tok, fp32=True).reshape(got.shape),
                       oracle.ll_combine(y_u, inp.topk, wts, *args, tokens=tok).reshape(got.shape),
                       oracle.ll_combine(bf16_abs(y_u), inp.topk, np.abs(wts), *args, tokens=tok).reshape(got.shape),
-                      K)
+                      K, cancelling=what.startswith("cancelling"))
         del y_u
     del packed
     assert buf.sync_status() == 0

@@ -111,7 +111,7 @@ def test_layout_handle_dispatch_combine(ep, w):
     exact, _ = oracle.combine(yc, h, wc)
     abs_sum, _ = oracle.combine(bf16_abs(yc), h)
     check_combine(f"{w.name}: combine, cancelling rows", u16(out3), ref32, exact, abs_sum,
-                  min(w.num_ranks, w.topk))
+                  min(w.num_ranks, w.topk), cancelling=True)
     np.testing.assert_array_equal(out3_w.cpu().numpy(), ref32_w, err_msg="combined weights, fixed order")
 
     # cached dispatch of new rows with the same handle
@@ -254,7 +254,8 @@ def test_low_latency(ep, w):
         ref32 = oracle.ll_combine(y_u16, inp.topk, wts, *args, fp32=True)
         exact = oracle.ll_combine(y_u16, inp.topk, wts, *args)
         abs_ref = oracle.ll_combine(bf16_abs(y_u16), inp.topk, np.abs(wts), *args)
-        check_combine(f"{w.name}: ll combine, {what}", u16(out), ref32, exact, abs_ref, w.topk)
+        check_combine(f"{w.name}: ll combine, {what}", u16(out), ref32, exact, abs_ref, w.topk,
+                      cancelling=what.startswith("cancelling"))
     assert buf.sync_status() == 0
     buf.destroy()
 
@@ -624,7 +625,8 @@ def test_load_balance_prefetch_and_reduce(ep, E, W, N):
         check_combine(f"lb reduce E{E} W{W} N{N}, {what}", got,
                       oracle.lb_reduce_grads(rg, mapping, grads, fp32=True),
                       oracle.lb_reduce_grads(rg, mapping, grads),
-                      oracle.lb_reduce_grads(bf16_abs(rg), mapping, bf16_abs(grads)), n_terms)
+                      oracle.lb_reduce_grads(bf16_abs(rg), mapping, bf16_abs(grads)), n_terms,
+                      cancelling=what.startswith("cancelling"))
         np.testing.assert_array_equal(got[untouched], grads[untouched])
     buf.destroy()
 

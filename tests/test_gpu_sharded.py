@@ -131,7 +131,7 @@ def test_local_shards_match_one_gpu(ep, case):
                       oracle.combine(y, h, fp32=True, **bias)[0], oracle.combine(y, h, **bias)[0],
                       oracle.combine(bf16_abs(y), h, bias0=bf16_abs(bias["bias0"]),
                                      bias1=bf16_abs(bias["bias1"]))[0], min(R, K) + 2,
-                      one_ulp=what == "N(0,1) rows")
+                      one_ulp=what == "N(0,1) rows", cancelling=what == "cancelling rows")
     for b in group.shards:
         assert b.sync_status() == 0
     group.destroy()
