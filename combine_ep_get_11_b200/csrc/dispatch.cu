@@ -34,6 +34,7 @@
 // (fan-out * (H + H/32) bytes in the FP8 packed form, ll_fp8_copy_kernel below).
 
 #include <algorithm>
+#include <climits>
 
 #include <cuda_fp8.h>
 
@@ -49,21 +50,67 @@ constexpr int kDispatchWarps = kDispatchThreads / 32;
 constexpr int kVecPerLane = 28;   // 16-byte vectors held per lane per pass
 
 // Packed (low-latency) destination of lane k's top-k slot of token g: the row
-// of its expert's list that the slot scan gave it, or -1 (unused slot, a
-// repeated expert after its first slot, a masked source or destination rank,
-// or a slot past the capacity, which is recorded).
-__device__ __forceinline__ long long packed_row(const DispatchParams& p, long long g, int lane) {
+// of its expert's list, or -1 (unused slot, a repeated expert after its first
+// slot, a masked source or destination rank, or a slot past the capacity,
+// which is recorded).  Waits (programmatic dependent launch) for the kernel
+// before it -- the slot scan, or the direct-slot histogram -- before reading
+// what that kernel writes; topk_idx and the rank mask are inputs of the call.
+//
+// Slot scan: the slot is the scan's slot map entry.  Direct slots (sources of
+// at most kLLDirectMaxT tokens): slot = base[s][e] + the tokens t' < t of
+// source s that name e, counted here while the histogram kernel still runs: in
+// chunks of 32 earlier tokens, lane j tests token t' = chunk + j against the
+// token's experts (kept in shared memory, s_ek) and a ballot per expert counts
+// the hits.  The warp of column slice 0 then writes the slot map (a hint for the
+// low-latency combine) and src_info.
+__device__ __forceinline__ long long packed_row(const DispatchParams& p, long long g, int lane, int part,
+                                                int* s_ek) {
+    const int L = p.E / p.R;
+    const int s = (int)(g / p.T), t = (int)(g % p.T);
     long long e = -1;
     if (lane < p.K) e = p.topk_idx[g * p.K + lane];
     // slots from or to a masked rank are not sent
-    bool valid = e >= 0 && e < p.E && p.rank_mask[g / p.T] == 0 && p.rank_mask[(int)e / (p.E / p.R)] == 0;
+    const bool live = e >= 0 && e < p.E && p.rank_mask[s] == 0 && p.rank_mask[(int)e / L] == 0;
+    bool first = live;
     for (int k = 0; k < p.K; ++k) {   // a repeated expert is sent once
         const long long ek = __shfl_sync(kFullMask, e, k);
-        if (k < lane && ek == e) valid = false;
+        if (k < lane && ek == e) first = false;
+    }
+    int within = 0;
+    if (p.ll_base != nullptr) {
+        s_ek[lane] = live ? (int)e : INT_MIN;
+        __syncwarp();
+        for (int c0 = 0; c0 < t; c0 += 32) {
+            const int tp = c0 + lane;        // an earlier token of source s
+            uint32_t hits = 0;               // bit k: token tp names the expert of slot k
+            if (tp < t) {
+                const int64_t* ids = p.topk_idx + ((long long)s * p.T + tp) * p.K;
+                for (int k2 = 0; k2 < p.K; ++k2) {
+                    const int64_t v = ids[k2];
+                    for (int k = 0; k < p.K; ++k) hits |= (uint32_t)(v == (int64_t)s_ek[k]) << k;
+                }
+            }
+            for (int k = 0; k < p.K; ++k) {
+                const int n = __popc(__ballot_sync(kFullMask, (hits >> k) & 1u));
+                if (lane == k) within += n;
+            }
+        }
+    }
+    pdl_wait();
+    int slot = -1;
+    if (live) {
+        if (p.ll_base != nullptr) {
+            slot = p.ll_base[(long long)s * p.E + e] + within;
+            if (part == 0 && slot < p.ll_capacity) {
+                p.slot_map[g * p.K + lane] = slot;
+                if (first) p.ll_src_info[e * p.ll_capacity + slot] = t;
+            }
+        } else if (first) {
+            slot = p.slot_map[g * p.K + lane];
+        }
     }
     long long row = -1;
-    if (valid) {
-        const int slot = p.slot_map[g * p.K + lane];
+    if (first) {
         if (slot >= 0 && slot < p.ll_capacity)
             row = e * p.ll_capacity + slot;
         else
@@ -76,6 +123,7 @@ template <int kMode, int kVec = kVecPerLane>
 __global__ void __launch_bounds__(kDispatchThreads, 2)
 dispatch_kernel(const DispatchParams p) {
     __shared__ long long s_rows[kDispatchWarps][32];
+    __shared__ int s_ek[kMode == kModeLowLatency ? kDispatchWarps : 1][32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const long long wid = (long long)blockIdx.x * kDispatchWarps + warp;
     const long long g = wid / p.splits;          // token
@@ -83,8 +131,9 @@ dispatch_kernel(const DispatchParams p) {
     if (g >= p.G) return;   // whole warp
 
     // The normal and packed forms are launched right behind the handle / slot
-    // scan and may start before it ends: pull this warp's slice of the source
-    // row (never written by the scan) into L2 meanwhile, then wait for the scan.
+    // scan (or the slot histogram) and may start before it ends: pull this
+    // warp's slice of the source row (never written by that kernel) into L2
+    // meanwhile, then wait for it (the packed form inside packed_row).
     if constexpr (kMode == kModeNormal || kMode == kModeLowLatency) {
         if (lane == 0) {
             const int nv = p.H / 8;
@@ -92,13 +141,13 @@ dispatch_kernel(const DispatchParams p) {
             const int lo = part * per, hi = min(nv, lo + per);
             if (lo < hi) prefetch_l2(p.x + g * p.H + (long long)lo * 8, (uint32_t)(hi - lo) * 16u);
         }
-        pdl_wait();
+        if (kMode == kModeNormal) pdl_wait();
     }
 
     constexpr bool kPacked = kMode == kModeLowLatency;
     long long row = -1;
     if (kPacked) {
-        row = packed_row(p, g, lane);
+        row = packed_row(p, g, lane, part, s_ek[kPacked ? warp : 0]);
     } else if (lane < p.R) {
         const int h = p.send_head[g * p.R + lane];
         if (h >= 0) {
@@ -191,12 +240,14 @@ dispatch_kernel(const DispatchParams p) {
 // destination row and step, 512 contiguous bytes per warp instruction).  The
 // block scales of a pass (4 per step) are gathered one per lane, so each
 // destination row gets all of them from a single coalesced store.  A warp
-// holds up to kFp8Steps steps of its row (7: a 7168-wide row in two column
-// slices), loads them all before converting any, then streams the codes
-// to every destination.  Traffic per token: H*2 bytes read, fan-out * (H +
+// holds up to kFp8Steps steps of its row (2: a 7168-wide row in seven column
+// slices, 64 registers, four blocks per SM; measured on B200 against 3, 4 and 7
+// steps per warp: 29.3 vs 30.0, 33.3 and 31.6 us on the low-latency shape),
+// loads them all before converting any, then streams the codes to every
+// destination.  Traffic per token: H*2 bytes read, fan-out * (H +
 // H/32) bytes written.
 #ifndef EP_FP8_STEPS
-#define EP_FP8_STEPS 7
+#define EP_FP8_STEPS 2
 #endif
 constexpr int kFp8Steps = EP_FP8_STEPS;             // 512-channel steps held per warp per pass
 constexpr int kFp8LanesPerBlock = kFp8Block / 16;   // 8 lanes x 16 channels
@@ -211,6 +262,7 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
 __global__ void __launch_bounds__(kDispatchThreads, kFp8Steps <= 3 ? 4 : 2)
 ll_fp8_copy_kernel(const DispatchParams p) {
     __shared__ long long s_rows[kDispatchWarps][32];
+    __shared__ int s_ek[kDispatchWarps][32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const long long wid = (long long)blockIdx.x * kDispatchWarps + warp;
     const long long g = wid / p.splits;          // token
@@ -221,13 +273,12 @@ ll_fp8_copy_kernel(const DispatchParams p) {
     const int nstep = (nvec + 63) / 64;
     const int per = (nstep + p.splits - 1) / p.splits;
     const int s_lo = part * per, s_hi = min(nstep, s_lo + per);
-    // launched right behind the slot scan: pull this warp's slice of the source
-    // row into L2 while the scan finishes, then wait for it
+    // launched right behind the slot scan (or histogram): pull this warp's slice
+    // of the source row into L2 while it finishes (packed_row waits for it)
     if (lane == 0 && s_lo < s_hi)
         prefetch_l2(p.x + g * p.H + (long long)s_lo * 512, (uint32_t)(min(nvec, s_hi * 64) - s_lo * 64) * 16u);
-    pdl_wait();
 
-    const long long row = packed_row(p, g, lane);
+    const long long row = packed_row(p, g, lane, part, s_ek[warp]);
     const uint32_t m = __ballot_sync(kFullMask, row >= 0);
     const int f = __popc(m);
     if (row >= 0) s_rows[warp][__popc(m & lanemask_lt())] = row;
@@ -293,9 +344,15 @@ ll_fp8_copy_kernel(const DispatchParams p) {
     }
 }
 
+#ifndef EP_FP8_SPLITS
+#define EP_FP8_SPLITS 0
+#endif
+
 cudaError_t launch_ll_copy_fp8(DispatchParams p, cudaStream_t stream, bool after_scan) {
     const int nstep = (p.H / 8 + 63) / 64;
-    p.splits = (nstep + kFp8Steps - 1) / kFp8Steps;   // the fewest column slices with one pass each
+    // column slices per row: the fewest with one pass each (EP_FP8_SPLITS 0), or a
+    // fixed count whose warps loop over several passes
+    p.splits = EP_FP8_SPLITS > 0 ? min(EP_FP8_SPLITS, nstep) : (nstep + kFp8Steps - 1) / kFp8Steps;
     const long long blocks = (p.G * p.splits + kDispatchWarps - 1) / kDispatchWarps;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)blocks);

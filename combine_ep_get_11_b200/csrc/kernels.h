@@ -74,9 +74,12 @@ struct DispatchParams {
     float* recv_topk_weights;          // [cap][K] or null
     int* recv_src_idx;                 // [cap] or null
     // low latency
-    const int* slot_map;               // [G][K]
+    int* slot_map;                     // [G][K]: read (slot scan) or written (direct slots)
     const int* rank_mask;              // [R], 0 active / 1 masked
     int64_t ll_capacity;               // R * Tmax slots per expert
+    const int* ll_base;                // [R][E] direct slots: first slot of source s in expert e's
+                                       // list (from ll_hist_kernel), or null: slots from slot_map
+    int* ll_src_info;                  // [E][ll_capacity] direct slots: written by the copy
     uint16_t* recv_x;                  // normal/cached: [cap][H]; LL: [E][ll_cap][H]
     // low latency, FP8 form (recv_x unused)
     uint8_t* recv_fp8;                 // [E][ll_cap][H] E4M3 codes
@@ -162,6 +165,27 @@ struct LLCountParams {
 };
 constexpr int kLLTile = 256;   // tokens per tile == threads per block
 cudaError_t launch_ll_count(const LLCountParams& p, cudaStream_t stream);
+
+// Direct low-latency slots, for sources of at most kLLDirectMaxT tokens (decode
+// batches): slot(s, t, e) = base[s][e] + (tokens t' < t of source s naming e).
+// ll_hist_kernel (one block per source) counts the tokens of each source that
+// name each expert; its last block turns the counts into base, layout_range and
+// the per-expert counts.  The copy kernel, launched behind it, counts the
+// earlier tokens of its own source while the histogram runs, then adds base.
+// Nothing waits on another block, so nothing needs a bounded wait.
+struct LLHistParams {
+    const int64_t* topk_idx;   // [G][K]
+    const int* rank_mask;      // [R]
+    int* cnt;                  // [R][E] tokens of source s naming e (each call overwrites)
+    int* base;                 // [R][E] first slot of source s in expert e's list
+    int* layout_range;         // [E][R][2]
+    int* packed_recv_count;    // [E]
+    unsigned int* done;        // blocks finished; the last block resets it to 0
+    int* err;
+    int R, E, T, K;
+};
+constexpr int kLLDirectMaxT = 256;   // == kLLTile: one block per source
+cudaError_t launch_ll_hist(const LLHistParams& p, cudaStream_t stream);
 cudaError_t ll_prepare(int E);   // once per device: shared-memory opt-in
 
 struct LLCombineParams {

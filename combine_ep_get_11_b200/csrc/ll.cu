@@ -29,6 +29,9 @@ namespace ep {
 
 namespace {
 
+#ifndef EP_LL_COMBINE_PREFETCH
+#define EP_LL_COMBINE_PREFETCH 0
+#endif
 constexpr int kLLCombineThreads = 256;
 constexpr int kLLCombineWarps = kLLCombineThreads / 32;
 constexpr int kLLRowsPerGroup = 8;
@@ -225,6 +228,65 @@ ll_slot_kernel(const LLCountParams p) {
     }
 }
 
+// Direct slots, histogram part: block s counts, per expert, the tokens of
+// source s that name it (a token naming an expert twice counts once; tokens of
+// a masked source and experts of a masked rank count nothing) and stores the
+// counts; the last block to finish turns every expert's column of counts into
+// its exclusive prefix over sources (base, layout_range) and the total
+// (packed_recv_count), then resets the finish counter for the next call.
+template <int kMaxK>
+__global__ void __launch_bounds__(kLLTile)
+ll_hist_kernel(const LLHistParams p) {
+    extern __shared__ int h_cnt[];   // [E]
+    __shared__ bool s_last;
+    pdl_launch_dependents();         // the copy may start counting its source's earlier tokens
+    const int s = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+    const int E = p.E, L = p.E / p.R;
+    for (int e = tid; e < E; e += kLLTile) h_cnt[e] = 0;
+    const uint32_t mbits = __ballot_sync(kFullMask, lane < p.R && p.rank_mask[lane] != 0);
+    __syncthreads();
+    if (tid < p.T) {
+        const long long g = (long long)s * p.T + tid;
+        const bool src_live = ((mbits >> s) & 1u) == 0;
+        int ids[kMaxK];
+        bool bad = false;
+#pragma unroll
+        for (int k = 0; k < kMaxK; ++k) {
+            const int64_t e = k < p.K ? __ldg(p.topk_idx + g * p.K + k) : -1;
+            bad |= e < -1 || e >= E;
+            ids[k] = (e >= 0 && e < E && src_live && ((mbits >> ((int)e / L)) & 1u) == 0) ? (int)e : -1;
+        }
+        if (bad) record_error(p.err, EP_ERR_BAD_TOPK);
+#pragma unroll
+        for (int k = 0; k < kMaxK; ++k) {
+            bool first = ids[k] >= 0;
+#pragma unroll
+            for (int k2 = 0; k2 < k; ++k2) first = first && ids[k2] != ids[k];
+            if (first) atomicAdd(&h_cnt[ids[k]], 1);
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kLLTile) p.cnt[(size_t)s * E + e] = h_cnt[e];
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(p.done, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int e = tid; e < E; e += kLLTile) {
+        int run = 0;
+        for (int src = 0; src < p.R; ++src) {
+            const int c = __ldcg(p.cnt + (size_t)src * E + e);
+            p.base[(size_t)src * E + e] = run;
+            p.layout_range[((size_t)e * p.R + src) * 2 + 0] = run;
+            p.layout_range[((size_t)e * p.R + src) * 2 + 1] = c;
+            run += c;
+        }
+        p.packed_recv_count[e] = run;
+    }
+    if (tid == 0) *p.done = 0u;
+}
+
 __device__ __forceinline__ void fma_bf16x8(float* acc, float w, const uint4& v) {
     acc[0] = __fmaf_rn(w, bf16_lo(v.x), acc[0]);
     acc[1] = __fmaf_rn(w, bf16_hi(v.x), acc[1]);
@@ -306,7 +368,16 @@ ll_combine_kernel(const LLCombineParams p) {
         uint4* out = reinterpret_cast<uint4*>(p.out_x + g * p.H);
         const int per = ((nvec + p.splits - 1) / p.splits + 31) / 32 * 32;
         const int clo = part * per, chi = min(nvec, clo + per);
+#if EP_LL_COMBINE_PREFETCH
+        // lane i asks for the next column slab of row i ahead of its loads (a bulk L2 prefetch)
+        const uint4* pf_row = lane < nv ? reinterpret_cast<const uint4*>(p.y + s_rows[warp][lane] * p.H) : nullptr;
+        if (pf_row != nullptr && clo < chi) prefetch_l2(pf_row + clo, (uint32_t)min(32 * U, chi - clo) * 16u);
+#endif
         for (int c0 = clo; c0 < chi; c0 += 32 * U) {
+#if EP_LL_COMBINE_PREFETCH
+            const int nxt = c0 + 32 * U;
+            if (pf_row != nullptr && nxt < chi) prefetch_l2(pf_row + nxt, (uint32_t)min(32 * U, chi - nxt) * 16u);
+#endif
             float acc[U][8];
 #pragma unroll
             for (int u = 0; u < U; ++u)
@@ -357,6 +428,18 @@ __global__ void set_mask_kernel(int* rank_mask, int rank, int value) { rank_mask
 
 cudaError_t launch_set_mask(int* rank_mask, int rank, int value, cudaStream_t stream) {
     set_mask_kernel<<<1, 1, 0, stream>>>(rank_mask, rank, value);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ll_hist(const LLHistParams& p, cudaStream_t stream) {
+    if (p.R == 0 || p.E == 0) return cudaSuccess;
+    const size_t smem = (size_t)p.E * sizeof(int);
+    if (p.K <= 8)
+        ll_hist_kernel<8><<<p.R, kLLTile, smem, stream>>>(p);
+    else if (p.K <= 16)
+        ll_hist_kernel<16><<<p.R, kLLTile, smem, stream>>>(p);
+    else
+        ll_hist_kernel<32><<<p.R, kLLTile, smem, stream>>>(p);
     return cudaGetLastError();
 }
 

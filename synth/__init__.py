@@ -54,7 +54,7 @@ class Workload:
     num_tokens: int         # T (per rank)
     hidden: int             # H
     topk: int               # K
-    routing: str            # uniform | uniform_masked | zipf | group_limited
+    routing: str            # uniform | uniform_masked | uniform_repeats | zipf | group_limited
     seed: int
     num_channels: int = 10  # C
     max_tokens_per_rank: int = 0   # Tmax for the low-latency path (0 -> T)
@@ -123,6 +123,9 @@ def topk_idx(w: Workload) -> np.ndarray:
         rng = _rng(w.seed, s, _KIND_ROUTING)
         if w.routing in ("uniform", "uniform_masked"):
             out[s] = _distinct_uniform(rng, T, E, K)
+        elif w.routing == "uniform_repeats":
+            # K independent uniform draws: a token may name an expert twice
+            out[s] = rng.integers(0, E, (T, K))
         elif w.routing == "zipf":
             # Sequential draws without replacement, each proportional to the
             # remaining popularity mass, are the top-K of log p + Gumbel noise.

@@ -35,6 +35,8 @@ CASES = [
     synth.Workload("H32768", 2, 4, 20, 32768, 2, "uniform", 88, num_channels=3),
     synth.Workload("H8", 2, 4, 33, 8, 2, "uniform_masked", 87, num_channels=2, mask_prob=0.2),
     synth.Workload("E4096", 8, 4096, 50, 16, 8, "uniform", 86, num_channels=4),
+    # a token may name an expert twice (counted twice per expert, once per rank)
+    synth.Workload("repeats", 4, 16, 70, 64, 5, "uniform_repeats", 76, num_channels=3, mask_prob=0.1),
 ]
 
 
@@ -217,8 +219,13 @@ LL_CASES = [
     synth.Workload("ll-big", 32, 256, 160, 64, 8, "uniform", 94),
     synth.Workload("ll-k20", 4, 64, 50, 32, 20, "uniform_masked", 93, mask_prob=0.1),
     synth.Workload("ll-E4096", 8, 4096, 40, 128, 8, "uniform", 92),
-    # sources longer than one 256-token slot tile (3 tiles each, the last one ragged)
+    # sources longer than one 256-token slot tile (3 tiles each, the last one ragged):
+    # the lookback scan; at most 256 tokens per source: direct slots
     synth.Workload("ll-T600", 4, 32, 600, 64, 4, "uniform_masked", 91, mask_prob=0.1),
+    synth.Workload("ll-T256", 4, 32, 256, 128, 8, "uniform_masked", 79, mask_prob=0.05),
+    synth.Workload("ll-T257", 4, 32, 257, 128, 8, "uniform_masked", 78, mask_prob=0.05),
+    # repeated experts within a token (a token counts once per expert)
+    synth.Workload("ll-rep-experts", 4, 8, 90, 128, 6, "uniform_repeats", 77, mask_prob=0.1),
 ]
 
 
@@ -278,22 +285,27 @@ def test_repeated_calls_on_one_context(ep):
     assert buf.sync_status() == 0
     buf.destroy()
 
-    base = synth.Workload("ll-rep", 8, 64, 300, 64, 6, "uniform_masked", 84, mask_prob=0.1)
-    buf = make_buffer(ep, base)
-    for seed in (base.seed, base.seed + 1, base.seed, base.seed + 2):
-        w = dataclasses.replace(base, seed=seed)
-        inp = Inputs(w)
-        packed, count, (src_info, layout_range) = buf.low_latency_dispatch(inp.x_d, inp.topk_d)
-        ll = oracle.ll_dispatch(inp.x_u16, inp.topk, w.num_experts, w.tmax)
-        np.testing.assert_array_equal(count.cpu().numpy(), ll["packed_recv_count"])
-        np.testing.assert_array_equal(layout_range.cpu().numpy(), ll["layout_range"])
-        si = src_info.cpu().numpy()
-        for d in range(w.num_ranks):
-            for j in range(w.local_experts):
-                n = int(ll["packed_recv_count"][d, j])
-                np.testing.assert_array_equal(si[d, j, :n], ll["src_info"][d, j, :n])
-    assert buf.sync_status() == 0
-    buf.destroy()
+    # low-latency slots: the lookback scan (300 tokens per source) and the direct
+    # slots (200 tokens per source: per-source histogram, whose finish counter must
+    # be back at zero for every next call)
+    for base in (synth.Workload("ll-rep", 8, 64, 300, 64, 6, "uniform_masked", 84, mask_prob=0.1),
+                 synth.Workload("ll-rep-direct", 8, 64, 200, 64, 6, "uniform_masked", 85, mask_prob=0.1)):
+        buf = make_buffer(ep, base)
+        for seed in (base.seed, base.seed + 1, base.seed, base.seed + 2):
+            w = dataclasses.replace(base, seed=seed)
+            inp = Inputs(w)
+            packed, count, (src_info, layout_range) = buf.low_latency_dispatch(inp.x_d, inp.topk_d)
+            ll = oracle.ll_dispatch(inp.x_u16, inp.topk, w.num_experts, w.tmax)
+            np.testing.assert_array_equal(count.cpu().numpy(), ll["packed_recv_count"])
+            np.testing.assert_array_equal(layout_range.cpu().numpy(), ll["layout_range"])
+            si, pk = src_info.cpu().numpy(), u16(packed)
+            for d in range(w.num_ranks):
+                for j in range(w.local_experts):
+                    n = int(ll["packed_recv_count"][d, j])
+                    np.testing.assert_array_equal(si[d, j, :n], ll["src_info"][d, j, :n])
+                    np.testing.assert_array_equal(pk[d, j, :n], ll["packed_recv_x"][d, j, :n])
+        assert buf.sync_status() == 0
+        buf.destroy()
 
 
 def test_ll_combine_with_an_older_handle(ep):
@@ -525,7 +537,7 @@ def test_low_latency_fp8(ep, w):
 
 
 def test_low_latency_fp8_rejects_unaligned_hidden(ep):
-    w = LL_CASES[-3]            # hidden 40: not a multiple of 128
+    w = next(c for c in LL_CASES if c.name == "ll-odd")      # hidden 40: not a multiple of 128
     assert w.hidden % 128 != 0
     inp = Inputs(w)
     buf = make_buffer(ep, w)
