@@ -10,12 +10,12 @@
 //   ep_get_num_recv        : one device-to-host copy of the [R][R] counts + a stream sync
 //   ep_dispatch_cached     : dispatch_kernel<cached>
 //   ep_combine             : combine_kernel
-//   ep_ll_dispatch[_fp8]   : T <= 256: ll_hist_kernel (per-source counts; its last block
-//                            writes the per-source bases) + dispatch_kernel<packed> /
-//                            ll_fp8_copy_kernel (programmatic launch behind it; each token's
-//                            earlier tokens counted while the histogram runs);
-//                            larger T: ll_slot_kernel (call-tagged scan state, nothing to
-//                            clear) + the same copy kernels reading its slot map
+//   ep_ll_dispatch[_fp8]   : T <= 256: ll_rank_kernel (per-source counts and each token's
+//                            rank within its source) + dispatch_kernel<packed> /
+//                            ll_fp8_copy_kernel (programmatic launch behind it; they add
+//                            the earlier sources' counts and write src_info, layout_range,
+//                            the counts); larger T: ll_slot_kernel (call-tagged scan state,
+//                            nothing to clear) + the same copy kernels reading its slot map
 //   ep_ll_combine          : ll_combine_kernel
 //   ep_lb_prefetch_weights : lb_prefetch_kernel;  ep_lb_reduce_grads : lb_reduce_kernel
 //   ep_sharded_handle      : shard_offsets_kernel + scan_kernel (with the shard's base)
@@ -64,8 +64,7 @@ struct ep_ctx {
     int ll_tiles_per_src;
     int ll_tiles;
     int* ll_cnt;                // [R][E] direct low-latency slots: tokens of source s naming e
-    int* ll_base;               // [R][E] direct low-latency slots: first slot of source s per expert
-    unsigned int* ll_done;      // direct low-latency slots: histogram blocks finished (0 between calls)
+    int* ll_within;             // [G][K] direct low-latency slots: rank of a token among its source's
     int* rank_mask;             // [R] low-latency rank mask (0 active, 1 masked)
     int* shard_base;            // [R] tokens of earlier shards per destination (sharded scan base)
     char last_error[256];
@@ -269,8 +268,7 @@ int create_impl(const ep_config* cfg, int num_shards, int shard, ep_ctx** out) {
     const size_t off_llb = off;            off += align256((size_t)c->R * c->E * sizeof(unsigned long long));
     const size_t off_llc = off;            off += align256(sizeof(unsigned long long));
     const size_t off_llh = off;            off += align256((size_t)c->R * c->E * sizeof(int));
-    const size_t off_llbase = off;         off += align256((size_t)c->R * c->E * sizeof(int));
-    const size_t off_lldone = off;         off += align256(sizeof(unsigned int));
+    const size_t off_llwithin = off;       off += align256((size_t)c->G * c->K * sizeof(int));
     const size_t off_mask = off;           off += align256((size_t)c->R * sizeof(int));
     const size_t off_sbase = off;          off += align256((size_t)c->R * sizeof(int));
     c->ws_bytes = off;
@@ -289,8 +287,7 @@ int create_impl(const ep_config* cfg, int num_shards, int shard, ep_ctx** out) {
     c->ll_src_begin = reinterpret_cast<unsigned long long*>(c->ws + off_llb);
     c->ll_ticket = reinterpret_cast<unsigned long long*>(c->ws + off_llc);
     c->ll_cnt = reinterpret_cast<int*>(c->ws + off_llh);
-    c->ll_base = reinterpret_cast<int*>(c->ws + off_llbase);
-    c->ll_done = reinterpret_cast<unsigned int*>(c->ws + off_lldone);   // zeroed below
+    c->ll_within = reinterpret_cast<int*>(c->ws + off_llwithin);
     c->rank_mask = reinterpret_cast<int*>(c->ws + off_mask);   // zeroed below: every rank active
     c->shard_base = reinterpret_cast<int*>(c->ws + off_sbase);
     if (cudaMemset(c->ws, 0, c->ws_bytes) != cudaSuccess) rc = EP_ERR_CUDA;
@@ -662,13 +659,12 @@ int ll_dispatch_impl(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint
         if (e == cudaSuccess) e = cudaMemsetAsync(layout_range, 0, sizeof(int) * 2 * (size_t)c->E * c->R, s);
         return cuda_check(c, e, "zero low-latency counts");
     }
-    // slots: direct (a per-source histogram; the copy counts each token's earlier
-    // tokens) for sources of up to kLLDirectMaxT tokens, else the lookback scan
+    // slots: direct (per-source ranking; the copy adds the earlier sources' counts)
+    // for sources of up to kLLDirectMaxT tokens, else the lookback scan
     const bool direct = c->T <= ep::kLLDirectMaxT;
     if (direct) {
-        ep::LLHistParams hp{topk_idx, c->rank_mask, c->ll_cnt, c->ll_base, layout_range, packed_recv_count,
-                            c->ll_done, c->err, c->R, c->E, c->T, c->K};
-        rc = launch(c, kLLCount, true, s, [&] { return ep::launch_ll_hist(hp, s); });
+        ep::LLRankParams rp{topk_idx, c->rank_mask, c->ll_cnt, c->ll_within, c->err, c->R, c->E, c->T, c->K};
+        rc = launch(c, kLLCount, true, s, [&] { return ep::launch_ll_rank(rp, s); });
     } else {
         ep::LLCountParams cp{topk_idx, c->slot_map, packed_recv_count, src_info, layout_range,
                              c->ll_status, c->ll_src_begin, c->ll_ticket,
@@ -681,8 +677,11 @@ int ll_dispatch_impl(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint
     dp.x = x;
     dp.topk_idx = topk_idx;
     dp.slot_map = c->slot_map;
-    dp.ll_base = direct ? c->ll_base : nullptr;
+    dp.ll_cnt = direct ? c->ll_cnt : nullptr;
+    dp.ll_within = c->ll_within;
     dp.ll_src_info = src_info;
+    dp.ll_layout_range = layout_range;
+    dp.ll_count = packed_recv_count;
     dp.rank_mask = c->rank_mask;
     dp.ll_capacity = c->ll_cap;
     dp.recv_x = packed_recv_x;

@@ -34,7 +34,6 @@
 // (fan-out * (H + H/32) bytes in the FP8 packed form, ll_fp8_copy_kernel below).
 
 #include <algorithm>
-#include <climits>
 
 #include <cuda_fp8.h>
 
@@ -53,18 +52,16 @@ constexpr int kVecPerLane = 28;   // 16-byte vectors held per lane per pass
 // of its expert's list, or -1 (unused slot, a repeated expert after its first
 // slot, a masked source or destination rank, or a slot past the capacity,
 // which is recorded).  Waits (programmatic dependent launch) for the kernel
-// before it -- the slot scan, or the direct-slot histogram -- before reading
-// what that kernel writes; topk_idx and the rank mask are inputs of the call.
+// before it -- the slot scan, or the direct-slot ranking -- before reading what
+// that kernel writes; topk_idx and the rank mask are inputs of the call.
 //
 // Slot scan: the slot is the scan's slot map entry.  Direct slots (sources of
-// at most kLLDirectMaxT tokens): slot = base[s][e] + the tokens t' < t of
-// source s that name e, counted here while the histogram kernel still runs: in
-// chunks of 32 earlier tokens, lane j tests token t' = chunk + j against the
-// token's experts (kept in shared memory, s_ek) and a ballot per expert counts
-// the hits.  The warp of column slice 0 then writes the slot map (a hint for the
-// low-latency combine) and src_info.
-__device__ __forceinline__ long long packed_row(const DispatchParams& p, long long g, int lane, int part,
-                                                int* s_ek) {
+// at most kLLDirectMaxT tokens): slot = the tokens of earlier sources naming
+// the expert (a sum over the ranking's per-source counts) + the token's rank
+// among its own source's tokens naming it (the ranking's within); the warp of
+// column slice 0 writes the slot map (a hint for the low-latency combine) and
+// src_info.
+__device__ __forceinline__ long long packed_row(const DispatchParams& p, long long g, int lane, int part) {
     const int L = p.E / p.R;
     const int s = (int)(g / p.T), t = (int)(g % p.T);
     long long e = -1;
@@ -76,32 +73,17 @@ __device__ __forceinline__ long long packed_row(const DispatchParams& p, long lo
         const long long ek = __shfl_sync(kFullMask, e, k);
         if (k < lane && ek == e) first = false;
     }
-    int within = 0;
-    if (p.ll_base != nullptr) {
-        s_ek[lane] = live ? (int)e : INT_MIN;
-        __syncwarp();
-        for (int c0 = 0; c0 < t; c0 += 32) {
-            const int tp = c0 + lane;        // an earlier token of source s
-            uint32_t hits = 0;               // bit k: token tp names the expert of slot k
-            if (tp < t) {
-                const int64_t* ids = p.topk_idx + ((long long)s * p.T + tp) * p.K;
-                for (int k2 = 0; k2 < p.K; ++k2) {
-                    const int64_t v = ids[k2];
-                    for (int k = 0; k < p.K; ++k) hits |= (uint32_t)(v == (int64_t)s_ek[k]) << k;
-                }
-            }
-            for (int k = 0; k < p.K; ++k) {
-                const int n = __popc(__ballot_sync(kFullMask, (hits >> k) & 1u));
-                if (lane == k) within += n;
-            }
-        }
-    }
     pdl_wait();
     int slot = -1;
     if (live) {
-        if (p.ll_base != nullptr) {
-            slot = p.ll_base[(long long)s * p.E + e] + within;
-            if (part == 0 && slot < p.ll_capacity) {
+        if (p.ll_cnt != nullptr) {
+            slot = p.ll_within[g * p.K + lane];
+            const int* col = p.ll_cnt + e;
+            int base = 0;
+#pragma unroll 4
+            for (int s2 = 0; s2 < s; ++s2) base += col[(long long)s2 * p.E];
+            slot += base;
+            if (part == 0 && slot >= 0 && slot < p.ll_capacity) {
                 p.slot_map[g * p.K + lane] = slot;
                 if (first) p.ll_src_info[e * p.ll_capacity + slot] = t;
             }
@@ -119,11 +101,39 @@ __device__ __forceinline__ long long packed_row(const DispatchParams& p, long lo
     return row;
 }
 
-template <int kMode, int kVec = kVecPerLane>
-__global__ void __launch_bounds__(kDispatchThreads, 2)
+// Direct slots: the per-expert tables of the packed lists from the ranking's
+// per-source counts -- layout_range[e][s] = (tokens of earlier sources, tokens
+// of s) and the list length -- one expert per warp (an exclusive scan over the
+// lanes, lane s holding source s), spread over all the copy's warps.
+__device__ __forceinline__ void ll_direct_tables(const DispatchParams& p, long long wid, int lane) {
+    const long long nwarps = p.G * p.splits;
+    for (long long e = wid; e < p.E; e += nwarps) {
+        const int c = lane < p.R ? p.ll_cnt[(long long)lane * p.E + e] : 0;
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(kFullMask, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane < p.R) {
+            p.ll_layout_range[(e * p.R + lane) * 2 + 0] = incl - c;
+            p.ll_layout_range[(e * p.R + lane) * 2 + 1] = c;
+        }
+        if (lane == p.R - 1) p.ll_count[e] = incl;
+    }
+}
+
+#ifndef EP_LL_COPY_VEC
+#define EP_LL_COPY_VEC 28
+#endif
+#ifndef EP_LL_COPY_MINB
+#define EP_LL_COPY_MINB 2
+#endif
+
+template <int kMode, int kVec = kVecPerLane, int kMinBlocks = 2>
+__global__ void __launch_bounds__(kDispatchThreads, kMinBlocks)
 dispatch_kernel(const DispatchParams p) {
     __shared__ long long s_rows[kDispatchWarps][32];
-    __shared__ int s_ek[kMode == kModeLowLatency ? kDispatchWarps : 1][32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const long long wid = (long long)blockIdx.x * kDispatchWarps + warp;
     const long long g = wid / p.splits;          // token
@@ -147,7 +157,8 @@ dispatch_kernel(const DispatchParams p) {
     constexpr bool kPacked = kMode == kModeLowLatency;
     long long row = -1;
     if (kPacked) {
-        row = packed_row(p, g, lane, part, s_ek[kPacked ? warp : 0]);
+        row = packed_row(p, g, lane, part);
+        if (p.ll_cnt != nullptr) ll_direct_tables(p, wid, lane);
     } else if (lane < p.R) {
         const int h = p.send_head[g * p.R + lane];
         if (h >= 0) {
@@ -262,7 +273,6 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
 __global__ void __launch_bounds__(kDispatchThreads, kFp8Steps <= 3 ? 4 : 2)
 ll_fp8_copy_kernel(const DispatchParams p) {
     __shared__ long long s_rows[kDispatchWarps][32];
-    __shared__ int s_ek[kDispatchWarps][32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const long long wid = (long long)blockIdx.x * kDispatchWarps + warp;
     const long long g = wid / p.splits;          // token
@@ -278,7 +288,8 @@ ll_fp8_copy_kernel(const DispatchParams p) {
     if (lane == 0 && s_lo < s_hi)
         prefetch_l2(p.x + g * p.H + (long long)s_lo * 512, (uint32_t)(min(nvec, s_hi * 64) - s_lo * 64) * 16u);
 
-    const long long row = packed_row(p, g, lane, part, s_ek[warp]);
+    const long long row = packed_row(p, g, lane, part);
+    if (p.ll_cnt != nullptr) ll_direct_tables(p, wid, lane);
     const uint32_t m = __ballot_sync(kFullMask, row >= 0);
     const int f = __popc(m);
     if (row >= 0) s_rows[warp][__popc(m & lanemask_lt())] = row;
@@ -370,7 +381,8 @@ cudaError_t launch_ll_copy_fp8(DispatchParams p, cudaStream_t stream, bool after
 template <int kMode>
 cudaError_t launch_mode(const DispatchParams& p, cudaStream_t stream, bool after_scan) {
     const long long blocks = (p.G * p.splits + kDispatchWarps - 1) / kDispatchWarps;
-    constexpr int kVec = kVecPerLane;
+    constexpr int kVec = kMode == kModeLowLatency ? EP_LL_COPY_VEC : kVecPerLane;
+    constexpr int kMinB = kMode == kModeLowLatency ? EP_LL_COPY_MINB : 2;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)blocks);
     cfg.blockDim = dim3(kDispatchThreads);
@@ -381,7 +393,7 @@ cudaError_t launch_mode(const DispatchParams& p, cudaStream_t stream, bool after
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = after_scan ? 1 : 0;   // may overlap the scan's tail (see pdl_wait above)
-    return cudaLaunchKernelEx(&cfg, dispatch_kernel<kMode, kVec>, p);
+    return cudaLaunchKernelEx(&cfg, dispatch_kernel<kMode, kVec, kMinB>, p);
 }
 
 }  // namespace

@@ -77,9 +77,12 @@ struct DispatchParams {
     int* slot_map;                     // [G][K]: read (slot scan) or written (direct slots)
     const int* rank_mask;              // [R], 0 active / 1 masked
     int64_t ll_capacity;               // R * Tmax slots per expert
-    const int* ll_base;                // [R][E] direct slots: first slot of source s in expert e's
-                                       // list (from ll_hist_kernel), or null: slots from slot_map
-    int* ll_src_info;                  // [E][ll_capacity] direct slots: written by the copy
+    // direct slots (ll_rank_kernel ran before; null ll_cnt: slots from slot_map)
+    const int* ll_cnt;                 // [R][E] tokens of source s naming e
+    const int* ll_within;              // [G][K] rank of the token among its source's tokens naming e
+    int* ll_src_info;                  // [E][ll_capacity] written by the copy
+    int* ll_layout_range;              // [E][R][2] written by the copy
+    int* ll_count;                     // [E] written by the copy
     uint16_t* recv_x;                  // normal/cached: [cap][H]; LL: [E][ll_cap][H]
     // low latency, FP8 form (recv_x unused)
     uint8_t* recv_fp8;                 // [E][ll_cap][H] E4M3 codes
@@ -167,25 +170,25 @@ constexpr int kLLTile = 256;   // tokens per tile == threads per block
 cudaError_t launch_ll_count(const LLCountParams& p, cudaStream_t stream);
 
 // Direct low-latency slots, for sources of at most kLLDirectMaxT tokens (decode
-// batches): slot(s, t, e) = base[s][e] + (tokens t' < t of source s naming e).
-// ll_hist_kernel (one block per source) counts the tokens of each source that
-// name each expert; its last block turns the counts into base, layout_range and
-// the per-expert counts.  The copy kernel, launched behind it, counts the
-// earlier tokens of its own source while the histogram runs, then adds base.
-// Nothing waits on another block, so nothing needs a bounded wait.
-struct LLHistParams {
+// batches): slot(s, t, e) = base[s][e] + within[s][t][e], where within counts
+// the tokens t' < t of source s naming e and base the tokens of sources s' < s
+// naming e.  ll_rank_kernel (one block per source, one thread per token) writes
+// the source's per-expert counts and every (token, k)'s within; the copy kernel,
+// launched behind it, sums the counts of the earlier sources (base) and writes
+// src_info, layout_range and the per-expert counts.  No block waits on another.
+struct LLRankParams {
     const int64_t* topk_idx;   // [G][K]
     const int* rank_mask;      // [R]
-    int* cnt;                  // [R][E] tokens of source s naming e (each call overwrites)
-    int* base;                 // [R][E] first slot of source s in expert e's list
-    int* layout_range;         // [E][R][2]
-    int* packed_recv_count;    // [E]
-    unsigned int* done;        // blocks finished; the last block resets it to 0
+    int* cnt;                  // [R][E] tokens of source s naming e
+    int* within;               // [G][K] tokens before t in its source naming slot k's expert (-1: not sent)
     int* err;
     int R, E, T, K;
 };
-constexpr int kLLDirectMaxT = 256;   // == kLLTile: one block per source
-cudaError_t launch_ll_hist(const LLHistParams& p, cudaStream_t stream);
+#ifndef EP_LL_DIRECT_MAX_T
+#define EP_LL_DIRECT_MAX_T 256
+#endif
+constexpr int kLLDirectMaxT = EP_LL_DIRECT_MAX_T;   // <= kLLTile: one block per source
+cudaError_t launch_ll_rank(const LLRankParams& p, cudaStream_t stream);
 cudaError_t ll_prepare(int E);   // once per device: shared-memory opt-in
 
 struct LLCombineParams {

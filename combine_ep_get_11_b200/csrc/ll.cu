@@ -29,9 +29,6 @@ namespace ep {
 
 namespace {
 
-#ifndef EP_LL_COMBINE_PREFETCH
-#define EP_LL_COMBINE_PREFETCH 0
-#endif
 constexpr int kLLCombineThreads = 256;
 constexpr int kLLCombineWarps = kLLCombineThreads / 32;
 constexpr int kLLRowsPerGroup = 8;
@@ -228,63 +225,66 @@ ll_slot_kernel(const LLCountParams p) {
     }
 }
 
-// Direct slots, histogram part: block s counts, per expert, the tokens of
-// source s that name it (a token naming an expert twice counts once; tokens of
-// a masked source and experts of a masked rank count nothing) and stores the
-// counts; the last block to finish turns every expert's column of counts into
-// its exclusive prefix over sources (base, layout_range) and the total
-// (packed_recv_count), then resets the finish counter for the next call.
+// Direct slots, ranking part: block s holds the tokens of source s, one per
+// thread.  Each token sets one bit per expert it names in a [E][8]-word
+// membership bitmap (a token naming an expert twice sets the same bit; tokens
+// of a masked source and experts of a masked rank set nothing).  Thread e then
+// stores expert e's count for the source, and each token's within for slot k is
+// the members of its expert before it: the bitmap words before its own plus the
+// bits below it in its word.  No block waits on another; the copy kernel adds
+// the earlier sources' counts.
 template <int kMaxK>
 __global__ void __launch_bounds__(kLLTile)
-ll_hist_kernel(const LLHistParams p) {
-    extern __shared__ int h_cnt[];   // [E]
-    __shared__ bool s_last;
-    pdl_launch_dependents();         // the copy may start counting its source's earlier tokens
+ll_rank_kernel(const LLRankParams p) {
+    extern __shared__ uint32_t rk_smem[];
+    const int E = p.E;
+    uint32_t* bits = rk_smem;                                                 // [E][kLLStride]
+    uint8_t* s_wpref = reinterpret_cast<uint8_t*>(bits + (size_t)E * kLLStride);   // [E][kLLWords]
+    pdl_launch_dependents();         // the copy may start prefetching its rows
     const int s = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
-    const int E = p.E, L = p.E / p.R;
-    for (int e = tid; e < E; e += kLLTile) h_cnt[e] = 0;
+    const int L = E / p.R;
     const uint32_t mbits = __ballot_sync(kFullMask, lane < p.R && p.rank_mask[lane] != 0);
+    for (int e = tid; e < E; e += kLLTile) {
+#pragma unroll
+        for (int q = 0; q < kLLStride; ++q) bits[e * kLLStride + q] = 0;
+    }
+    __syncthreads();
+    const int w = tid >> 5, b = lane;
+    const long long g = (long long)s * p.T + tid;
+    const bool src_live = ((mbits >> s) & 1u) == 0;
+    int ids[kMaxK];
+    bool bad = false;
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k) {
+        const int64_t e = (tid < p.T && k < p.K) ? __ldg(p.topk_idx + g * p.K + k) : -1;
+        bad |= e < -1 || e >= E;
+        ids[k] = (e >= 0 && e < E && src_live && ((mbits >> ((int)e / L)) & 1u) == 0) ? (int)e : -1;
+    }
+    if (bad) record_error(p.err, EP_ERR_BAD_TOPK);
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k)
+        if (ids[k] >= 0) atomicOr(&bits[ids[k] * kLLStride + w], 1u << b);
+    __syncthreads();
+    for (int e = tid; e < E; e += kLLTile) {
+        int agg = 0;
+#pragma unroll
+        for (int q = 0; q < kLLWords; ++q) {
+            s_wpref[e * kLLWords + q] = (uint8_t)agg;
+            agg += __popc(bits[e * kLLStride + q]);
+        }
+        p.cnt[(size_t)s * E + e] = agg;
+    }
     __syncthreads();
     if (tid < p.T) {
-        const long long g = (long long)s * p.T + tid;
-        const bool src_live = ((mbits >> s) & 1u) == 0;
-        int ids[kMaxK];
-        bool bad = false;
+        const uint32_t below = (1u << b) - 1u;
 #pragma unroll
         for (int k = 0; k < kMaxK; ++k) {
-            const int64_t e = k < p.K ? __ldg(p.topk_idx + g * p.K + k) : -1;
-            bad |= e < -1 || e >= E;
-            ids[k] = (e >= 0 && e < E && src_live && ((mbits >> ((int)e / L)) & 1u) == 0) ? (int)e : -1;
-        }
-        if (bad) record_error(p.err, EP_ERR_BAD_TOPK);
-#pragma unroll
-        for (int k = 0; k < kMaxK; ++k) {
-            bool first = ids[k] >= 0;
-#pragma unroll
-            for (int k2 = 0; k2 < k; ++k2) first = first && ids[k2] != ids[k];
-            if (first) atomicAdd(&h_cnt[ids[k]], 1);
+            if (k >= p.K) break;
+            const int e = ids[k];
+            p.within[g * p.K + k] =
+                e >= 0 ? (int)s_wpref[e * kLLWords + w] + __popc(bits[e * kLLStride + w] & below) : -1;
         }
     }
-    __syncthreads();
-    for (int e = tid; e < E; e += kLLTile) p.cnt[(size_t)s * E + e] = h_cnt[e];
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(p.done, 1u) == gridDim.x - 1;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    for (int e = tid; e < E; e += kLLTile) {
-        int run = 0;
-        for (int src = 0; src < p.R; ++src) {
-            const int c = __ldcg(p.cnt + (size_t)src * E + e);
-            p.base[(size_t)src * E + e] = run;
-            p.layout_range[((size_t)e * p.R + src) * 2 + 0] = run;
-            p.layout_range[((size_t)e * p.R + src) * 2 + 1] = c;
-            run += c;
-        }
-        p.packed_recv_count[e] = run;
-    }
-    if (tid == 0) *p.done = 0u;
 }
 
 __device__ __forceinline__ void fma_bf16x8(float* acc, float w, const uint4& v) {
@@ -368,16 +368,7 @@ ll_combine_kernel(const LLCombineParams p) {
         uint4* out = reinterpret_cast<uint4*>(p.out_x + g * p.H);
         const int per = ((nvec + p.splits - 1) / p.splits + 31) / 32 * 32;
         const int clo = part * per, chi = min(nvec, clo + per);
-#if EP_LL_COMBINE_PREFETCH
-        // lane i asks for the next column slab of row i ahead of its loads (a bulk L2 prefetch)
-        const uint4* pf_row = lane < nv ? reinterpret_cast<const uint4*>(p.y + s_rows[warp][lane] * p.H) : nullptr;
-        if (pf_row != nullptr && clo < chi) prefetch_l2(pf_row + clo, (uint32_t)min(32 * U, chi - clo) * 16u);
-#endif
         for (int c0 = clo; c0 < chi; c0 += 32 * U) {
-#if EP_LL_COMBINE_PREFETCH
-            const int nxt = c0 + 32 * U;
-            if (pf_row != nullptr && nxt < chi) prefetch_l2(pf_row + nxt, (uint32_t)min(32 * U, chi - nxt) * 16u);
-#endif
             float acc[U][8];
 #pragma unroll
             for (int u = 0; u < U; ++u)
@@ -431,15 +422,19 @@ cudaError_t launch_set_mask(int* rank_mask, int rank, int value, cudaStream_t st
     return cudaGetLastError();
 }
 
-cudaError_t launch_ll_hist(const LLHistParams& p, cudaStream_t stream) {
+__host__ __device__ inline size_t ll_rank_smem(int E) {
+    return (size_t)E * kLLStride * sizeof(uint32_t) + (size_t)E * kLLWords;
+}
+
+cudaError_t launch_ll_rank(const LLRankParams& p, cudaStream_t stream) {
     if (p.R == 0 || p.E == 0) return cudaSuccess;
-    const size_t smem = (size_t)p.E * sizeof(int);
+    const size_t smem = ll_rank_smem(p.E);
     if (p.K <= 8)
-        ll_hist_kernel<8><<<p.R, kLLTile, smem, stream>>>(p);
+        ll_rank_kernel<8><<<p.R, kLLTile, smem, stream>>>(p);
     else if (p.K <= 16)
-        ll_hist_kernel<16><<<p.R, kLLTile, smem, stream>>>(p);
+        ll_rank_kernel<16><<<p.R, kLLTile, smem, stream>>>(p);
     else
-        ll_hist_kernel<32><<<p.R, kLLTile, smem, stream>>>(p);
+        ll_rank_kernel<32><<<p.R, kLLTile, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -452,6 +447,13 @@ cudaError_t ll_prepare(int E) {
         e = cudaFuncSetAttribute(ll_slot_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(ll_slot_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int rsmem = (int)ll_rank_smem(E);
+    if (e == cudaSuccess && rsmem > 48 * 1024)
+        e = cudaFuncSetAttribute(ll_rank_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem);
+    if (e == cudaSuccess && rsmem > 48 * 1024)
+        e = cudaFuncSetAttribute(ll_rank_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem);
+    if (e == cudaSuccess && rsmem > 48 * 1024)
+        e = cudaFuncSetAttribute(ll_rank_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem);
     return e;
 }
 
