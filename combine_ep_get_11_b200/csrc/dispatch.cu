@@ -129,13 +129,21 @@ __device__ __forceinline__ void ll_direct_tables(const DispatchParams& p, long l
 #ifndef EP_LL_COPY_MINB
 #define EP_LL_COPY_MINB 2
 #endif
+// The packed (low-latency) copy runs one-warp blocks: with few tokens its 2 x G
+// warps fill 1.7 waves of the GPU, and single-warp blocks let the scheduler hand
+// out the second wave warp by warp (measured on B200, LL shape: step 90.3 vs
+// 91.2 us for 8-warp blocks; 2- and 4-warp blocks 91.2).
+#ifndef EP_LL_COPY_THREADS
+#define EP_LL_COPY_THREADS 32
+#endif
 
-template <int kMode, int kVec = kVecPerLane, int kMinBlocks = 2>
-__global__ void __launch_bounds__(kDispatchThreads, kMinBlocks)
+template <int kMode, int kVec = kVecPerLane, int kMinBlocks = 2, int kThreads = kDispatchThreads>
+__global__ void __launch_bounds__(kThreads, kMinBlocks)
 dispatch_kernel(const DispatchParams p) {
-    __shared__ long long s_rows[kDispatchWarps][32];
+    constexpr int kWarps = kThreads / 32;
+    __shared__ long long s_rows[kWarps][32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const long long wid = (long long)blockIdx.x * kDispatchWarps + warp;
+    const long long wid = (long long)blockIdx.x * kWarps + warp;
     const long long g = wid / p.splits;          // token
     const int part = (int)(wid % p.splits);      // column slice of its row
     if (g >= p.G) return;   // whole warp
@@ -270,11 +278,17 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
     return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
-__global__ void __launch_bounds__(kDispatchThreads, kFp8Steps <= 3 ? 4 : 2)
+#ifndef EP_FP8_THREADS
+#define EP_FP8_THREADS 256
+#endif
+constexpr int kFp8Threads = EP_FP8_THREADS;
+
+__global__ void __launch_bounds__(kFp8Threads, (kFp8Steps <= 3 ? 4 : 2) * (kDispatchThreads / kFp8Threads))
 ll_fp8_copy_kernel(const DispatchParams p) {
-    __shared__ long long s_rows[kDispatchWarps][32];
+    constexpr int kWarps = kFp8Threads / 32;
+    __shared__ long long s_rows[kWarps][32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const long long wid = (long long)blockIdx.x * kDispatchWarps + warp;
+    const long long wid = (long long)blockIdx.x * kWarps + warp;
     const long long g = wid / p.splits;          // token
     const int part = (int)(wid % p.splits);      // column slice of its row (whole steps)
     if (g >= p.G) return;   // whole warp
@@ -364,10 +378,10 @@ cudaError_t launch_ll_copy_fp8(DispatchParams p, cudaStream_t stream, bool after
     // column slices per row: the fewest with one pass each (EP_FP8_SPLITS 0), or a
     // fixed count whose warps loop over several passes
     p.splits = EP_FP8_SPLITS > 0 ? min(EP_FP8_SPLITS, nstep) : (nstep + kFp8Steps - 1) / kFp8Steps;
-    const long long blocks = (p.G * p.splits + kDispatchWarps - 1) / kDispatchWarps;
+    const long long blocks = (p.G * p.splits + kFp8Threads / 32 - 1) / (kFp8Threads / 32);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)blocks);
-    cfg.blockDim = dim3(kDispatchThreads);
+    cfg.blockDim = dim3(kFp8Threads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -380,12 +394,13 @@ cudaError_t launch_ll_copy_fp8(DispatchParams p, cudaStream_t stream, bool after
 
 template <int kMode>
 cudaError_t launch_mode(const DispatchParams& p, cudaStream_t stream, bool after_scan) {
-    const long long blocks = (p.G * p.splits + kDispatchWarps - 1) / kDispatchWarps;
+    constexpr int kThreads = kMode == kModeLowLatency ? EP_LL_COPY_THREADS : kDispatchThreads;
     constexpr int kVec = kMode == kModeLowLatency ? EP_LL_COPY_VEC : kVecPerLane;
-    constexpr int kMinB = kMode == kModeLowLatency ? EP_LL_COPY_MINB : 2;
+    constexpr int kMinB = kMode == kModeLowLatency ? EP_LL_COPY_MINB * (kDispatchThreads / kThreads) : 2;
+    const long long blocks = (p.G * p.splits + kThreads / 32 - 1) / (kThreads / 32);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)blocks);
-    cfg.blockDim = dim3(kDispatchThreads);
+    cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -393,7 +408,7 @@ cudaError_t launch_mode(const DispatchParams& p, cudaStream_t stream, bool after
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = after_scan ? 1 : 0;   // may overlap the scan's tail (see pdl_wait above)
-    return cudaLaunchKernelEx(&cfg, dispatch_kernel<kMode, kVec, kMinB>, p);
+    return cudaLaunchKernelEx(&cfg, dispatch_kernel<kMode, kVec, kMinB, kThreads>, p);
 }
 
 }  // namespace
