@@ -45,7 +45,6 @@ namespace ep {
 namespace {
 
 constexpr int kDispatchThreads = 256;
-constexpr int kDispatchWarps = kDispatchThreads / 32;
 constexpr int kVecPerLane = 28;   // 16-byte vectors held per lane per pass
 
 // Packed (low-latency) destination of lane k's top-k slot of token g: the row
