@@ -243,23 +243,28 @@ ll_rank_kernel(const LLRankParams p) {
     pdl_launch_dependents();         // the copy may start prefetching its rows
     const int s = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
     const int L = E / p.R;
-    const uint32_t mbits = __ballot_sync(kFullMask, lane < p.R && p.rank_mask[lane] != 0);
+    const int w = tid >> 5, b = lane;
+    const long long g = (long long)s * p.T + tid;
+    // the token's ids and the rank mask are independent loads: issue both before using either
+    int64_t raw[kMaxK];
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k) raw[k] = (tid < p.T && k < p.K) ? __ldg(p.topk_idx + g * p.K + k) : -1;
+    const int mask_lane = lane < p.R ? p.rank_mask[lane] : 0;
     for (int e = tid; e < E; e += kLLTile) {
 #pragma unroll
         for (int q = 0; q < kLLStride; ++q) bits[e * kLLStride + q] = 0;
     }
-    __syncthreads();
-    const int w = tid >> 5, b = lane;
-    const long long g = (long long)s * p.T + tid;
+    const uint32_t mbits = __ballot_sync(kFullMask, mask_lane != 0);
     const bool src_live = ((mbits >> s) & 1u) == 0;
     int ids[kMaxK];
     bool bad = false;
 #pragma unroll
     for (int k = 0; k < kMaxK; ++k) {
-        const int64_t e = (tid < p.T && k < p.K) ? __ldg(p.topk_idx + g * p.K + k) : -1;
+        const int64_t e = raw[k];
         bad |= e < -1 || e >= E;
         ids[k] = (e >= 0 && e < E && src_live && ((mbits >> ((int)e / L)) & 1u) == 0) ? (int)e : -1;
     }
+    __syncthreads();   // the bitmap is clear
     if (bad) record_error(p.err, EP_ERR_BAD_TOPK);
 #pragma unroll
     for (int k = 0; k < kMaxK; ++k)
