@@ -48,6 +48,7 @@ __device__ __forceinline__ void add_bf16x8(float* acc, const uint4& v) {
 template <int U, bool kSharded, int kGroup = kRowsPerGroup>
 __global__ void __launch_bounds__(kCombineThreads, 2)
 combine_kernel(const CombineParams p) {
+    pdl_wait();   // (launched with programmatic serialization: reads nothing before this)
     __shared__ long long s_rows[kCombineWarps][32];             // row index, or (sharded) row address
     __shared__ long long s_wrow[kSharded ? kCombineWarps : 1][32];   // sharded: weight-row address
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -167,11 +168,8 @@ cudaError_t launch_combine(const CombineParams& p, int num_sms, cudaStream_t str
     // one warp per token (or column slice): the block scheduler balances the work
     (void)num_sms;
     const long long blocks = (p.G * p.splits + kCombineWarps - 1) / kCombineWarps;
-    if (p.sharded)
-        combine_kernel<U, true><<<(unsigned)blocks, kCombineThreads, 0, stream>>>(p);
-    else
-        combine_kernel<U, false><<<(unsigned)blocks, kCombineThreads, 0, stream>>>(p);
-    return cudaGetLastError();
+    if (p.sharded) return launch_pdl(combine_kernel<U, true>, dim3((unsigned)blocks), dim3(kCombineThreads), 0, stream, p);
+    return launch_pdl(combine_kernel<U, false>, dim3((unsigned)blocks), dim3(kCombineThreads), 0, stream, p);
 }
 
 }  // namespace ep

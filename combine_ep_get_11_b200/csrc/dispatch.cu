@@ -147,19 +147,31 @@ dispatch_kernel(const DispatchParams p) {
     const int part = (int)(wid % p.splits);      // column slice of its row
     if (g >= p.G) return;   // whole warp
 
-    // The normal and packed forms are launched right behind the handle / slot
-    // scan (or the slot histogram) and may start before it ends: pull this
-    // warp's slice of the source row (never written by that kernel) into L2
-    // meanwhile, then wait for it (the packed form inside packed_row).
-    if constexpr (kMode == kModeNormal || kMode == kModeLowLatency) {
-        if (lane == 0) {
-            const int nv = p.H / 8;
-            const int per = ((nv + p.splits - 1) / p.splits + 31) / 32 * 32;
-            const int lo = part * per, hi = min(nv, lo + per);
-            if (lo < hi) prefetch_l2(p.x + g * p.H + (long long)lo * 8, (uint32_t)(hi - lo) * 16u);
+    // this warp's column slice: whole 32-vector strides
+    const int nvec = p.H / 8;
+    const int per = ((nvec + p.splits - 1) / p.splits + 31) / 32 * 32;
+    const int lo = part * per, hi = min(nvec, lo + per);
+    const uint4* src = reinterpret_cast<const uint4*>(p.x + g * p.H);
+    uint4 v[kVec];
+    // The sharded form loads the first pass of its slice at once, before it reads
+    // the handle (measured faster).  The normal and packed forms are launched
+    // right behind the handle / slot kernel and may start before it ends: they
+    // pull the slice (an input of the call, never written by that kernel) into L2
+    // meanwhile and wait for that kernel (the packed form inside packed_row);
+    // holding the slice in registers across the wait measured slower on B200
+    // (DSv3 dispatch 459 vs 452 us).
+    constexpr bool kPreload = kMode == kModeSharded;
+    if constexpr (kPreload) {
+#pragma unroll
+        for (int u = 0; u < kVec; ++u) {
+            const int c = lo + lane + 32 * u;
+            if (c < hi) v[u] = ld_nc_v4(src + c);
         }
-        if (kMode == kModeNormal) pdl_wait();
     }
+    if constexpr (kMode == kModeNormal || kMode == kModeLowLatency) {
+        if (lane == 0 && lo < hi) prefetch_l2(src + lo, (uint32_t)(hi - lo) * 16u);
+    }
+    if constexpr (kMode == kModeNormal) pdl_wait();
 
     constexpr bool kPacked = kMode == kModeLowLatency;
     long long row = -1;
@@ -205,7 +217,7 @@ dispatch_kernel(const DispatchParams p) {
             }
         }
     }
-    if (kMode == kModeNormal && p.recv_x == nullptr) return;   // metadata only
+    if (kMode == kModeNormal && p.recv_x == nullptr) return;   // metadata only (the loaded row unused)
     if (kMode == kModeSharded && row >= 0)                     // keep the row's address
         row = (long long)reinterpret_cast<uintptr_t>(p.shard_rows[shard] + row * p.H);
 
@@ -214,17 +226,13 @@ dispatch_kernel(const DispatchParams p) {
     if (row >= 0) s_rows[warp][__popc(m & lanemask_lt())] = row;
     __syncwarp();
 
-    // this warp's column slice: whole 32-vector strides
-    const int nvec = p.H / 8;
-    const int per = ((nvec + p.splits - 1) / p.splits + 31) / 32 * 32;
-    const int lo = part * per, hi = min(nvec, lo + per);
-    const uint4* src = reinterpret_cast<const uint4*>(p.x + g * p.H);
     for (int c0 = lo; c0 < hi; c0 += 32 * kVec) {
-        uint4 v[kVec];
+        if (!kPreload || c0 != lo) {
 #pragma unroll
-        for (int u = 0; u < kVec; ++u) {
-            const int c = c0 + lane + 32 * u;
-            if (c < hi) v[u] = ld_nc_v4(src + c);
+            for (int u = 0; u < kVec; ++u) {
+                const int c = c0 + lane + 32 * u;
+                if (c < hi) v[u] = ld_nc_v4(src + c);
+            }
         }
         for (int i = 0; i < f; ++i) {
             uint4* dst = kMode == kModeSharded
@@ -277,6 +285,54 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
     return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
+// One pass of the FP8 form: the steps [st0, min(st0 + kFp8Steps, s_hi)) of a
+// row (lane l: channels [16 l, 16 l + 16) of each step), loaded and turned into
+// E4M3 codes (codes[k] for step st0 + k) and the pass's block scales gathered
+// one per lane (block j of the pass -- step j / 4, block j % 4 of the step --
+// in lane j).
+__device__ __forceinline__ void fp8_convert_pass(const uint4* src, int st0, int s_hi, int nvec, int lane,
+                                                 uint4 (&codes)[kFp8Steps], float& my_scale) {
+    uint4 a[kFp8Steps], b[kFp8Steps];
+#pragma unroll
+    for (int k = 0; k < kFp8Steps; ++k) {
+        const int c = (st0 + k) * 64 + 2 * lane;
+        if (st0 + k < s_hi && c < nvec) ld_nc_v8(src + c, a[k], b[k]);
+    }
+    float scale[kFp8Steps];
+#pragma unroll
+    for (int k = 0; k < kFp8Steps; ++k) {
+        scale[k] = 1.f;
+        if (st0 + k >= s_hi) break;                       // warp-uniform
+        const bool on = (st0 + k) * 64 + 2 * lane < nvec;
+        float xs[16];
+        xs[0] = bf16_lo(a[k].x);  xs[1] = bf16_hi(a[k].x);  xs[2] = bf16_lo(a[k].y);  xs[3] = bf16_hi(a[k].y);
+        xs[4] = bf16_lo(a[k].z);  xs[5] = bf16_hi(a[k].z);  xs[6] = bf16_lo(a[k].w);  xs[7] = bf16_hi(a[k].w);
+        xs[8] = bf16_lo(b[k].x);  xs[9] = bf16_hi(b[k].x);  xs[10] = bf16_lo(b[k].y); xs[11] = bf16_hi(b[k].y);
+        xs[12] = bf16_lo(b[k].z); xs[13] = bf16_hi(b[k].z); xs[14] = bf16_lo(b[k].w); xs[15] = bf16_hi(b[k].w);
+        float amax = 0.f;
+        if (on) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(xs[i]));
+        }
+        amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 4));
+        scale[k] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+        const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            w[q] = e4m3x4(__fmul_rn(xs[4 * q], inv), __fmul_rn(xs[4 * q + 1], inv),
+                          __fmul_rn(xs[4 * q + 2], inv), __fmul_rn(xs[4 * q + 3], inv));
+        codes[k] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+#pragma unroll
+    for (int k = 0; k < kFp8Steps; ++k) {
+        const float v = __shfl_sync(kFullMask, scale[k], (lane & 3) * kFp8LanesPerBlock);
+        if ((lane >> 2) == k) my_scale = v;
+    }
+}
+
 #ifndef EP_FP8_THREADS
 #define EP_FP8_THREADS 256
 #endif
@@ -296,10 +352,17 @@ ll_fp8_copy_kernel(const DispatchParams p) {
     const int nstep = (nvec + 63) / 64;
     const int per = (nstep + p.splits - 1) / p.splits;
     const int s_lo = part * per, s_hi = min(nstep, s_lo + per);
-    // launched right behind the slot scan (or histogram): pull this warp's slice
-    // of the source row into L2 while it finishes (packed_row waits for it)
-    if (lane == 0 && s_lo < s_hi)
-        prefetch_l2(p.x + g * p.H + (long long)s_lo * 512, (uint32_t)(min(nvec, s_hi * 64) - s_lo * 64) * 16u);
+    const uint4* src = reinterpret_cast<const uint4*>(p.x + g * p.H);
+    // Launched right behind the slot kernel: the row is an input of the call,
+    // never written by that kernel, so the first pass is loaded and converted
+    // while it runs; only the stores wait for the slots (packed_row).  Later
+    // passes (rows wider than kFp8Steps steps per warp) are pulled into L2.
+    if (lane == 0 && s_lo + kFp8Steps < s_hi)
+        prefetch_l2(p.x + g * p.H + (long long)(s_lo + kFp8Steps) * 512,
+                    (uint32_t)(min(nvec, s_hi * 64) - (s_lo + kFp8Steps) * 64) * 16u);
+    uint4 codes[kFp8Steps];
+    float my_scale = 1.f;
+    fp8_convert_pass(src, s_lo, s_hi, nvec, lane, codes, my_scale);
 
     const long long row = packed_row(p, g, lane, part);
     if (p.ll_cnt != nullptr) ll_direct_tables(p, wid, lane);
@@ -309,50 +372,8 @@ ll_fp8_copy_kernel(const DispatchParams p) {
     __syncwarp();
 
     const int nblk = p.H / kFp8Block;
-    const uint4* src = reinterpret_cast<const uint4*>(p.x + g * p.H);
     for (int st0 = s_lo; st0 < s_hi; st0 += kFp8Steps) {
-        uint4 a[kFp8Steps], b[kFp8Steps];
-#pragma unroll
-        for (int k = 0; k < kFp8Steps; ++k) {
-            const int c = (st0 + k) * 64 + 2 * lane;
-            if (st0 + k < s_hi && c < nvec) ld_nc_v8(src + c, a[k], b[k]);
-        }
-        uint4 codes[kFp8Steps];
-        float scale[kFp8Steps];
-#pragma unroll
-        for (int k = 0; k < kFp8Steps; ++k) {
-            scale[k] = 1.f;
-            if (st0 + k >= s_hi) break;                       // warp-uniform
-            const bool on = (st0 + k) * 64 + 2 * lane < nvec;
-            float xs[16];
-            xs[0] = bf16_lo(a[k].x);  xs[1] = bf16_hi(a[k].x);  xs[2] = bf16_lo(a[k].y);  xs[3] = bf16_hi(a[k].y);
-            xs[4] = bf16_lo(a[k].z);  xs[5] = bf16_hi(a[k].z);  xs[6] = bf16_lo(a[k].w);  xs[7] = bf16_hi(a[k].w);
-            xs[8] = bf16_lo(b[k].x);  xs[9] = bf16_hi(b[k].x);  xs[10] = bf16_lo(b[k].y); xs[11] = bf16_hi(b[k].y);
-            xs[12] = bf16_lo(b[k].z); xs[13] = bf16_hi(b[k].z); xs[14] = bf16_lo(b[k].w); xs[15] = bf16_hi(b[k].w);
-            float amax = 0.f;
-            if (on) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(xs[i]));
-            }
-            amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
-            amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
-            amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 4));
-            scale[k] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-            const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
-            uint32_t w[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                w[q] = e4m3x4(__fmul_rn(xs[4 * q], inv), __fmul_rn(xs[4 * q + 1], inv),
-                              __fmul_rn(xs[4 * q + 2], inv), __fmul_rn(xs[4 * q + 3], inv));
-            codes[k] = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        // block j of this pass (step j / 4, block j % 4 of the step) -> lane j
-        float my_scale = 1.f;
-#pragma unroll
-        for (int k = 0; k < kFp8Steps; ++k) {
-            const float v = __shfl_sync(kFullMask, scale[k], (lane & 3) * kFp8LanesPerBlock);
-            if ((lane >> 2) == k) my_scale = v;
-        }
+        if (st0 != s_lo) fp8_convert_pass(src, st0, s_hi, nvec, lane, codes, my_scale);
         const int blk0 = st0 * 4;
         const int nb = min(min(kFp8Steps, s_hi - st0) * 4, nblk - blk0);
         for (int i = 0; i < f; ++i) {
@@ -367,6 +388,7 @@ ll_fp8_copy_kernel(const DispatchParams p) {
         }
     }
 }
+
 
 #ifndef EP_FP8_SPLITS
 #define EP_FP8_SPLITS 0
@@ -394,7 +416,10 @@ cudaError_t launch_ll_copy_fp8(DispatchParams p, cudaStream_t stream, bool after
 template <int kMode>
 cudaError_t launch_mode(const DispatchParams& p, cudaStream_t stream, bool after_scan) {
     constexpr int kThreads = kMode == kModeLowLatency ? EP_LL_COPY_THREADS : kDispatchThreads;
-    constexpr int kVec = kMode == kModeLowLatency ? EP_LL_COPY_VEC : kVecPerLane;
+    // the sharded form holds its first pass across its handle reads: 14 vectors per
+    // lane (one pass of a 7168-wide row in two column slices) keep that within the
+    // register budget
+    constexpr int kVec = kMode == kModeLowLatency ? EP_LL_COPY_VEC : (kMode == kModeSharded ? 14 : kVecPerLane);
     constexpr int kMinB = kMode == kModeLowLatency ? EP_LL_COPY_MINB * (kDispatchThreads / kThreads) : 2;
     const long long blocks = (p.G * p.splits + kThreads / 32 - 1) / (kThreads / 32);
     cudaLaunchConfig_t cfg = {};

@@ -31,6 +31,7 @@ layout_kernel(const LayoutParams p) {
     extern __shared__ int sh[];
     int* sh_rank = sh;        // [32]
     int* sh_expert = sh + 32; // [E]
+    pdl_wait();               // (launched with programmatic serialization: reads nothing before this)
     for (int i = threadIdx.x; i < 32 + p.E; i += blockDim.x) sh[i] = 0;
 
     const int s = blockIdx.y;
@@ -83,13 +84,9 @@ cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream) {
     if (p.num_src == 0) return cudaSuccess;
     dim3 grid((p.T + kLayoutThreads - 1) / kLayoutThreads, p.num_src);
     const size_t smem = (32 + (size_t)p.E) * sizeof(int);
-    if (p.K <= 8)
-        layout_kernel<8><<<grid, kLayoutThreads, smem, stream>>>(p);
-    else if (p.K <= 16)
-        layout_kernel<16><<<grid, kLayoutThreads, smem, stream>>>(p);
-    else
-        layout_kernel<32><<<grid, kLayoutThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    if (p.K <= 8) return launch_pdl(layout_kernel<8>, grid, dim3(kLayoutThreads), smem, stream, p);
+    if (p.K <= 16) return launch_pdl(layout_kernel<16>, grid, dim3(kLayoutThreads), smem, stream, p);
+    return launch_pdl(layout_kernel<32>, grid, dim3(kLayoutThreads), smem, stream, p);
 }
 
 }  // namespace ep

@@ -27,6 +27,7 @@ constexpr int kLBMaxExperts = 4096;
 
 __global__ void __launch_bounds__(kLBThreads)
 lb_prefetch_kernel(const LBParams p) {
+    pdl_wait();   // (launched with programmatic serialization: reads nothing before this)
     const int i = blockIdx.y;
     const int e = p.mapping[i];
     if (e == -1) return;
@@ -65,6 +66,7 @@ lb_reduce_kernel(const LBParams p) {
     __shared__ int s_list[kLBMaxReplicas];
     __shared__ int s_warp[kLBThreads / 32];
     __shared__ int s_n, s_e;
+    pdl_wait();   // (launched with programmatic serialization: reads nothing before this)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int words = (p.E + 31) / 32;
     for (int i = tid; i < words; i += kLBThreads) s_touched[i] = 0;
@@ -160,16 +162,14 @@ lb_reduce_kernel(const LBParams p) {
 cudaError_t launch_lb_prefetch(const LBParams& p, cudaStream_t stream) {
     if (p.N == 0 || p.Wv == 0) return cudaSuccess;
     const dim3 grid((unsigned)((p.Wv + kLBChunk - 1) / kLBChunk), (unsigned)p.N);
-    lb_prefetch_kernel<<<grid, kLBThreads, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(lb_prefetch_kernel, grid, dim3(kLBThreads), 0, stream, p);
 }
 
 cudaError_t launch_lb_reduce(const LBParams& p, cudaStream_t stream) {
     if (p.N == 0 || p.Wv == 0) return cudaSuccess;
     // at most min(E, N) experts have replicas; rows past the touched count exit at once
     const dim3 grid((unsigned)((p.Wv + kLBChunk - 1) / kLBChunk), (unsigned)(p.N < p.E ? p.N : p.E));
-    lb_reduce_kernel<<<grid, kLBThreads, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(lb_reduce_kernel, grid, dim3(kLBThreads), 0, stream, p);
 }
 
 }  // namespace ep

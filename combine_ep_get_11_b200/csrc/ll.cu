@@ -80,7 +80,8 @@ ll_slot_kernel(const LLCountParams p) {
     __shared__ int s_tile;
     __shared__ unsigned long long s_tag;
     const int tid = threadIdx.x;
-    pdl_launch_dependents();   // the packed copy may start prefetching its rows
+    pdl_wait();                // everything before this kernel has completed ...
+    pdl_launch_dependents();   // ... so the packed copy may start prefetching its rows
     if (tid == 0) {
         const unsigned long long tk = atomicAdd(p.ticket, 1ull);
         s_tile = (int)(tk % (unsigned long long)p.num_tiles);
@@ -240,7 +241,8 @@ ll_rank_kernel(const LLRankParams p) {
     const int E = p.E;
     uint32_t* bits = rk_smem;                                                 // [E][kLLStride]
     uint8_t* s_wpref = reinterpret_cast<uint8_t*>(bits + (size_t)E * kLLStride);   // [E][kLLWords]
-    pdl_launch_dependents();         // the copy may start prefetching its rows
+    pdl_wait();                      // everything before this kernel has completed ...
+    pdl_launch_dependents();         // ... so the copy may start reading its rows
     const int s = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
     const int L = E / p.R;
     const int w = tid >> 5, b = lane;
@@ -306,6 +308,7 @@ __device__ __forceinline__ void fma_bf16x8(float* acc, float w, const uint4& v) 
 template <int U, int kGroup = kLLRowsPerGroup>
 __global__ void __launch_bounds__(kLLCombineThreads)
 ll_combine_kernel(const LLCombineParams p) {
+    pdl_wait();   // (launched with programmatic serialization: reads nothing before this)
     __shared__ long long s_rows[kLLCombineWarps][32];
     __shared__ float s_w[kLLCombineWarps][32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -434,13 +437,9 @@ __host__ __device__ inline size_t ll_rank_smem(int E) {
 cudaError_t launch_ll_rank(const LLRankParams& p, cudaStream_t stream) {
     if (p.R == 0 || p.E == 0) return cudaSuccess;
     const size_t smem = ll_rank_smem(p.E);
-    if (p.K <= 8)
-        ll_rank_kernel<8><<<p.R, kLLTile, smem, stream>>>(p);
-    else if (p.K <= 16)
-        ll_rank_kernel<16><<<p.R, kLLTile, smem, stream>>>(p);
-    else
-        ll_rank_kernel<32><<<p.R, kLLTile, smem, stream>>>(p);
-    return cudaGetLastError();
+    if (p.K <= 8) return launch_pdl(ll_rank_kernel<8>, dim3(p.R), dim3(kLLTile), smem, stream, p);
+    if (p.K <= 16) return launch_pdl(ll_rank_kernel<16>, dim3(p.R), dim3(kLLTile), smem, stream, p);
+    return launch_pdl(ll_rank_kernel<32>, dim3(p.R), dim3(kLLTile), smem, stream, p);
 }
 
 cudaError_t ll_prepare(int E) {
@@ -465,13 +464,9 @@ cudaError_t ll_prepare(int E) {
 cudaError_t launch_ll_count(const LLCountParams& p, cudaStream_t stream) {
     if (p.G == 0 || p.E == 0) return cudaSuccess;
     const size_t smem = ll_slot_smem(p.E);
-    if (p.K <= 8)
-        ll_slot_kernel<8><<<p.num_tiles, kLLTile, smem, stream>>>(p);
-    else if (p.K <= 16)
-        ll_slot_kernel<16><<<p.num_tiles, kLLTile, smem, stream>>>(p);
-    else
-        ll_slot_kernel<32><<<p.num_tiles, kLLTile, smem, stream>>>(p);
-    return cudaGetLastError();
+    if (p.K <= 8) return launch_pdl(ll_slot_kernel<8>, dim3(p.num_tiles), dim3(kLLTile), smem, stream, p);
+    if (p.K <= 16) return launch_pdl(ll_slot_kernel<16>, dim3(p.num_tiles), dim3(kLLTile), smem, stream, p);
+    return launch_pdl(ll_slot_kernel<32>, dim3(p.num_tiles), dim3(kLLTile), smem, stream, p);
 }
 
 cudaError_t launch_ll_combine(const LLCombineParams& p, int num_sms, cudaStream_t stream) {
@@ -479,8 +474,7 @@ cudaError_t launch_ll_combine(const LLCombineParams& p, int num_sms, cudaStream_
     (void)num_sms;
     const long long blocks = (p.G * p.splits + kLLCombineWarps - 1) / kLLCombineWarps;
     // 4 x 16-byte vectors per lane per row, groups of 4 rows (measured best on B200)
-    ll_combine_kernel<4, 4><<<(unsigned)blocks, kLLCombineThreads, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(ll_combine_kernel<4, 4>, dim3((unsigned)blocks), dim3(kLLCombineThreads), 0, stream, p);
 }
 
 }  // namespace ep

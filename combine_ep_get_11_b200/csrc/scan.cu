@@ -62,7 +62,8 @@ scan_kernel(const ScanParams p) {
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int R = p.R;
-    pdl_launch_dependents();   // the dispatch kernel may start prefetching its rows
+    pdl_wait();                // everything before this kernel has completed ...
+    pdl_launch_dependents();   // ... so the dispatch kernel may start prefetching its rows
     if (tid == 0) {
         const unsigned long long tk = atomicAdd(p.ticket, 1ull);
         s_tile = (int)(tk % (unsigned long long)p.num_tiles);
@@ -259,8 +260,7 @@ scan_kernel(const ScanParams p) {
 
 cudaError_t launch_scan(const ScanParams& p, cudaStream_t stream) {
     if (p.num_tiles == 0) return cudaSuccess;
-    scan_kernel<<<p.num_tiles, kScanTile, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(scan_kernel, dim3(p.num_tiles), dim3(kScanTile), 0, stream, p);
 }
 
 }  // namespace ep
