@@ -90,6 +90,12 @@ __device__ __forceinline__ void ld_nc_v8(const void* p, uint4& a, uint4& b) {
                  : "l"(p));
 }
 
+// default (write-back) caching: the line may stay in L2 for the next reader
+__device__ __forceinline__ void st_v4(uint4* p, const uint4& v) {
+    asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
 __device__ __forceinline__ void st_stream_v4(uint4* p, const uint4& v) {
     asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
                  "r"(v.z), "r"(v.w)

@@ -132,6 +132,15 @@ __device__ __forceinline__ void ll_direct_tables(const DispatchParams& p, long l
 // warps fill 1.7 waves of the GPU, and single-warp blocks let the scheduler hand
 // out the second wave warp by warp (measured on B200, LL shape: step 90.3 vs
 // 91.2 us for 8-warp blocks; 2- and 4-warp blocks 91.2).
+// The bf16 packed copy writes with the default (write-back) policy, the others
+// with streaming (evict-first) stores: the packed rows are read again right
+// away (by the experts; in the benchmark's step by the low-latency combine),
+// and those still in L2 are read from there (measured on B200, LL shape: step
+// 84.9 vs 88.3 us, combine 41.5 vs 45.9 us; for the FP8 copy the default
+// policy measured 0.5 us slower, its codes not being read by the combine).
+#ifndef EP_LL_STORE_STREAM
+#define EP_LL_STORE_STREAM 0
+#endif
 #ifndef EP_LL_COPY_THREADS
 #define EP_LL_COPY_THREADS 32
 #endif
@@ -241,7 +250,12 @@ dispatch_kernel(const DispatchParams p) {
 #pragma unroll
             for (int u = 0; u < kVec; ++u) {
                 const int c = c0 + lane + 32 * u;
-                if (c < hi) st_stream_v4(dst + c, v[u]);
+                if (c < hi) {
+                    if (kMode == kModeLowLatency && !EP_LL_STORE_STREAM)
+                        st_v4(dst + c, v[u]);
+                    else
+                        st_stream_v4(dst + c, v[u]);
+                }
             }
         }
     }
