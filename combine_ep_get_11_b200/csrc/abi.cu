@@ -682,6 +682,7 @@ int ll_dispatch_impl(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint
     dp.ll_src_info = src_info;
     dp.ll_layout_range = layout_range;
     dp.ll_count = packed_recv_count;
+    dp.num_sms = c->num_sms;
     dp.rank_mask = c->rank_mask;
     dp.ll_capacity = c->ll_cap;
     dp.recv_x = packed_recv_x;

@@ -280,12 +280,11 @@ dispatch_kernel(const DispatchParams p) {
 // destination row and step, 512 contiguous bytes per warp instruction).  The
 // block scales of a pass (4 per step) are gathered one per lane, so each
 // destination row gets all of them from a single coalesced store.  A warp
-// holds up to kFp8Steps steps of its row (2: a 7168-wide row in seven column
-// slices, 64 registers, four blocks per SM; measured on B200 against 3, 4 and 7
-// steps per warp: 29.3 vs 30.0, 33.3 and 31.6 us on the low-latency shape),
-// loads them all before converting any, then streams the codes to every
-// destination.  Traffic per token: H*2 bytes read, fan-out * (H +
-// H/32) bytes written.
+// walks its row in passes of kFp8Steps steps (2: 64 registers, four blocks per
+// SM), loading a pass, converting it, then streaming its codes to every
+// destination while the next pass's loads are in flight.  The first pass is
+// converted before the warp waits for the slots (the row is an input of the
+// call).  Traffic per token: H*2 bytes read, fan-out * (H + H/32) bytes written.
 #ifndef EP_FP8_STEPS
 #define EP_FP8_STEPS 2
 #endif
@@ -300,18 +299,22 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
 }
 
 // One pass of the FP8 form: the steps [st0, min(st0 + kFp8Steps, s_hi)) of a
-// row (lane l: channels [16 l, 16 l + 16) of each step), loaded and turned into
-// E4M3 codes (codes[k] for step st0 + k) and the pass's block scales gathered
-// one per lane (block j of the pass -- step j / 4, block j % 4 of the step --
-// in lane j).
-__device__ __forceinline__ void fp8_convert_pass(const uint4* src, int st0, int s_hi, int nvec, int lane,
-                                                 uint4 (&codes)[kFp8Steps], float& my_scale) {
-    uint4 a[kFp8Steps], b[kFp8Steps];
+// row (lane l: channels [16 l, 16 l + 16) of each step): fp8_load_pass loads
+// them, fp8_convert_loaded turns them into E4M3 codes (codes[k] for step
+// st0 + k) and gathers the pass's block scales one per lane (block j of the
+// pass -- step j / 4, block j % 4 of the step -- in lane j).
+__device__ __forceinline__ void fp8_load_pass(const uint4* src, int st0, int s_hi, int nvec, int lane,
+                                              uint4 (&a)[kFp8Steps], uint4 (&b)[kFp8Steps]) {
 #pragma unroll
     for (int k = 0; k < kFp8Steps; ++k) {
         const int c = (st0 + k) * 64 + 2 * lane;
         if (st0 + k < s_hi && c < nvec) ld_nc_v8(src + c, a[k], b[k]);
     }
+}
+
+__device__ __forceinline__ void fp8_convert_loaded(const uint4 (&a)[kFp8Steps], const uint4 (&b)[kFp8Steps], int st0,
+                                                   int s_hi, int nvec, int lane, uint4 (&codes)[kFp8Steps],
+                                                   float& my_scale) {
     float scale[kFp8Steps];
 #pragma unroll
     for (int k = 0; k < kFp8Steps; ++k) {
@@ -374,9 +377,10 @@ ll_fp8_copy_kernel(const DispatchParams p) {
     if (lane == 0 && s_lo + kFp8Steps < s_hi)
         prefetch_l2(p.x + g * p.H + (long long)(s_lo + kFp8Steps) * 512,
                     (uint32_t)(min(nvec, s_hi * 64) - (s_lo + kFp8Steps) * 64) * 16u);
-    uint4 codes[kFp8Steps];
+    uint4 codes[kFp8Steps], a[kFp8Steps], b[kFp8Steps];
     float my_scale = 1.f;
-    fp8_convert_pass(src, s_lo, s_hi, nvec, lane, codes, my_scale);
+    fp8_load_pass(src, s_lo, s_hi, nvec, lane, a, b);
+    fp8_convert_loaded(a, b, s_lo, s_hi, nvec, lane, codes, my_scale);
 
     const long long row = packed_row(p, g, lane, part);
     if (p.ll_cnt != nullptr) ll_direct_tables(p, wid, lane);
@@ -387,7 +391,9 @@ ll_fp8_copy_kernel(const DispatchParams p) {
 
     const int nblk = p.H / kFp8Block;
     for (int st0 = s_lo; st0 < s_hi; st0 += kFp8Steps) {
-        if (st0 != s_lo) fp8_convert_pass(src, st0, s_hi, nvec, lane, codes, my_scale);
+        // the next pass's loads go out before this pass's stores (they hit L2)
+        const bool more = st0 + kFp8Steps < s_hi;
+        if (more) fp8_load_pass(src, st0 + kFp8Steps, s_hi, nvec, lane, a, b);
         const int blk0 = st0 * 4;
         const int nb = min(min(kFp8Steps, s_hi - st0) * 4, nblk - blk0);
         for (int i = 0; i < f; ++i) {
@@ -400,19 +406,30 @@ ll_fp8_copy_kernel(const DispatchParams p) {
             }
             if (lane < nb) __stcs(p.recv_scales + r * nblk + blk0 + lane, my_scale);
         }
+        if (more) fp8_convert_loaded(a, b, st0 + kFp8Steps, s_hi, nvec, lane, codes, my_scale);
     }
 }
 
 
 #ifndef EP_FP8_SPLITS
-#define EP_FP8_SPLITS 0
+#define EP_FP8_SPLITS -1
 #endif
 
 cudaError_t launch_ll_copy_fp8(DispatchParams p, cudaStream_t stream, bool after_scan) {
     const int nstep = (p.H / 8 + 63) / 64;
-    // column slices per row: the fewest with one pass each (EP_FP8_SPLITS 0), or a
-    // fixed count whose warps loop over several passes
-    p.splits = EP_FP8_SPLITS > 0 ? min(EP_FP8_SPLITS, nstep) : (nstep + kFp8Steps - 1) / kFp8Steps;
+    // Column slices per row.  Default: one warp per row streaming its passes (the
+    // next pass's loads ahead of this pass's stores: measured on B200, LL shape,
+    // 29.4 us vs 30.7 for seven one-pass warps per row, 31.7 for two), unless
+    // there are too few rows to give the GPU ~8 warps per SM.  EP_FP8_SPLITS 0:
+    // the fewest slices with one pass each; > 0: a fixed count.
+    if (EP_FP8_SPLITS > 0) {
+        p.splits = min(EP_FP8_SPLITS, nstep);
+    } else if (EP_FP8_SPLITS == 0) {
+        p.splits = (nstep + kFp8Steps - 1) / kFp8Steps;
+    } else {
+        const long long want = (long long)p.num_sms * 8;
+        p.splits = (int)min((long long)nstep, max(1LL, (want + p.G - 1) / p.G));
+    }
     const long long blocks = (p.G * p.splits + kFp8Threads / 32 - 1) / (kFp8Threads / 32);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)blocks);

@@ -99,6 +99,7 @@ struct DispatchParams {
     long long G;
     int R, E, L, T, K, H;
     int splits;                        // warps per token (column slices of the row)
+    int num_sms;                       // the device's SM count (launch geometry)
 };
 // after_scan: launched right behind the handle / slot scan kernel, which lets
 // it start early (programmatic dependent launch); only the normal and packed
