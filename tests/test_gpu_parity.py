@@ -417,6 +417,8 @@ def test_no_tokens(ep):
     recv_x, recv_idx, _, handle = buf.dispatch(x, topk)
     assert recv_x.shape[0] == 0
     assert handle.recv_rank_offset.cpu().tolist() == [0] * 5
+    ntr, _, _ = buf.get_dispatch_layout(topk)
+    assert ep.ep_get_num_recv(buf.ctx, ntr, 4) == (0, [0, 0, 0, 0])
     assert not handle.rank_prefix_matrix.any() and not handle.channel_prefix_matrix.any()
     out, _ = buf.combine(recv_x, handle)
     assert out.numel() == 0
@@ -429,6 +431,8 @@ def test_all_slots_masked(ep):
     buf = make_buffer(ep, w)
     topk = torch.full((2, 100, 2), -1, dtype=torch.int64, device="cuda")
     x = torch.randn((2, 100, 64), device="cuda").to(torch.bfloat16)
+    ntr, _, _ = buf.get_dispatch_layout(topk)
+    assert ep.ep_get_num_recv(buf.ctx, ntr, 2) == (0, [0, 0])
     recv_x, _, _, handle = buf.dispatch(x, topk)
     assert recv_x.shape[0] == 0
     assert (handle.send_head == -1).all()

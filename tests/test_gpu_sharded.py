@@ -150,6 +150,8 @@ def test_sharded_refusals_and_capacity(ep):
     with pytest.raises(EpError):
         ep.ep_dispatch(b.ctx, inp.x_d[:4], inp.topk_d[:4], None, None, None, None, handle,
                        torch.empty((8, w.hidden), dtype=torch.bfloat16, device="cuda"), None, None, 8)
+    with pytest.raises(EpError):          # a shard's receive count comes from ep_sharded_handle
+        ep.ep_get_num_recv(b.ctx, torch.zeros((4, 8), dtype=torch.int32, device="cuda"), 8)
     # receive buffers of 8 rows are far too small: rows past them are dropped and reported
     group.dispatch([inp.x_d[:4], inp.x_d[4:]], [inp.topk_d[:4], inp.topk_d[4:]])
     assert b.sync_status() == 3          # EP_ERR_CAPACITY
