@@ -650,6 +650,8 @@ int ll_dispatch_impl(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, uint
     if (!aligned16(x) || !aligned16(packed_recv_x) || !aligned16(packed_fp8))
         return fail(c, EP_ERR_ALIGNMENT, "row buffers must be 16-byte aligned");
     if (!aligned(topk_idx, 8) || !aligned(packed_scales, 4)) return fail(c, EP_ERR_ALIGNMENT, "array misaligned");
+    if (fp8 && !aligned(x, 32))   // the FP8 copy reads x in 32-byte vectors
+        return fail(c, EP_ERR_ALIGNMENT, "FP8 packing needs x 32-byte aligned");
     DeviceGuard guard(c->device);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     int rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));

@@ -55,7 +55,8 @@ typedef struct CUevent_st* ep_event_t;
 typedef enum ep_status {
     EP_OK = 0,
     EP_ERR_INVALID_ARG = 1,     /* bad argument or unsupported shape */
-    EP_ERR_ALIGNMENT = 2,       /* pointer not 16-byte aligned, or H*2 not a multiple of 16 */
+    EP_ERR_ALIGNMENT = 2,       /* pointer not 16-byte aligned (x of the FP8 packing: 32), or
+                                   H*2 not a multiple of 16 */
     EP_ERR_CAPACITY = 3,        /* a receive buffer is too small */
     EP_ERR_BAD_TOPK = 4,        /* an expert id outside [-1, E) */
     EP_ERR_HANDLE_MISMATCH = 5, /* handle arrays missing or not made for this context */
@@ -304,7 +305,8 @@ EP_API int ep_ll_dispatch(ep_ctx* ctx, const uint16_t* x, const int64_t* topk_id
  * an all-zero block has scale 1 and zero codes; x ~= value(code) * scale.
  *   packed_recv_x_fp8   u8  [R][L][R*Tmax][H]      out (16-byte aligned)
  *   packed_recv_scales  f32 [R][L][R*Tmax][H/128]  out
- * Requires H % 128 == 0 (EP_ERR_INVALID_ARG otherwise). */
+ * Requires H % 128 == 0 (EP_ERR_INVALID_ARG otherwise) and x 32-byte aligned
+ * (EP_ERR_ALIGNMENT otherwise: the copy reads x in 32-byte vectors). */
 EP_API int ep_ll_dispatch_fp8(ep_ctx* ctx, const uint16_t* x, const int64_t* topk_idx,
                               uint8_t* packed_recv_x_fp8, float* packed_recv_scales,
                               int32_t* packed_recv_count, int32_t* src_info, int32_t* layout_range,

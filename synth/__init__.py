@@ -44,6 +44,7 @@ _KIND_BIAS = 6
 _KIND_PERM = 7
 _KIND_REDUNDANCY = 8
 _KIND_CANCEL = 9
+_KIND_FP8 = 10
 
 
 @dataclasses.dataclass(frozen=True)
@@ -235,6 +236,46 @@ def cancel_rows_device(seed: int, num_rows: int, hidden: int, device="cuda", p_b
         small = torch.randn(shape, generator=gen, device=device)
         y[lo:hi] = torch.where(big, sign * float(2 ** big_exp), small)
     return y
+
+
+def fp8_block_rows(seed: int, num_rows: int, hidden: int, block: int = 128):
+    """[num_rows, H] numpy uint16 bf16 bit patterns whose 128-channel blocks take
+    the cases an FP8 block quantiser must get right, one kind per block in turn:
+    all +0; all -0; signed zeros with a single +1 or -1; a negative largest
+    magnitude among small positives; N(0,1) x 2^124; N(0,1) x 2^-100 (the
+    block's 448 / amax still finite); E4M3 rounding ties (amax 448, so the
+    products are the values themselves: halfway points between E4M3 neighbours,
+    normal and subnormal); N(0,1) with a few bf16 subnormals."""
+    rng = _rng(seed, 0, _KIND_FP8)
+    nb = hidden // block
+    v = np.zeros((num_rows, hidden), dtype=np.float32)
+    # halfway points between adjacent E4M3 values (exact in bf16: 5 significant bits)
+    ties = np.array([1.0625, 1.1875, 3.25 + 0.125, 2.0 ** -7 + 2.0 ** -10, 2.0 ** -9 * 1.5,
+                     2.0 ** -9 * 0.5, 240.0 + 8.0, 416.0 + 16.0], dtype=np.float32)
+    for r in range(num_rows):
+        for b in range(nb):
+            kind = (r * nb + b) % 8
+            blk = v[r, b * block:(b + 1) * block]
+            if kind == 1:
+                blk[:] = -0.0
+            elif kind == 2:
+                blk[:] = np.where(rng.random(block) < 0.5, -0.0, 0.0)
+                blk[rng.integers(block)] = 1.0 if rng.random() < 0.5 else -1.0
+            elif kind == 3:
+                blk[:] = rng.random(block) * 0.5
+                blk[rng.integers(block)] = -3.5
+            elif kind == 4:
+                blk[:] = rng.standard_normal(block) * 2.0 ** 124
+            elif kind == 5:
+                blk[:] = rng.standard_normal(block) * 2.0 ** -100
+            elif kind == 6:
+                blk[:] = rng.choice(ties, block) * np.where(rng.random(block) < 0.5, -1.0, 1.0)
+                blk[rng.integers(block)] = 448.0
+            elif kind == 7:
+                blk[:] = rng.standard_normal(block)
+                blk[rng.integers(block, size=4)] = 2.0 ** -130
+    import torch
+    return torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
 
 
 def bias_rows(w: Workload, which: int):

@@ -540,6 +540,37 @@ def test_low_latency_fp8(ep, w):
     buf.destroy()
 
 
+def test_low_latency_fp8_special_blocks(ep):
+    """FP8 packing of the blocks a block quantiser can get wrong -- all +0 / -0,
+    signed zeros around one +-1, a negative amax, N(0,1) x 2^124 and x 2^-100,
+    E4M3 rounding ties, bf16 subnormals -- codes and scales bit-exact.  Rows of
+    13 blocks: the last 512-channel step of a row is a quarter full."""
+    w = W["ll"].scaled(num_tokens=24, hidden=13 * 128)
+    inp = Inputs(w)
+    x_u16 = synth.fp8_block_rows(w.seed + 11, w.num_ranks * w.num_tokens, w.hidden)
+    x_d = to_bf16_tensor(x_u16.reshape(w.num_ranks, w.num_tokens, w.hidden)).cuda()
+    buf = make_buffer(ep, w)
+    (codes, scales), count, (src_info, _) = buf.low_latency_dispatch(x_d, inp.topk_d, use_fp8=True)
+    assert buf.sync_status() == 0
+    ll = oracle.ll_dispatch(x_u16.reshape(w.num_ranks, w.num_tokens, w.hidden), inp.topk,
+                            w.num_experts, w.tmax)
+    np.testing.assert_array_equal(count.cpu().numpy(), ll["packed_recv_count"])
+    c, sc = codes.cpu().numpy(), scales.cpu().numpy()
+    checked = 0
+    for d in range(w.num_ranks):
+        for j in range(w.local_experts):
+            n = int(ll["packed_recv_count"][d, j])
+            if n == 0:
+                continue
+            e_codes, e_scales = oracle.quantize_e4m3_blocks(ll["packed_recv_x"][d, j, :n], 128)
+            np.testing.assert_array_equal(c[d, j, :n], e_codes, err_msg=f"codes of expert ({d},{j})")
+            np.testing.assert_array_equal(sc[d, j, :n].view(np.uint32), e_scales.view(np.uint32),
+                                          err_msg=f"scales of expert ({d},{j})")
+            checked += n
+    assert checked > 0
+    buf.destroy()
+
+
 def test_low_latency_fp8_rejects_unaligned_hidden(ep):
     w = next(c for c in LL_CASES if c.name == "ll-odd")      # hidden 40: not a multiple of 128
     assert w.hidden % 128 != 0
@@ -548,6 +579,28 @@ def test_low_latency_fp8_rejects_unaligned_hidden(ep):
     with pytest.raises(ep.EpError) as e:
         buf.low_latency_dispatch(inp.x_d, inp.topk_d, use_fp8=True)
     assert e.value.status == 1
+    buf.destroy()
+
+
+def test_low_latency_fp8_rejects_x_off_32_bytes(ep):
+    """The FP8 copy reads x in 32-byte vectors: an x 16 bytes past a 32-byte boundary
+    is refused before any launch (EP_ERR_ALIGNMENT); the bf16 form takes it."""
+    w = W["ll"].scaled(num_tokens=8, hidden=256)
+    inp = Inputs(w)
+    buf = make_buffer(ep, w)
+    n = inp.x_d.numel()
+    base = torch.empty(n + 16, dtype=torch.bfloat16, device="cuda")
+    off = 8 if base.data_ptr() % 32 == 0 else 0          # elements: 16 bytes
+    x = base[off:off + n].view(inp.x_d.shape)
+    assert x.data_ptr() % 32 == 16
+    x.copy_(inp.x_d)
+    with pytest.raises(ep.EpError) as e:
+        buf.low_latency_dispatch(x, inp.topk_d, use_fp8=True)
+    assert e.value.status == 2
+    packed, count, _ = buf.low_latency_dispatch(x, inp.topk_d)
+    assert buf.sync_status() == 0
+    ll = oracle.ll_dispatch(inp.x_u16, inp.topk, w.num_experts, w.tmax)
+    np.testing.assert_array_equal(count.cpu().numpy(), ll["packed_recv_count"])
     buf.destroy()
 
 
