@@ -823,6 +823,9 @@ def run_ours(args):
     if rank == 0:
         if flush:
             l2 = f"L2 flushed between steps (read of {2 * L2_BYTES >> 20} MB, outside the timed pairs)"
+        elif w.name == "lb":
+            l2 = (f"inputs larger than L2 (expert weights {LB_EXPERTS * LB_EXPERT_ELEMS * 2 / 1e9:.2f} GB, "
+                  f"replicas {LB_REPLICAS * LB_EXPERT_ELEMS * 2 / 1e9:.2f} GB > 126 MB); no flush")
         else:
             l2 = (f"inputs larger than L2 (x {R*T*H*2/1e6:.0f} MB, received rows "
                   f"{path.N*H*2/1e9:.2f} GB > 126 MB); no flush")
@@ -830,14 +833,20 @@ def run_ours(args):
                 if sharded else ("one GPU" if world == 1 else f"{world} independent replicas"))
         cfg = dict(config_dict(w, l2_note=l2), mode=mode,
                    **({"ll_packing": "fp8 e4m3, 128-channel fp32 scales"} if args.fp8 else {}))
+        if w.name == "lb":   # weights, not tokens: the token fields only size the context
+            cfg = {"workload": f"lb: {LB_EXPERTS} experts of {LB_EXPERT_ELEMS} bf16 (DeepSeek-V3 expert size), "
+                               f"{LB_REPLICAS} redundant replicas: weight prefetch + gradient reduction",
+                   "experts": LB_EXPERTS, "elems_per_expert": LB_EXPERT_ELEMS, "replicas": LB_REPLICAS,
+                   "l2": l2, "mode": mode}
         line = {
             "metric": METRIC,
             "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_med / args.steps, 4),
             "higher_is_better": True, "scaling": "weak" if (world > 1 and not sharded) else "strong",
             "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded; DeepSeek-V3-shaped routing)",
-            "tokens_per_s": round(tokens_per_s, 1),
+            "data": ("synthetic (seeded N(0,1) expert weights and gradients, seeded redundancy mapping)"
+                     if w.name == "lb" else "synthetic (seeded; DeepSeek-V3-shaped routing)"),
+            "tokens_per_s": None if w.name == "lb" else round(tokens_per_s, 1),
             "us_per_step": round(ms_med / args.steps * 1e3, 2),
             "timing": {"repeats": args.repeats,
                        "us_per_step": {k: round(v / args.steps * 1e3, 2) for k, v in spread(per).items()},
