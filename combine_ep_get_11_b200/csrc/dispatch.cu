@@ -273,167 +273,142 @@ dispatch_kernel(const DispatchParams p) {
 // fp32 operation rounded to nearest even; E4M3 nearest even, saturating; an
 // all-zero block has scale 1 and zero codes).
 //
-// The row is walked in steps of 512 channels: in a step lane l holds channels
-// [16 l, 16 l + 16) (one 32-byte load), so the 8 lanes of an aligned group
-// hold one 128-channel block and find its amax with three xor shuffles.  A
-// lane turns its 16 values into 16 code bytes (one 16-byte store per
-// destination row and step, 512 contiguous bytes per warp instruction).  The
-// block scales of a pass (4 per step) are gathered one per lane, so each
-// destination row gets all of them from a single coalesced store.  A warp
-// walks its row in passes of kFp8Steps steps (2: 64 registers, four blocks per
-// SM), loading a pass, converting it, then streaming its codes to every
-// destination while the next pass's loads are in flight.  The first pass is
+// The row is cut into 512-channel steps and each warp (a one-warp block) takes
+// a slice of kFp8Steps steps -- seven warps per 7168-wide row -- and loads all
+// of it at once.  In a step lane l holds channels [16 l, 16 l + 16) (one 32-byte
+// load), so the 8 lanes of an aligned group hold one 128-channel block.  A
+// block's amax is a max over bf16 magnitudes, whose bit patterns order like the
+// values: a packed bf16x2 max-of-magnitudes over the lane's 8 words, then three
+// xor shuffles.  Lane j takes the amax of block j of the slice and computes its
+// scale and 448 / amax (one division pair per block); each step's lanes fetch
+// their block's multiplier back with a shuffle.  A lane turns its 16 values into
+// 16 code bytes (one 16-byte store per destination row and step, 512 B per warp
+// instruction), and lane j stores block j's scale, so a destination row gets
+// the slice's scales from one coalesced store.  The slice is loaded and
 // converted before the warp waits for the slots (the row is an input of the
 // call).  Traffic per token: H*2 bytes read, fan-out * (H + H/32) bytes written.
-#ifndef EP_FP8_STEPS
-#define EP_FP8_STEPS 2
-#endif
-constexpr int kFp8Steps = EP_FP8_STEPS;             // 512-channel steps held per warp per pass
+//
+// Measured on B200 (16 ranks, H 7168, top-8): 28.8 us at 128 tokens/rank
+// against 29.4 for warps walking whole rows in two-step passes, 51.8 against
+// 61.0 at 256 tokens/rank; one-step slices 34.1 us, 256-thread blocks the same
+// as one-warp blocks.
+constexpr int kFp8Steps = 2;                        // 512-channel steps per warp
 constexpr int kFp8LanesPerBlock = kFp8Block / 16;   // 8 lanes x 16 channels
+constexpr int kFp8MinBlocks = 32;                   // one-warp blocks per SM (64 registers)
 static_assert(kFp8LanesPerBlock == 8, "a block is 8 lanes of 16 channels");
+static_assert(kFp8Steps * 4 <= 32, "one lane per block of the slice");
 
-__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
-    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+// largest magnitude of each bf16 half of x and y (the result's sign bits are
+// not meaningful); a NaN half yields the other operand's half
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t x, uint32_t y) {
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(x), "r"(y));
+    return d;
+}
+
+// E4M3 codes of the 4 channels of bf16 pairs w0, w1, each multiplied by inv in
+// fp32 (rounded to nearest even) first
+__device__ __forceinline__ uint32_t e4m3x4_scaled(uint32_t w0, uint32_t w1, float inv) {
+    const float x0 = __fmul_rn(bf16_lo(w0), inv), x1 = __fmul_rn(bf16_hi(w0), inv);
+    const float x2 = __fmul_rn(bf16_lo(w1), inv), x3 = __fmul_rn(bf16_hi(w1), inv);
+    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(x2, x3), __NV_SATFINITE, __NV_E4M3);
     return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
-// One pass of the FP8 form: the steps [st0, min(st0 + kFp8Steps, s_hi)) of a
-// row (lane l: channels [16 l, 16 l + 16) of each step): fp8_load_pass loads
-// them, fp8_convert_loaded turns them into E4M3 codes (codes[k] for step
-// st0 + k) and gathers the pass's block scales one per lane (block j of the
-// pass -- step j / 4, block j % 4 of the step -- in lane j).
-__device__ __forceinline__ void fp8_load_pass(const uint4* src, int st0, int s_hi, int nvec, int lane,
-                                              uint4 (&a)[kFp8Steps], uint4 (&b)[kFp8Steps]) {
-#pragma unroll
-    for (int k = 0; k < kFp8Steps; ++k) {
-        const int c = (st0 + k) * 64 + 2 * lane;
-        if (st0 + k < s_hi && c < nvec) ld_nc_v8(src + c, a[k], b[k]);
-    }
-}
-
-__device__ __forceinline__ void fp8_convert_loaded(const uint4 (&a)[kFp8Steps], const uint4 (&b)[kFp8Steps], int st0,
-                                                   int s_hi, int nvec, int lane, uint4 (&codes)[kFp8Steps],
-                                                   float& my_scale) {
-    float scale[kFp8Steps];
-#pragma unroll
-    for (int k = 0; k < kFp8Steps; ++k) {
-        scale[k] = 1.f;
-        if (st0 + k >= s_hi) break;                       // warp-uniform
-        const bool on = (st0 + k) * 64 + 2 * lane < nvec;
-        float xs[16];
-        xs[0] = bf16_lo(a[k].x);  xs[1] = bf16_hi(a[k].x);  xs[2] = bf16_lo(a[k].y);  xs[3] = bf16_hi(a[k].y);
-        xs[4] = bf16_lo(a[k].z);  xs[5] = bf16_hi(a[k].z);  xs[6] = bf16_lo(a[k].w);  xs[7] = bf16_hi(a[k].w);
-        xs[8] = bf16_lo(b[k].x);  xs[9] = bf16_hi(b[k].x);  xs[10] = bf16_lo(b[k].y); xs[11] = bf16_hi(b[k].y);
-        xs[12] = bf16_lo(b[k].z); xs[13] = bf16_hi(b[k].z); xs[14] = bf16_lo(b[k].w); xs[15] = bf16_hi(b[k].w);
-        float amax = 0.f;
-        if (on) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(xs[i]));
-        }
-        amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
-        amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 4));
-        scale[k] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-        const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
-        uint32_t w[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            w[q] = e4m3x4(__fmul_rn(xs[4 * q], inv), __fmul_rn(xs[4 * q + 1], inv),
-                          __fmul_rn(xs[4 * q + 2], inv), __fmul_rn(xs[4 * q + 3], inv));
-        codes[k] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-#pragma unroll
-    for (int k = 0; k < kFp8Steps; ++k) {
-        const float v = __shfl_sync(kFullMask, scale[k], (lane & 3) * kFp8LanesPerBlock);
-        if ((lane >> 2) == k) my_scale = v;
-    }
-}
-
-#ifndef EP_FP8_THREADS
-#define EP_FP8_THREADS 256
-#endif
-constexpr int kFp8Threads = EP_FP8_THREADS;
-
-__global__ void __launch_bounds__(kFp8Threads, (kFp8Steps <= 3 ? 4 : 2) * (kDispatchThreads / kFp8Threads))
+__global__ void __launch_bounds__(32, kFp8MinBlocks)
 ll_fp8_copy_kernel(const DispatchParams p) {
-    constexpr int kWarps = kFp8Threads / 32;
-    __shared__ long long s_rows[kWarps][32];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const long long wid = (long long)blockIdx.x * kWarps + warp;
+    __shared__ long long s_rows[32];
+    const int lane = threadIdx.x;
+    const long long wid = blockIdx.x;
     const long long g = wid / p.splits;          // token
-    const int part = (int)(wid % p.splits);      // column slice of its row (whole steps)
-    if (g >= p.G) return;   // whole warp
+    const int part = (int)(wid % p.splits);      // slice of its row (whole steps)
+    if (g >= p.G) return;
 
     const int nvec = p.H / 8;                    // 16-byte vectors (8 channels) per row
     const int nstep = (nvec + 63) / 64;
-    const int per = (nstep + p.splits - 1) / p.splits;
+    const int per = (nstep + p.splits - 1) / p.splits;   // <= kFp8Steps (launch_ll_copy_fp8)
     const int s_lo = part * per, s_hi = min(nstep, s_lo + per);
     const uint4* src = reinterpret_cast<const uint4*>(p.x + g * p.H);
-    // Launched right behind the slot kernel: the row is an input of the call,
-    // never written by that kernel, so the first pass is loaded and converted
-    // while it runs; only the stores wait for the slots (packed_row).  Later
-    // passes (rows wider than kFp8Steps steps per warp) are pulled into L2.
-    if (lane == 0 && s_lo + kFp8Steps < s_hi)
-        prefetch_l2(p.x + g * p.H + (long long)(s_lo + kFp8Steps) * 512,
-                    (uint32_t)(min(nvec, s_hi * 64) - (s_lo + kFp8Steps) * 64) * 16u);
-    uint4 codes[kFp8Steps], a[kFp8Steps], b[kFp8Steps];
-    float my_scale = 1.f;
-    fp8_load_pass(src, s_lo, s_hi, nvec, lane, a, b);
-    fp8_convert_loaded(a, b, s_lo, s_hi, nvec, lane, codes, my_scale);
+    uint4 a[kFp8Steps], b[kFp8Steps];
+#pragma unroll
+    for (int k = 0; k < kFp8Steps; ++k) {
+        const int c = (s_lo + k) * 64 + 2 * lane;
+        if (s_lo + k < s_hi && c < nvec) ld_nc_v8(src + c, a[k], b[k]);
+    }
+    // block amax as a bf16 bit pattern; a half that is all NaN counts as 0, as a
+    // float max that skips NaN would have it
+    uint32_t amax_bits[kFp8Steps];
+#pragma unroll
+    for (int k = 0; k < kFp8Steps; ++k) {
+        uint32_t m = 0;
+        if (s_lo + k < s_hi && (s_lo + k) * 64 + 2 * lane < nvec) {
+            m = absmax_bf16x2(a[k].x, a[k].y);
+            m = absmax_bf16x2(m, a[k].z);
+            m = absmax_bf16x2(m, a[k].w);
+            m = absmax_bf16x2(m, b[k].x);
+            m = absmax_bf16x2(m, b[k].y);
+            m = absmax_bf16x2(m, b[k].z);
+            m = absmax_bf16x2(m, b[k].w);
+        }
+        uint32_t lo = m & 0x7fffu, hi = (m >> 16) & 0x7fffu;
+        lo = lo > 0x7f80u ? 0u : lo;
+        hi = hi > 0x7f80u ? 0u : hi;
+        uint32_t v = max(lo, hi);
+        v = max(v, __shfl_xor_sync(kFullMask, v, 1));
+        v = max(v, __shfl_xor_sync(kFullMask, v, 2));
+        v = max(v, __shfl_xor_sync(kFullMask, v, 4));
+        amax_bits[k] = v;
+    }
+    // lane j: block j of the slice (step j / 4, block j % 4 of the step)
+    uint32_t mine = 0;
+#pragma unroll
+    for (int k = 0; k < kFp8Steps; ++k) {
+        const uint32_t v = __shfl_sync(kFullMask, amax_bits[k], (lane & 3) * kFp8LanesPerBlock);
+        if ((lane >> 2) == k) mine = v;
+    }
+    const float amax = __uint_as_float(mine << 16);
+    const float my_scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    const float my_inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
+    uint4 codes[kFp8Steps];
+#pragma unroll
+    for (int k = 0; k < kFp8Steps; ++k) {
+        const float inv = __shfl_sync(kFullMask, my_inv, k * 4 + lane / kFp8LanesPerBlock);
+        codes[k] = make_uint4(e4m3x4_scaled(a[k].x, a[k].y, inv), e4m3x4_scaled(a[k].z, a[k].w, inv),
+                              e4m3x4_scaled(b[k].x, b[k].y, inv), e4m3x4_scaled(b[k].z, b[k].w, inv));
+    }
 
     const long long row = packed_row(p, g, lane, part);
     if (p.ll_cnt != nullptr) ll_direct_tables(p, wid, lane);
     const uint32_t m = __ballot_sync(kFullMask, row >= 0);
     const int f = __popc(m);
-    if (row >= 0) s_rows[warp][__popc(m & lanemask_lt())] = row;
+    if (row >= 0) s_rows[__popc(m & lanemask_lt())] = row;
     __syncwarp();
 
     const int nblk = p.H / kFp8Block;
-    for (int st0 = s_lo; st0 < s_hi; st0 += kFp8Steps) {
-        // the next pass's loads go out before this pass's stores (they hit L2)
-        const bool more = st0 + kFp8Steps < s_hi;
-        if (more) fp8_load_pass(src, st0 + kFp8Steps, s_hi, nvec, lane, a, b);
-        const int blk0 = st0 * 4;
-        const int nb = min(min(kFp8Steps, s_hi - st0) * 4, nblk - blk0);
-        for (int i = 0; i < f; ++i) {
-            const long long r = s_rows[warp][i];
-            uint8_t* dst = p.recv_fp8 + r * p.H;
+    const int nb = min((s_hi - s_lo) * 4, nblk - s_lo * 4);   // blocks of the slice
+    for (int i = 0; i < f; ++i) {
+        const long long r = s_rows[i];
+        uint8_t* dst = p.recv_fp8 + r * p.H;
 #pragma unroll
-            for (int k = 0; k < kFp8Steps; ++k) {
-                const int c = (st0 + k) * 64 + 2 * lane;
-                if (st0 + k < s_hi && c < nvec) st_stream_v4(reinterpret_cast<uint4*>(dst + (long long)c * 8), codes[k]);
-            }
-            if (lane < nb) __stcs(p.recv_scales + r * nblk + blk0 + lane, my_scale);
+        for (int k = 0; k < kFp8Steps; ++k) {
+            const int c = (s_lo + k) * 64 + 2 * lane;
+            if (s_lo + k < s_hi && c < nvec) st_stream_v4(reinterpret_cast<uint4*>(dst + (long long)c * 8), codes[k]);
         }
-        if (more) fp8_convert_loaded(a, b, st0 + kFp8Steps, s_hi, nvec, lane, codes, my_scale);
+        if (lane < nb) __stcs(p.recv_scales + r * nblk + s_lo * 4 + lane, my_scale);
     }
 }
 
-
-#ifndef EP_FP8_SPLITS
-#define EP_FP8_SPLITS -1
-#endif
-
 cudaError_t launch_ll_copy_fp8(DispatchParams p, cudaStream_t stream, bool after_scan) {
     const int nstep = (p.H / 8 + 63) / 64;
-    // Column slices per row.  Default: one warp per row streaming its passes (the
-    // next pass's loads ahead of this pass's stores: measured on B200, LL shape,
-    // 29.4 us vs 30.7 for seven one-pass warps per row, 31.7 for two), unless
-    // there are too few rows to give the GPU ~8 warps per SM.  EP_FP8_SPLITS 0:
-    // the fewest slices with one pass each; > 0: a fixed count.
-    if (EP_FP8_SPLITS > 0) {
-        p.splits = min(EP_FP8_SPLITS, nstep);
-    } else if (EP_FP8_SPLITS == 0) {
-        p.splits = (nstep + kFp8Steps - 1) / kFp8Steps;
-    } else {
-        const long long want = (long long)p.num_sms * 8;
-        p.splits = (int)min((long long)nstep, max(1LL, (want + p.G - 1) / p.G));
-    }
-    const long long blocks = (p.G * p.splits + kFp8Threads / 32 - 1) / (kFp8Threads / 32);
+    // slices of at most kFp8Steps steps; more (down to one step) when there are
+    // too few rows to give the GPU ~8 warps per SM
+    const long long want = (long long)p.num_sms * 8;
+    p.splits = (int)min((long long)nstep,
+                        max((long long)(nstep + kFp8Steps - 1) / kFp8Steps, (want + p.G - 1) / p.G));
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)blocks);
-    cfg.blockDim = dim3(kFp8Threads);
+    cfg.gridDim = dim3((unsigned)(p.G * p.splits));
+    cfg.blockDim = dim3(32);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
