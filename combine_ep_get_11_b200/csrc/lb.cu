@@ -121,18 +121,31 @@ lb_reduce_kernel(const LBParams p) {
     const uint4* __restrict__ red = reinterpret_cast<const uint4*>(p.redundant);
     const long long base = (long long)blockIdx.x * kLBChunk + tid;
     float acc[kLBVec][8];
-#pragma unroll
-    for (int u = 0; u < kLBVec; ++u) {
-        const long long c = base + (long long)u * kLBThreads;
-        const uint4 g0 = c < p.Wv ? g[c] : make_uint4(0, 0, 0, 0);
-        acc[u][0] = bf16_lo(g0.x); acc[u][1] = bf16_hi(g0.x); acc[u][2] = bf16_lo(g0.y); acc[u][3] = bf16_hi(g0.y);
-        acc[u][4] = bf16_lo(g0.z); acc[u][5] = bf16_hi(g0.z); acc[u][6] = bf16_lo(g0.w); acc[u][7] = bf16_hi(g0.w);
-    }
-    // each replica's chunk into L2 one replica ahead of its loads
     const long long chunk0 = (long long)blockIdx.x * kLBChunk;
     const uint32_t chunk_bytes = (uint32_t)(min(kLBChunk, p.Wv - chunk0) * 16);
-    if (tid == 0 && n > 0 && chunk0 < p.Wv) prefetch_l2(red + (long long)s_list[0] * p.Wv + chunk0, chunk_bytes);
-    for (int j = 0; j < n; ++j) {      // replicas in ascending order; all loads of one replica in flight
+    // The gradient chunk and the first replica's chunk are loaded together (measured
+    // on B200, 32 DSv3-sized experts with 8 replicas: 336 -> 308 us against loading
+    // the gradient chunk first); each later replica's chunk is pulled into L2 one
+    // replica ahead of its loads.
+    {
+        uint4 gv[kLBVec], v0[kLBVec];
+        const uint4* r0 = red + (long long)(n > 0 ? s_list[0] : 0) * p.Wv;
+        if (tid == 0 && n > 1 && chunk0 < p.Wv) prefetch_l2(red + (long long)s_list[1] * p.Wv + chunk0, chunk_bytes);
+#pragma unroll
+        for (int u = 0; u < kLBVec; ++u) {
+            const long long c = base + (long long)u * kLBThreads;
+            gv[u] = c < p.Wv ? ld_stream_v4(g + c) : make_uint4(0, 0, 0, 0);
+            if (n > 0 && c < p.Wv) v0[u] = ld_stream_v4(r0 + c);
+        }
+#pragma unroll
+        for (int u = 0; u < kLBVec; ++u) {
+            const uint4 g0 = gv[u];
+            acc[u][0] = bf16_lo(g0.x); acc[u][1] = bf16_hi(g0.x); acc[u][2] = bf16_lo(g0.y); acc[u][3] = bf16_hi(g0.y);
+            acc[u][4] = bf16_lo(g0.z); acc[u][5] = bf16_hi(g0.z); acc[u][6] = bf16_lo(g0.w); acc[u][7] = bf16_hi(g0.w);
+            if (n > 0 && base + (long long)u * kLBThreads < p.Wv) add8(acc[u], v0[u]);
+        }
+    }
+    for (int j = 1; j < n; ++j) {      // later replicas in ascending order; all loads of one replica in flight
         if (tid == 0 && j + 1 < n && chunk0 < p.Wv)
             prefetch_l2(red + (long long)s_list[j + 1] * p.Wv + chunk0, chunk_bytes);
         const uint4* r = red + (long long)s_list[j] * p.Wv;
