@@ -409,7 +409,7 @@ class Buffer:
 
     def check_handle(self, topk_idx, handle: Handle, stream=None) -> bool:
         """True if `handle` is the dispatch handle of this routing (the reuse
-        contract); synchronizes the stream to read the verdict."""
+        contract); synchronizes the stream to read the result."""
         hs = handle.c_struct()
         _check(load().ep_check_handle(self.ctx, _ptr(topk_idx), ctypes.byref(hs), _stream(stream), None),
                "ep_check_handle", self.ctx)
