@@ -286,8 +286,8 @@ def test_repeated_calls_on_one_context(ep):
     buf.destroy()
 
     # low-latency slots: the lookback scan (300 tokens per source) and the direct
-    # slots (200 tokens per source: per-source histogram, whose finish counter must
-    # be back at zero for every next call)
+    # slots (200 tokens per source: per-source counts and ranks rewritten by every
+    # call, with routings that change between calls)
     for base in (synth.Workload("ll-rep", 8, 64, 300, 64, 6, "uniform_masked", 84, mask_prob=0.1),
                  synth.Workload("ll-rep-direct", 8, 64, 200, 64, 6, "uniform_masked", 85, mask_prob=0.1)):
         buf = make_buffer(ep, base)
