@@ -141,8 +141,9 @@ typedef struct ep_handle_sizes {
  *
  * Concurrency: a context's workspace is shared by its calls -- the handle
  * scan's ticket counter and status words, the low-latency slot scan's counter,
- * status words and slot map (which ep_ll_combine reads as a hint), the rank
- * mask, the internal layout arrays and the error word.  Calls on one context
+ * status words and slot map (which ep_ll_combine reads as a hint), the direct
+ * slots' per-source counts and ranks, the rank mask, the internal layout arrays
+ * and the error word.  Calls on one context
  * must therefore be ordered with respect to each other on the GPU: issue them
  * on one stream (or order the streams with events), and from one host thread
  * at a time.  Two dispatches of one context running at once would interleave
