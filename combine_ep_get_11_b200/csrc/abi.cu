@@ -3,7 +3,7 @@
 // contract of every call.
 //
 // Entry point -> kernels (all on the caller's stream):
-//   ep_get_dispatch_layout : memset(histograms) + layout_kernel
+//   ep_get_dispatch_layout : layout_kernel (one CTA cluster per source; a memset only when T = 0)
 //   ep_dispatch            : [layout_kernel] + scan_kernel (call-tagged scan state, nothing to clear)
 //                            [+ one host read of N] + dispatch_kernel<normal> (programmatic
 //                            launch behind the scan)
@@ -420,10 +420,13 @@ int ep_get_dispatch_layout(ep_ctx* c, const int64_t* topk_idx, int32_t* num_toke
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     int rc = begin_call(c, s, reinterpret_cast<cudaEvent_t>(wait_event));
     if (rc != EP_OK) return rc;
-    rc = cuda_check(c, cudaMemsetAsync(num_tokens_per_rank, 0, sizeof(int) * c->Rl * c->R, s), "memset");
-    if (rc == EP_OK)
-        rc = cuda_check(c, cudaMemsetAsync(num_tokens_per_expert, 0, sizeof(int) * (size_t)c->Rl * c->E, s), "memset");
-    if (rc != EP_OK) return rc;
+    if (c->G == 0) {   // no tokens: zero counts, nothing to launch (the kernel writes every count otherwise)
+        rc = cuda_check(c, cudaMemsetAsync(num_tokens_per_rank, 0, sizeof(int) * c->Rl * c->R, s), "memset");
+        if (rc == EP_OK)
+            rc = cuda_check(c, cudaMemsetAsync(num_tokens_per_expert, 0, sizeof(int) * (size_t)c->Rl * c->E, s),
+                            "memset");
+        return rc;
+    }
     ep::LayoutParams p{topk_idx, is_token_in_rank, num_tokens_per_rank, num_tokens_per_expert, c->err,
                        c->R, c->E, c->L, c->T, c->K, c->Rl};
     return launch(c, kLayout, c->G > 0, s, [&] { return ep::launch_layout(p, s); });
@@ -474,9 +477,6 @@ int ep_dispatch(ep_ctx* c, const uint16_t* x, const int64_t* topk_idx, const flo
     // 1. layout
     const int* nte = num_tokens_per_expert;
     if (given == 0) {
-        rc = cuda_check(c, cudaMemsetAsync(c->ntr_ws, 0, sizeof(int) * c->R * c->R, s), "memset");
-        if (rc == EP_OK) rc = cuda_check(c, cudaMemsetAsync(c->nte_ws, 0, sizeof(int) * (size_t)c->R * c->E, s), "memset");
-        if (rc != EP_OK) return rc;
         ep::LayoutParams lp{topk_idx, h->is_token_in_rank, c->ntr_ws, c->nte_ws, c->err, c->R, c->E, c->L, c->T, c->K,
                             c->R};
         rc = launch(c, kLayout, c->G > 0, s, [&] { return ep::launch_layout(lp, s); });

@@ -25,7 +25,7 @@ struct LayoutParams {
     int R, E, L, T, K;
     int num_src;               // S: R, or the ranks of one shard
 };
-constexpr int kLayoutThreads = 256;
+constexpr int kLayoutThreads = 512;
 cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream);
 
 // -------------------------------------------------------------------- scan
