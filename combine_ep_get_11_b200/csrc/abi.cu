@@ -946,6 +946,7 @@ int ep_sharded_combine(ep_ctx* c, int num_shards, const uint16_t* const* y, cons
     p.out_x = out_x;
     p.out_topk_weights = out_topk_weights;
     p.sharded = true;
+    p.self_shard = c->shard;
     p.dst_offset = reinterpret_cast<const long long*>(dst_offset);
     p.ranks_per_shard = c->Rl;
     for (int w = 0; w < num_shards; ++w) {

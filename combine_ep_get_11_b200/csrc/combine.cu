@@ -18,10 +18,11 @@
 // every U-vector slab it issues the loads of a group of 4 rows at once
 // (4 x 4 vectors; measured best on B200 for fan-ins of 3.6 and 5.2), then adds
 // them in rank order, group after group.  Lane i also asks for the next column
-// slab of row i ahead of time (a bulk L2 prefetch), so the slab's loads hit L2.  Traffic per token: fan-out *
-// H*2 bytes read (streaming), H*2 written.  The sharded form reads rank d's
-// rows from the GPU hosting d (its own memory or a peer's, mapped into this
-// process): the return exchange happens inside the reduction.
+// slab of row i ahead of time (a bulk L2 prefetch), so the slab's loads hit L2.
+// Traffic per token: fan-out * H*2 bytes read (streaming), H*2 written.  The
+// sharded form reads rank d's rows from the GPU hosting d (its own memory or a
+// peer's, mapped into this process): the return exchange happens inside the
+// reduction; it prefetches only the rows in this GPU's own memory.
 
 #include "common.cuh"
 #include "kernels.h"
@@ -51,6 +52,7 @@ combine_kernel(const CombineParams p) {
     pdl_wait();   // (launched with programmatic serialization: reads nothing before this)
     __shared__ long long s_rows[kCombineWarps][32];             // row index, or (sharded) row address
     __shared__ long long s_wrow[kSharded ? kCombineWarps : 1][32];   // sharded: weight-row address
+    __shared__ bool s_local[kSharded ? kCombineWarps : 1][32];       // sharded: row in this GPU's memory
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const long long wid = (long long)blockIdx.x * kCombineWarps + warp;
     const long long g = wid / p.splits;          // token
@@ -76,6 +78,7 @@ combine_kernel(const CombineParams p) {
         if constexpr (kSharded) {   // rank d's rows are in shard d / ranks_per_shard (own or peer memory)
             const int shard = lane / p.ranks_per_shard;
             s_rows[warp][at] = (long long)reinterpret_cast<uintptr_t>(p.shard_y[shard] + row * p.H);
+            s_local[warp][at] = shard == p.self_shard;
             s_wrow[warp][at] =
                 p.shard_w[shard] ? (long long)reinterpret_cast<uintptr_t>(p.shard_w[shard] + row * p.K) : 0;
         } else {
@@ -92,10 +95,16 @@ combine_kernel(const CombineParams p) {
     const int nvec = p.H / 8;
     const int per = ((nvec + p.splits - 1) / p.splits + 31) / 32 * 32;
     const int lo = part * per, hi = min(nvec, lo + per);
-    // rows' next column slab into L2 ahead of its loads (lane i: row i of the token)
-    // (not in the sharded form, whose rows may live in a peer GPU's memory)
+    // rows' next column slab into L2 ahead of its loads (lane i: row i of the token);
+    // in the sharded form only rows in this GPU's own memory (never a peer's)
     const uint4* pf_row = nullptr;
-    if (!kSharded && lane < f) pf_row = reinterpret_cast<const uint4*>(p.y + s_rows[warp][lane] * p.H);
+    if (lane < f) {
+        if constexpr (kSharded) {
+            if (s_local[warp][lane]) pf_row = reinterpret_cast<const uint4*>(static_cast<uintptr_t>(s_rows[warp][lane]));
+        } else {
+            pf_row = reinterpret_cast<const uint4*>(p.y + s_rows[warp][lane] * p.H);
+        }
+    }
     if (pf_row != nullptr && lo < hi) prefetch_l2(pf_row + lo, (uint32_t)min(32 * U, hi - lo) * 16u);
     for (int c0 = lo; c0 < hi; c0 += 32 * U) {
         const int nxt = c0 + 32 * U;

@@ -124,6 +124,7 @@ struct CombineParams {
     int ranks_per_shard;
     const uint16_t* shard_y[kMaxShards];   // [y_rows][H] per shard
     const float* shard_w[kMaxShards];      // [y_rows][K] per shard, or null
+    int self_shard;                        // the tables' index of this GPU's own buffers
     int* err;
     long long G;
     int R, K, H;
