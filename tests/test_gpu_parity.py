@@ -37,6 +37,9 @@ CASES = [
     synth.Workload("E4096", 8, 4096, 50, 16, 8, "uniform", 86, num_channels=4),
     # a token may name an expert twice (counted twice per expert, once per rank)
     synth.Workload("repeats", 4, 16, 70, 64, 5, "uniform_repeats", 76, num_channels=3, mask_prob=0.1),
+    # more tokens per source than one layout cluster covers in one pass (8 CTAs of 512
+    # threads): each CTA walks two token blocks, the last one ragged
+    synth.Workload("layout-2pass", 3, 12, 4700, 32, 4, "uniform_masked", 75, num_channels=6, mask_prob=0.1),
 ]
 
 
