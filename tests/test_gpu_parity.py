@@ -229,6 +229,8 @@ LL_CASES = [
     synth.Workload("ll-T257", 4, 32, 257, 128, 8, "uniform_masked", 78, mask_prob=0.05),
     # repeated experts within a token (a token counts once per expert)
     synth.Workload("ll-rep-experts", 4, 8, 90, 128, 6, "uniform_repeats", 77, mask_prob=0.1),
+    # the widest row (FP8: 64 steps of 512 channels, 32 slices per token)
+    synth.Workload("ll-H32768", 2, 4, 12, 32768, 2, "uniform", 73),
 ]
 
 
